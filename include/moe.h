@@ -1,0 +1,215 @@
+/*
+ * moe.h -- C ABI of the B200 top-k routed mixture-of-experts FFN forward.
+ *
+ * The operation (sources are the pages on the MoE FFN, by title and item):
+ *   "ClikaRT::nn::QMoEWoQ", forward(): one fused MoE step, x [T, H] and the
+ *     caller-computed router_logits [T, E] -> [T, H] in x's dtype; an optional
+ *     shared_output [T, H] folds into the routed combine.
+ *   "Struct MoeSpec" fields: router_bias (added to every logit before scoring),
+ *     score (softmax over every logit, or each logit's own sigmoid),
+ *     selection_bias (choose by score + B[e], weigh by score alone), groups
+ *     (only the best groups' experts are eligible), renormalize (kept weights
+ *     rescaled to sum to one, the sum clamped at 2^-14 per sum_can_clamp),
+ *     scale (every kept weight times S, after renormalization), weigh_inputs
+ *     (the weight scales the expert's input instead of its output), biases
+ *     (gate, up and down bias rows per expert), act (the gated activation).
+ *   "MoE" graph-op page: fc1 [E, 2*inter, hidden] (fused gate||up, interleaved
+ *     or not per swiglu_fusion), fc2 [E, hidden, inter], activation_alpha,
+ *     activation_beta, swiglu_limit, k, normalize_routing_weights.
+ *   "Struct Moe": shared experts (shared_dff) with an optional sigmoid gate
+ *     sigma(x . g); groups scored by their two best experts.
+ *   "ClikaRT::nn::QMoEWoQ" class notes: weight-only quantized (MXFP4) expert
+ *     stacks decoded block by block inside the GEMM, never as a dense copy.
+ *
+ * Readings where the pages are silent: ties go to the lower expert (group)
+ * index; a group's score is the sum of its two best keys; the renormalizing sum
+ * is max(sum, 2^-14); SiLU gating is h = g*sigmoid(alpha*g) * (u + beta) with
+ * limit L > 0 applying g <- min(g, L), u <- clamp(u, -L, L); gate rows come
+ * first (concat) or at even indices (interleaved).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are caller-owned CUDA device memory of the current
+ *     device; the library allocates no device memory.  Row-major layouts.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  After validation every call is asynchronous on that stream,
+ *     performs no host synchronisation and may be captured in a CUDA graph.
+ *   - Validation is synchronous and happens before any launch; a rejected call
+ *     launches nothing, returns a nonzero moe_status and sets a thread-local
+ *     message readable with moe_last_error().
+ *   - Thread-safe and reentrant: no global mutable state except the
+ *     thread-local error message and a per-device cache of kernel attributes.
+ */
+#ifndef MOE_B200_MOE_H
+#define MOE_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---- */
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_NULL = 1,        /* a required pointer is NULL */
+  MOE_ERR_SHAPE = 2,       /* a size is out of range or inconsistent */
+  MOE_ERR_DTYPE = 3,       /* unknown dtype code or unsupported combination */
+  MOE_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned (TMA requirement) */
+  MOE_ERR_UNSUPPORTED = 5, /* valid per the pages but not built here */
+  MOE_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than moe_workspace_size() */
+  MOE_ERR_CUDA = 7,        /* a CUDA runtime call failed (message has the name) */
+  MOE_ERR_TIMEOUT = 8,     /* a device-side bounded wait gave up (moe_debug_status) */
+  MOE_ERR_ARG = 9          /* an option value is out of range */
+} moe_status;
+
+/* ---- dtype codes ---- */
+enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_MXFP4 = 2 };
+/* ---- scoring ("Struct MoeSpec" score) ---- */
+enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };
+/* ---- gated activation ("Struct MoeSpec" act; graph-op activation_type) ---- */
+enum { MOE_ACT_SILU = 0, MOE_ACT_GELU_ERF = 1, MOE_ACT_GELU_TANH = 2, MOE_ACT_RELU = 3,
+       MOE_ACT_IDENTITY = 4 };
+/* ---- fused gate||up layout (graph-op swiglu_fusion: 2 = concat, 1 = interleaved) ---- */
+enum { MOE_GU_CONCAT = 0, MOE_GU_INTERLEAVED = 1 };
+
+/*
+ * Problem sizes.  T tokens (a 3-D x [B, S, d] is passed as T = B*S), d hidden,
+ * F expert dff, E routed experts, k experts per token (1 <= k <= E), Fs the
+ * shared expert's dff (0 = no shared expert).
+ * Supported dtype combinations (act_dtype, w_dtype): (F32, F32), (BF16, BF16),
+ * (BF16, MXFP4).  logit_dtype is F32 or BF16.
+ */
+typedef struct {
+  int64_t T, d, F, E, k, Fs;
+  int32_t act_dtype;   /* x, y, expert biases, shared weights, shared gate, shared_output */
+  int32_t w_dtype;     /* routed expert stacks */
+  int32_t logit_dtype; /* router_logits and router_bias */
+  int32_t reserved;    /* must be 0 */
+} moe_shape;
+
+/* Routing and activation options.  Initialise with moe_options_init(). */
+typedef struct {
+  int32_t score;       /* MOE_SCORE_*                                   default SOFTMAX */
+  int32_t renormalize; /* 0/1; w <- w / max(sum_kept w, 2^-14)           default 0       */
+  float routed_scale;  /* S, applied after renormalization               default 1       */
+  int32_t n_group;     /* 0 = no group limit; else E % n_group == 0      default 0       */
+  int32_t topk_group;  /* groups kept; topk_group * E/n_group >= k        default 0       */
+  int32_t weigh_inputs;/* 0/1: weight scales the expert input (Llama 4)   default 0       */
+  int32_t act;         /* MOE_ACT_*                                      default SILU    */
+  float alpha;         /* SiLU slope: g * sigmoid(alpha * g)             default 1       */
+  float beta;          /* h = act(g) * (u + beta)                        default 0       */
+  float limit;         /* SiLU clamp; 0 = none                           default 0       */
+  int32_t gu_layout;   /* MOE_GU_*                                       default CONCAT  */
+  int32_t shared_gate; /* 0/1: shared expert output times sigmoid(x . g) default 0       */
+} moe_options;
+
+/*
+ * Tensors (device pointers; NULL = absent where marked optional).
+ *   x               [T, d] act_dtype
+ *   router_logits   [T, E] logit_dtype
+ *   router_bias     [E] logit_dtype, optional; l' = fp32(l) + fp32(bias)
+ *   selection_bias  [E] fp32, optional
+ *   gate_up         [E, 2F, d] w_dtype; MXFP4: e2m1 codes [E, 2F, d/2] u8, two per
+ *                   byte, the even k in the low nibble
+ *   gate_up_scales  MXFP4 only: e8m0 block scales [E, 2F, d/32] u8 (blocks of 32 along d)
+ *   gate_up_bias    [E, 2F] act_dtype, optional (same row order as gate_up)
+ *   down            [E, d, F] w_dtype; MXFP4: codes [E, d, F/2]
+ *   down_scales     MXFP4 only: [E, d, F/32]
+ *   down_bias       [E, d] act_dtype, optional
+ *   shared_gate_up  [2Fs, d] act_dtype (required when Fs > 0; same layout option)
+ *   shared_down     [d, Fs] act_dtype (required when Fs > 0)
+ *   shared_gate_vec [d] act_dtype (required when shared_gate)
+ *   shared_output   [T, d] act_dtype, optional; added to y
+ *   y               [T, d] act_dtype, output (must not alias any input)
+ *   topk_idx        [T, k] int32, optional output: chosen experts, best first
+ *   topk_w          [T, k] fp32, optional output: their weights
+ */
+typedef struct {
+  const void *x, *router_logits, *router_bias;
+  const float *selection_bias;
+  const void *gate_up;
+  const uint8_t *gate_up_scales;
+  const void *gate_up_bias;
+  const void *down;
+  const uint8_t *down_scales;
+  const void *down_bias;
+  const void *shared_gate_up, *shared_down, *shared_gate_vec, *shared_output;
+  void *y;
+  int32_t *topk_idx;
+  float *topk_w;
+} moe_tensors;
+
+/* Fill `opts` with the defaults listed in moe_options (the graph-op page's
+ * defaults: alpha 1, beta 0, limit 0, k from the shape; renormalize off). */
+MOE_API void moe_options_init(moe_options *opts);
+
+/*
+ * Bytes of device workspace moe_forward / moe_route need for this problem
+ * (0 if the arguments are invalid; moe_last_error() then says why).
+ * The workspace holds the routing, the expert-sorted row permutation and the
+ * intermediate activations; its contents do not persist between calls.
+ */
+MOE_API size_t moe_workspace_size(const moe_shape *shape, const moe_options *opts);
+
+/*
+ * The whole forward ("ClikaRT::nn::QMoEWoQ" forward(); "Struct MoeSpec"):
+ * route -> sort rows by expert -> gate_up GEMM + bias + gated activation ->
+ * down GEMM + bias + routing weight -> deterministic combine (+ shared expert,
+ * + shared_output) -> y [T, d] in act_dtype.
+ * workspace: device memory of at least moe_workspace_size() bytes, 256-byte
+ * aligned, used exclusively by this call until it completes on `stream`.
+ * Errors: MOE_ERR_NULL / SHAPE / DTYPE / ALIGN / ARG / UNSUPPORTED / WORKSPACE
+ * before any launch; MOE_ERR_CUDA if a launch fails.  T == 0 is a no-op.
+ * Results are bitwise reproducible run to run for the same inputs.
+ */
+MOE_API int moe_forward(const moe_shape *shape, const moe_options *opts, const moe_tensors *t,
+                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Routing only ("Struct MoeSpec" score, selection_bias, groups, renormalize,
+ * scale): writes t->topk_idx [T, k] and t->topk_w [T, k] (both required here).
+ * Only x (when shared_gate), router_logits, router_bias and selection_bias
+ * are read.  Same workspace rules as moe_forward.
+ */
+MOE_API int moe_route(const moe_shape *shape, const moe_options *opts, const moe_tensors *t,
+              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * moe_forward that also records caller-created CUDA events (cudaEvent_t passed
+ * as void*) on `stream` at the stage boundaries, for per-kernel timing:
+ *   events[0] before routing          events[4] after the gate_up GEMM
+ *   events[1] after routing           events[5] after the down GEMM
+ *   events[2] after sort/scan/scatter events[6] after the combine
+ *   events[3] after the row gather
+ * n_events <= MOE_STAGE_EVENTS; NULL entries are skipped.  Same results,
+ * errors and workspace rules as moe_forward.
+ */
+#define MOE_STAGE_EVENTS 7
+MOE_API int moe_forward_events(const moe_shape *shape, const moe_options *opts, const moe_tensors *t,
+                               void *workspace, size_t workspace_bytes, void *stream,
+                               void *const *events, int n_events);
+
+/* Message of the last failed call on this thread ("" if none). */
+MOE_API const char *moe_last_error(void);
+
+/*
+ * Synchronises `stream` and reads the device status word a previous call left
+ * in `workspace` (MOE_OK, or MOE_ERR_TIMEOUT if a bounded device wait gave up,
+ * MOE_ERR_SHAPE if a device-side consistency check failed).  Intended for tests.
+ */
+MOE_API int moe_debug_status(const void *workspace, void *stream);
+
+/* Library version string. */
+MOE_API const char *moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_MOE_H */

@@ -1,0 +1,393 @@
+// api.cu -- the C ABI of libmoe_b200: argument validation, the workspace plan,
+// and the launch sequence of one MoE forward on the caller's stream.
+//
+//   route -> histogram/scan/scatter -> gather -> gate_up GEMM -> down GEMM -> combine
+//
+// Validation follows the error conventions of "ClikaRT::nn::QMoEWoQ"
+// (forward raises on a shape/dtype mismatch; set_weights on a geometry mismatch
+// or a bias without its slot; a dtype it cannot serve is Unsupported), mapped
+// to status codes.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape_opts(const moe_shape* s, const moe_options* o) {
+  if (!s || !o) return fail(MOE_ERR_NULL, "shape and options must not be NULL");
+  if (s->reserved != 0) return fail(MOE_ERR_ARG, "moe_shape.reserved must be 0");
+  if (s->act_dtype != MOE_F32 && s->act_dtype != MOE_BF16)
+    return fail(MOE_ERR_DTYPE, "act_dtype %d must be MOE_F32 or MOE_BF16", s->act_dtype);
+  if (s->logit_dtype != MOE_F32 && s->logit_dtype != MOE_BF16)
+    return fail(MOE_ERR_DTYPE, "logit_dtype %d must be MOE_F32 or MOE_BF16", s->logit_dtype);
+  const bool combo = (s->act_dtype == MOE_F32 && s->w_dtype == MOE_F32) ||
+                     (s->act_dtype == MOE_BF16 && s->w_dtype == MOE_BF16) ||
+                     (s->act_dtype == MOE_BF16 && s->w_dtype == MOE_MXFP4);
+  if (!combo)
+    return fail(MOE_ERR_DTYPE, "(act_dtype, w_dtype) = (%d, %d): supported are (F32,F32), (BF16,BF16), (BF16,MXFP4)",
+                s->act_dtype, s->w_dtype);
+  if (s->T < 0 || s->d < 8 || s->F < 8 || s->E < 1 || s->Fs < 0)
+    return fail(MOE_ERR_SHAPE, "need T >= 0, d >= 8, F >= 8, E >= 1, Fs >= 0 (got T=%lld d=%lld F=%lld E=%lld Fs=%lld)",
+                (long long)s->T, (long long)s->d, (long long)s->F, (long long)s->E, (long long)s->Fs);
+  if (s->k < 1 || s->k > s->E) return fail(MOE_ERR_SHAPE, "need 1 <= k <= E (k=%lld E=%lld)", (long long)s->k, (long long)s->E);
+  if (s->E > kMaxE) return fail(MOE_ERR_UNSUPPORTED, "E=%lld exceeds %d experts", (long long)s->E, kMaxE);
+  if (s->k > kMaxK) return fail(MOE_ERR_UNSUPPORTED, "k=%lld exceeds %d", (long long)s->k, kMaxK);
+  if (s->d % 8 || s->F % 8 || s->Fs % 8)
+    return fail(MOE_ERR_SHAPE, "d, F and Fs must be multiples of 8 (16-byte rows)");
+  if (s->w_dtype == MOE_MXFP4 && (s->d % 32 || s->F % 32))
+    return fail(MOE_ERR_SHAPE, "MXFP4 experts need d and F multiples of 32 (block size)");
+  if (s->w_dtype == MOE_MXFP4) return fail(MOE_ERR_UNSUPPORTED, "MXFP4 expert weights are not built in this version");
+  const int64_t rows = s->T * s->k + (s->Fs > 0 ? s->T : 0);
+  if (s->T > (1ll << 26) || rows >= (1ll << 31))
+    return fail(MOE_ERR_SHAPE, "T*k + T must stay below 2^31 rows (T=%lld)", (long long)s->T);
+
+  if (o->score != MOE_SCORE_SOFTMAX && o->score != MOE_SCORE_SIGMOID) return fail(MOE_ERR_ARG, "score %d", o->score);
+  if (o->act < MOE_ACT_SILU || o->act > MOE_ACT_IDENTITY) return fail(MOE_ERR_ARG, "act %d", o->act);
+  if (o->gu_layout != MOE_GU_CONCAT && o->gu_layout != MOE_GU_INTERLEAVED)
+    return fail(MOE_ERR_ARG, "gu_layout %d", o->gu_layout);
+  if ((o->renormalize & ~1) || (o->weigh_inputs & ~1) || (o->shared_gate & ~1))
+    return fail(MOE_ERR_ARG, "renormalize, weigh_inputs and shared_gate are 0 or 1");
+  if (!std::isfinite(o->routed_scale) || !std::isfinite(o->alpha) || !std::isfinite(o->beta) ||
+      !std::isfinite(o->limit) || o->limit < 0.f)
+    return fail(MOE_ERR_ARG, "routed_scale, alpha, beta must be finite and limit finite and >= 0");
+  if (o->n_group < 0) return fail(MOE_ERR_ARG, "n_group %d < 0", o->n_group);
+  if (o->n_group > 0) {
+    if (o->n_group > kMaxGroups) return fail(MOE_ERR_UNSUPPORTED, "n_group %d exceeds %d", o->n_group, kMaxGroups);
+    if (s->E % o->n_group) return fail(MOE_ERR_ARG, "E=%lld is not a multiple of n_group=%d", (long long)s->E, o->n_group);
+    if (o->topk_group < 1 || o->topk_group > o->n_group)
+      return fail(MOE_ERR_ARG, "need 1 <= topk_group <= n_group (topk_group=%d)", o->topk_group);
+    if ((int64_t)o->topk_group * (s->E / o->n_group) < s->k)
+      return fail(MOE_ERR_ARG, "topk_group * E/n_group < k: not enough eligible experts");
+  }
+  if (o->shared_gate && s->Fs == 0) return fail(MOE_ERR_ARG, "shared_gate needs a shared expert (Fs > 0)");
+  return MOE_OK;
+}
+
+int check_tensors(const moe_shape* s, const moe_options* o, const moe_tensors* t, bool full) {
+  if (!t) return fail(MOE_ERR_NULL, "tensors must not be NULL");
+  if (s->T == 0) return MOE_OK;  // nothing is read or written (empty tensors may have NULL data)
+  if (!t->router_logits) return fail(MOE_ERR_NULL, "router_logits is required");
+  if (o->shared_gate && !t->shared_gate_vec) return fail(MOE_ERR_NULL, "shared_gate needs shared_gate_vec");
+  if (o->shared_gate && !t->x) return fail(MOE_ERR_NULL, "shared_gate needs x");
+  if (!full) {
+    if (!t->topk_idx || !t->topk_w) return fail(MOE_ERR_NULL, "moe_route needs topk_idx and topk_w");
+    return MOE_OK;
+  }
+  if (!t->x || !t->gate_up || !t->down || !t->y) return fail(MOE_ERR_NULL, "x, gate_up, down and y are required");
+  if (s->w_dtype == MOE_MXFP4 && (!t->gate_up_scales || !t->down_scales))
+    return fail(MOE_ERR_NULL, "MXFP4 experts need gate_up_scales and down_scales");
+  if (s->Fs > 0 && (!t->shared_gate_up || !t->shared_down))
+    return fail(MOE_ERR_NULL, "Fs > 0 needs shared_gate_up and shared_down");
+  const void* tma[] = {t->x, t->gate_up, t->down, t->y, t->shared_output, t->shared_gate_up, t->shared_down};
+  for (const void* p : tma)
+    if (p && !aligned16(p)) return fail(MOE_ERR_ALIGN, "x, weights, y and shared_output must be 16-byte aligned");
+  if (t->y == t->x || (t->shared_output && t->y == t->shared_output))
+    return fail(MOE_ERR_ARG, "y must not alias an input");
+  return MOE_OK;
+}
+
+int num_sms_of_current_device() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+template <typename P>
+P* at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws, size_t ws_bytes,
+        void* stream, bool full, void* const* events = nullptr, int n_events = 0) {
+  int rc = check_shape_opts(s, o);
+  if (rc) return rc;
+  rc = check_tensors(s, o, t, full);
+  if (rc) return rc;
+  Plan p;
+  const size_t need = make_plan(s, o, &p);
+  if (!ws || ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (n_events < 0 || n_events > MOE_STAGE_EVENTS) return fail(MOE_ERR_ARG, "n_events must be 0..%d", MOE_STAGE_EVENTS);
+  if (p.T == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) -> cudaError_t {
+    if (events && i < n_events && events[i]) return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
+    return cudaSuccess;
+  };
+  int* status = at<int>(ws, p.o_status);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  if ((e = mark(0)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+
+  RouteArgs ra{};
+  ra.logits = t->router_logits;
+  ra.router_bias = t->router_bias;
+  ra.sel_bias = t->selection_bias;
+  ra.T = (int)p.T;
+  ra.E = (int)p.E;
+  ra.k = (int)p.k;
+  ra.logit_bf16 = s->logit_dtype == MOE_BF16;
+  ra.score = o->score;
+  ra.renorm = o->renormalize;
+  ra.scale = o->routed_scale;
+  ra.n_group = o->n_group;
+  ra.topk_group = o->topk_group;
+  ra.idx = at<int32_t>(ws, p.o_idx);
+  ra.w = at<float>(ws, p.o_w);
+  ra.idx_user = t->topk_idx;
+  ra.w_user = t->topk_w;
+  ra.x = t->x;
+  ra.gvec = t->shared_gate_vec;
+  ra.d = (int)p.d;
+  ra.act_bf16 = s->act_dtype == MOE_BF16;
+  ra.sgate = (full && o->shared_gate) ? at<float>(ws, p.o_sgate) : nullptr;
+  if ((e = launch_route(ra, st)) != cudaSuccess) return cuda_fail(e, "route kernel");
+  if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if (!full) return MOE_OK;
+
+  SortArgs sa{};
+  sa.idx = ra.idx;
+  sa.w = ra.w;
+  sa.T = (int)p.T;
+  sa.k = (int)p.k;
+  sa.E = (int)p.E;
+  sa.NS = (int)p.NS;
+  sa.nchunks = (int)p.nchunks;
+  sa.R = (int)p.R;
+  sa.shared_rows = p.Fs > 0 ? (int)p.T : 0;
+  sa.hist = at<int32_t>(ws, p.o_hist);
+  sa.cnt = at<int32_t>(ws, p.o_cnt);
+  sa.off = at<int32_t>(ws, p.o_off);
+  sa.tile_gu = at<int32_t>(ws, p.o_tgu);
+  sa.tile_dn = at<int32_t>(ws, p.o_tdn);
+  sa.bm = p.bm;
+  sa.nt_gu_routed = p.nt_gu_routed;
+  sa.nt_gu_shared = p.nt_gu_shared;
+  sa.nt_dn_routed = p.nt_dn_routed;
+  sa.nt_dn_shared = p.nt_dn_shared;
+  sa.pos = at<int32_t>(ws, p.o_pos);
+  sa.perm = at<int32_t>(ws, p.o_perm);
+  sa.roww = at<float>(ws, p.o_roww);
+  sa.status = status;
+  if ((e = launch_sort(sa, st)) != cudaSuccess) return cuda_fail(e, "sort kernels");
+  if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+
+  GatherArgs ga{t->x, sa.perm, sa.roww, at<void>(ws, p.o_x), (int)p.R, (int)p.d, (int)p.T,
+                s->act_dtype == MOE_BF16, o->weigh_inputs, status};
+  if ((e = launch_gather(ga, st)) != cudaSuccess) return cuda_fail(e, "gather kernel");
+  if ((e = mark(3)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+
+  GemmCommon gc{};
+  gc.NS = (int)p.NS;
+  gc.E = (int)p.E;
+  gc.R = (int)p.R;
+  gc.T = (int)p.T;
+  gc.cnt = sa.cnt;
+  gc.off = sa.off;
+  gc.d = (int)p.d;
+  gc.F = (int)p.F;
+  gc.Fs = (int)p.Fs;
+  gc.Fmax = (int)p.Fmax;
+  gc.gu_layout = o->gu_layout;
+  gc.act = ActParams{o->act, o->alpha, o->beta, o->limit};
+  gc.weigh_inputs = o->weigh_inputs;
+  gc.status = status;
+  // Upper bound of the M tiles: every non-empty expert adds at most one partial tile.
+  const int64_t mt_routed = p.R / p.bm + std::min<int64_t>(p.E, p.R);
+  const int64_t mt_shared = p.Fs > 0 ? cdiv(p.T, p.bm) : 0;
+  GemmCommon gu = gc, dn = gc;
+  gu.tiles = sa.tile_gu;
+  gu.max_tiles = (int)(mt_routed * p.nt_gu_routed + mt_shared * p.nt_gu_shared);
+  dn.tiles = sa.tile_dn;
+  dn.max_tiles = (int)(mt_routed * p.nt_dn_routed + mt_shared * p.nt_dn_shared);
+
+  if (p.tc) {
+    TcArgs ta{};
+    ta.x = t->x;
+    ta.xg = at<void>(ws, p.o_x);
+    ta.gate_up = t->gate_up;
+    ta.gate_up_bias = t->gate_up_bias;
+    ta.down = t->down;
+    ta.down_bias = t->down_bias;
+    ta.sh_gate_up = t->shared_gate_up;
+    ta.sh_down = t->shared_down;
+    ta.roww = sa.roww;
+    ta.h = at<void>(ws, p.o_h);
+    ta.Y = at<void>(ws, p.o_y);
+    ta.num_sms = num_sms_of_current_device();
+    ta.c = gu;
+    if ((e = launch_tc_gate_up(ta, st)) != cudaSuccess) return cuda_fail(e, "tensor-core gate_up GEMM");
+    if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    ta.c = dn;
+    if ((e = launch_tc_down(ta, st)) != cudaSuccess) return cuda_fail(e, "tensor-core down GEMM");
+  } else {
+    SimtArgs sm{};
+    sm.x = (const float*)t->x;
+    sm.xg = at<float>(ws, p.o_x);
+    sm.gate_up = (const float*)t->gate_up;
+    sm.gate_up_bias = (const float*)t->gate_up_bias;
+    sm.down = (const float*)t->down;
+    sm.down_bias = (const float*)t->down_bias;
+    sm.sh_gate_up = (const float*)t->shared_gate_up;
+    sm.sh_down = (const float*)t->shared_down;
+    sm.roww = sa.roww;
+    sm.h = at<float>(ws, p.o_h);
+    sm.Y = at<float>(ws, p.o_y);
+    sm.c = gu;
+    if ((e = launch_simt_gate_up(sm, st)) != cudaSuccess) return cuda_fail(e, "SIMT gate_up GEMM");
+    if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    sm.c = dn;
+    if ((e = launch_simt_down(sm, st)) != cudaSuccess) return cuda_fail(e, "SIMT down GEMM");
+  }
+  if ((e = mark(5)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+
+  CombineArgs ca{at<void>(ws, p.o_y), sa.pos, ra.sgate, t->shared_output, t->y, (int)p.T, (int)p.d, (int)p.k,
+                 (int)p.R, p.Fs > 0, s->act_dtype == MOE_BF16, status};
+  if ((e = launch_combine(ca, st)) != cudaSuccess) return cuda_fail(e, "combine kernel");
+  if ((e = mark(6)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  return MOE_OK;
+}
+
+}  // namespace
+
+size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
+  (void)o;
+  p->T = s->T;
+  p->d = s->d;
+  p->F = s->F;
+  p->E = s->E;
+  p->k = s->k;
+  p->Fs = s->Fs;
+  p->R = s->T * s->k;
+  p->NS = s->E + (s->Fs > 0 ? 1 : 0);
+  p->rows = p->R + (s->Fs > 0 ? s->T : 0);
+  p->Fmax = s->Fs > s->F ? s->Fs : s->F;
+  p->nchunks = cdiv(s->T, kChunkTokens);
+  p->act_dtype = s->act_dtype;
+  p->w_dtype = s->w_dtype;
+  p->logit_dtype = s->logit_dtype;
+  p->tc = s->act_dtype == MOE_BF16;
+  if (p->tc) {
+    p->bm = kTcBM;
+    p->nt_gu_routed = (int)cdiv(s->F, kTcGuBN);
+    p->nt_gu_shared = (int)cdiv(s->Fs, kTcGuBN);
+    p->nt_dn_routed = p->nt_dn_shared = (int)cdiv(s->d, kTcDnBN);
+  } else {
+    p->bm = kSimtBM;
+    p->nt_gu_routed = (int)cdiv(s->F, 32);
+    p->nt_gu_shared = (int)cdiv(s->Fs, 32);
+    p->nt_dn_routed = p->nt_dn_shared = (int)cdiv(s->d, 64);
+  }
+  const size_t elt = p->tc ? 2 : 4;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = off;
+    off = align256(off + bytes);
+    return r;
+  };
+  p->o_status = take(256);
+  p->o_idx = take(p->R * 4);
+  p->o_w = take(p->R * 4);
+  p->o_hist = take(p->nchunks * p->E * 4);
+  p->o_cnt = take(p->NS * 4);
+  p->o_off = take((p->NS + 1) * 4);
+  p->o_tgu = take((p->NS + 1) * 4);
+  p->o_tdn = take((p->NS + 1) * 4);
+  p->o_pos = take(p->R * 4);
+  p->o_perm = take(p->R * 4);
+  p->o_roww = take(p->R * 4);
+  p->o_sgate = take(p->T * 4);
+  p->o_x = take(p->R * p->d * elt);
+  p->o_h = take(p->rows * p->Fmax * elt);
+  p->o_y = take(p->rows * p->d * elt);
+  p->total = off;
+  return off;
+}
+
+}  // namespace moe
+
+extern "C" {
+
+void moe_options_init(moe_options* o) {
+  if (!o) return;
+  std::memset(o, 0, sizeof *o);
+  o->score = MOE_SCORE_SOFTMAX;
+  o->routed_scale = 1.f;
+  o->act = MOE_ACT_SILU;
+  o->alpha = 1.f;
+  o->beta = 0.f;
+  o->limit = 0.f;
+  o->gu_layout = MOE_GU_CONCAT;
+}
+
+size_t moe_workspace_size(const moe_shape* s, const moe_options* o) {
+  if (moe::check_shape_opts(s, o) != MOE_OK) return 0;
+  moe::Plan p;
+  return moe::make_plan(s, o, &p);
+}
+
+int moe_forward(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws, size_t ws_bytes,
+                void* stream) {
+  return moe::run(s, o, t, ws, ws_bytes, stream, true);
+}
+
+int moe_route(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws, size_t ws_bytes,
+              void* stream) {
+  return moe::run(s, o, t, ws, ws_bytes, stream, false);
+}
+
+int moe_forward_events(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws, size_t ws_bytes,
+                       void* stream, void* const* events, int n_events) {
+  return moe::run(s, o, t, ws, ws_bytes, stream, true, events, n_events);
+}
+
+const char* moe_last_error(void) { return moe::g_err.c_str(); }
+
+int moe_debug_status(const void* ws, void* stream) {
+  if (!ws) return moe::fail(MOE_ERR_NULL, "workspace must not be NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return moe::cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  e = cudaMemcpy(&v, ws, sizeof v, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return moe::cuda_fail(e, "cudaMemcpy(status)");
+  return v;
+}
+
+const char* moe_version(void) { return "moe_b200 0.1"; }
+
+}  // extern "C"

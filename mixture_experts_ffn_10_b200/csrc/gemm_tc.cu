@@ -1,0 +1,418 @@
+// gemm_tc.cu -- bf16 grouped GEMMs on the sm_100a tensor cores (tcgen05 + TMA + TMEM).
+//
+//   gate_up (MODE 0): per expert e and row r of its segment,
+//       g = W_gate[e] . x_r + b_gate,  u = W_up[e] . x_r + b_up,  h = gated(g, u) -> bf16
+//   down    (MODE 1): Y_r = (W_down[e] . h_r + b_down) * w_r -> bf16
+// (graph-op page "MoE": fc1 [E, 2*inter, hidden] fused gate||up, swiglu_fusion
+// interleaved or not; fc2 [E, hidden, inter]; "Struct MoeSpec" biases, act,
+// weigh_inputs).  The shared expert is one more segment whose rows are x itself.
+//
+// One persistent CTA per SM walks the device-computed tile list (segment-major,
+// then N block, then M block, so CTAs working at the same time share a weight
+// tile through L2).  Warp roles:
+//   warp 0     TMA producer: A tile 128 x 64 and B tile 256 x 64 (bf16, 128-byte
+//              swizzle) per stage into a 4-stage shared-memory ring;
+//   warp 1     TMEM allocator and MMA issuer: tcgen05.mma M=128 N=256 K=16,
+//              fp32 accumulators in TMEM, two accumulator buffers of 256 columns;
+//   warps 2-5  epilogue: tcgen05.ld the accumulator rows, bias + activation (or
+//              bias x routing weight), bf16 stores; overlaps the next tile's MMAs.
+// For gate_up the B tile is 128 gate rows followed by the 128 matching up rows,
+// fetched through a 4-D tensor map view of the stack that hides the layout:
+// concat [E][2][F][d] or interleaved [E][F][2][d].  So accumulator column j
+// (< 128) is gate feature f0 + j and column 128 + j its up partner.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = kTcBM;            // 128
+constexpr int BK = 64;               // one 128-byte swizzle row of bf16
+constexpr int BNB = 256;             // B rows per tile
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BNB * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int ACC_COLS = 256;
+constexpr int TMEM_COLS = 2 * ACC_COLS;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 64 + kEpiWarps * 32;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BNB);
+
+struct TcParams {
+  GemmCommon c;
+  const uint16_t* gate_up_bias;  // [E, 2F] or null
+  const uint16_t* down_bias;     // [E, d] or null
+  const float* roww;             // [R]
+  uint16_t* out;                 // h [rows, Fmax] or Y [rows, d]
+};
+
+struct Tile {
+  int seg, m0, n_blk, rows;
+};
+
+__device__ __forceinline__ Tile decode_tile(const GemmCommon& c, int tile) {
+  int lo = 0, hi = c.NS - 1;  // last segment s with tiles[s] <= tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (c.tiles[mid] <= tile) lo = mid;
+    else hi = mid - 1;
+  }
+  Tile t;
+  t.seg = lo;
+  t.rows = c.cnt[lo];
+  const int mt = (t.rows + BM - 1) / BM;
+  const int local = tile - c.tiles[lo];
+  t.n_blk = local / mt;
+  t.m0 = (local % mt) * BM;
+  return t;
+}
+
+template <int MODE>
+__device__ __forceinline__ int k_extent(const GemmCommon& c, bool shared) {
+  return MODE == 0 ? c.d : (shared ? c.Fs : c.F);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
+                   const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBs,
+                   const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const GemmCommon& c = p.c;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; b++) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kEpiWarps * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmAs);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmBs);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = c.tiles[c.NS];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const Tile t = decode_tile(c, tile);
+        const bool sh = t.seg >= c.E;
+        const int nkb = (k_extent<MODE>(c, sh) + BK - 1) / BK;
+        const int arow = sh ? t.m0 : c.off[t.seg] + t.m0;
+        const CUtensorMap* mA = sh ? &tmAs : &tmA;
+        const CUtensorMap* mB = sh ? &tmBs : &tmB;
+        const int e = sh ? 0 : t.seg;
+        for (int kb = 0; kb < nkb; kb++, it++) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, c.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          tma_load_2d(mA, &full[s], sa, kb * BK, arow);
+          if (MODE == 0) {
+            const int f0 = t.n_blk * (BNB / 2);
+            if (c.gu_layout == MOE_GU_INTERLEAVED) {
+              tma_load_4d(mB, &full[s], sb, kb * BK, 0, f0, e);
+              tma_load_4d(mB, &full[s], sb + B_BYTES / 2, kb * BK, 1, f0, e);
+            } else {
+              tma_load_4d(mB, &full[s], sb, kb * BK, f0, 0, e);
+              tma_load_4d(mB, &full[s], sb + B_BYTES / 2, kb * BK, f0, 1, e);
+            }
+          } else {
+            tma_load_3d(mB, &full[s], sb, kb * BK, t.n_blk * BNB, e);
+          }
+        }
+      }
+      // every load issued into a stage has landed before the CTA may exit
+      for (uint32_t j = (it > (uint32_t)STAGES ? it - STAGES : 0); j < it; j++) {
+        const uint64_t t0 = global_timer();
+        while (!mbar_try_wait(&full[j % STAGES], (j / STAGES) & 1) && global_timer() - t0 < kTimeoutNs) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, tcount++) {
+        const Tile t = decode_tile(c, tile);
+        const bool sh = t.seg >= c.E;
+        const int nkb = (k_extent<MODE>(c, sh) + BK - 1) / BK;
+        const int acc = tcount & 1;
+        if (!mbar_wait(&tempty[acc], ((tcount >> 1) & 1) ^ 1, abort_flag, c.status)) break;
+        tc_fence_after();
+        const uint32_t dt = tmem_base + acc * ACC_COLS;
+        for (int kb = 0; kb < nkb; kb++, it++) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag, c.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
+          const uint64_t ad = sdesc_k_sw128(sa), bd = sdesc_k_sw128(sa + A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; kk++)
+            mma_bf16(dt, ad + 2 * kk, bd + 2 * kk, IDESC, (kb | kk) != 0 ? 1u : 0u);
+          mma_commit(&empty[s]);
+        }
+        if (ok) mma_commit(&tfull[acc]);
+      }
+      // all issued MMAs complete before TMEM is released
+      mma_commit(drain);
+      const uint64_t t0 = global_timer();
+      while (!mbar_try_wait(drain, 0) && global_timer() - t0 < kTimeoutNs) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // this warp may read TMEM lanes 32q .. 32q+31
+    const int r_in_tile = q * 32 + lane;
+    uint32_t tcount = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, tcount++) {
+      const Tile t = decode_tile(c, tile);
+      const bool sh = t.seg >= c.E;
+      const int acc = tcount & 1;
+      if (!mbar_wait(&tfull[acc], (tcount >> 1) & 1, abort_flag, c.status)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
+      const int row = t.m0 + r_in_tile;
+      const bool valid = row < t.rows;
+      const int64_t grow = (int64_t)c.off[t.seg] + row;
+      if (__any_sync(0xffffffffu, valid)) {
+        if (MODE == 0) {
+          const int F = sh ? c.Fs : c.F;
+          const int f0 = t.n_blk * (BNB / 2);
+          const uint16_t* bias = (!sh && p.gate_up_bias) ? p.gate_up_bias + (int64_t)t.seg * 2 * c.F : nullptr;
+          const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
+          uint16_t* out = p.out + grow * c.Fmax;
+#pragma unroll 1
+          for (int ch = 0; ch < (BNB / 2) / 16; ch++) {
+            uint32_t g[16], u[16];
+            tmem_ld16(tb + ch * 16, g);
+            tmem_ld16(tb + BNB / 2 + ch * 16, u);
+            tmem_ld_wait();
+            const int fb = f0 + ch * 16;
+            if (valid && fb < F) {
+              uint32_t packed[8];
+#pragma unroll
+              for (int i = 0; i < 16; i += 2) {
+                float hv[2];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; h2++) {
+                  const int f = fb + i + h2;
+                  float gv = __uint_as_float(g[i + h2]), uv = __uint_as_float(u[i + h2]);
+                  if (bias && f < F) {
+                    gv += bf16_to_f32(bias[il ? 2 * f : f]);
+                    uv += bf16_to_f32(bias[il ? 2 * f + 1 : F + f]);
+                  }
+                  hv[h2] = gated_act(c.act, gv, uv);
+                }
+                packed[i / 2] = pack_bf16x2(hv[0], hv[1]);
+              }
+              if (fb + 16 <= F) {
+                uint4* dst = reinterpret_cast<uint4*>(out + fb);
+                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+              } else {
+                for (int i = 0; i < 16 && fb + i < F; i++)
+                  out[fb + i] = (uint16_t)(packed[i / 2] >> (16 * (i & 1)));
+              }
+            }
+          }
+        } else {
+          const int N = c.d;
+          const int n0 = t.n_blk * BNB;
+          const uint16_t* bias = (!sh && p.down_bias) ? p.down_bias + (int64_t)t.seg * c.d : nullptr;
+          const float w = (sh || c.weigh_inputs || !valid) ? 1.f : p.roww[grow];
+          uint16_t* out = p.out + grow * c.d;
+#pragma unroll 1
+          for (int ch = 0; ch < BNB / 16; ch++) {
+            uint32_t v[16];
+            tmem_ld16(tb + ch * 16, v);
+            tmem_ld_wait();
+            const int ob = n0 + ch * 16;
+            if (valid && ob < N) {
+              uint32_t packed[8];
+#pragma unroll
+              for (int i = 0; i < 16; i += 2) {
+                float o[2];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; h2++) {
+                  float a = __uint_as_float(v[i + h2]);
+                  if (bias && ob + i + h2 < N) a += bf16_to_f32(bias[ob + i + h2]);
+                  o[h2] = a * w;
+                }
+                packed[i / 2] = pack_bf16x2(o[0], o[1]);
+              }
+              if (ob + 16 <= N) {
+                uint4* dst = reinterpret_cast<uint4*>(out + ob);
+                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+              } else {
+                for (int i = 0; i < 16 && ob + i < N; i++)
+                  out[ob + i] = (uint16_t)(packed[i / 2] >> (16 * (i & 1)));
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor map, dims[0] innermost (elements), strides in bytes for dims 1.., box dims.
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+              const uint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// rows x K matrix with row pitch `pitch` elements; box 64 x box_rows.
+bool map_rows(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint64_t pitch, uint32_t box_rows) {
+  const uint64_t dims[2] = {K, rows > 0 ? rows : 1};
+  const uint64_t strides[1] = {pitch * 2};
+  const uint32_t box[2] = {BK, box_rows};
+  return make_map(m, base, 2, dims, strides, box);
+}
+
+// Fused gate||up stack [E][2F][d] seen as 4-D so that one box is 128 gate (or up) rows.
+bool map_gate_up(CUtensorMap* m, const void* base, uint64_t d, uint64_t F, uint64_t E, int layout) {
+  if (layout == MOE_GU_INTERLEAVED) {  // [E][F][2][d]: dims {d, 2, F, E}
+    const uint64_t dims[4] = {d, 2, F, E};
+    const uint64_t strides[3] = {d * 2, 2 * d * 2, 2 * F * d * 2};
+    const uint32_t box[4] = {BK, 1, BNB / 2, 1};
+    return make_map(m, base, 4, dims, strides, box);
+  }
+  const uint64_t dims[4] = {d, F, 2, E};  // [E][2][F][d]
+  const uint64_t strides[3] = {d * 2, F * d * 2, 2 * F * d * 2};
+  const uint32_t box[4] = {BK, BNB / 2, 1, 1};
+  return make_map(m, base, 4, dims, strides, box);
+}
+
+// Down stack [E][d][F]: dims {F, d, E}, box 64 x 256 x 1.
+bool map_down(CUtensorMap* m, const void* base, uint64_t F, uint64_t d, uint64_t E) {
+  const uint64_t dims[3] = {F, d, E};
+  const uint64_t strides[2] = {F * 2, d * F * 2};
+  const uint32_t box[3] = {BK, BNB, 1};
+  return make_map(m, base, 3, dims, strides, box);
+}
+
+template <int MODE>
+cudaError_t launch(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMap& b, const CUtensorMap& bs,
+                   const TcParams& p, int num_sms, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int grid = p.c.max_tiles < num_sms ? p.c.max_tiles : num_sms;
+  tc_gemm_kernel<MODE><<<grid, kThreads, SMEM_BYTES, st>>>(a, as, b, bs, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc_gate_up(const TcArgs& a, cudaStream_t st) {
+  const GemmCommon& c = a.c;
+  if (c.max_tiles == 0) return cudaSuccess;
+  CUtensorMap mA, mAs, mB, mBs;
+  bool ok = map_rows(&mA, a.xg, c.d, c.R, c.d, BM);
+  ok = ok && map_gate_up(&mB, a.gate_up, c.d, c.F, c.E, c.gu_layout);
+  if (c.Fs > 0) {
+    ok = ok && map_rows(&mAs, a.x, c.d, c.T, c.d, BM);
+    ok = ok && map_gate_up(&mBs, a.sh_gate_up, c.d, c.Fs, 1, c.gu_layout);
+  } else {
+    mAs = mA;
+    mBs = mB;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  TcParams p{c, (const uint16_t*)a.gate_up_bias, nullptr, a.roww, (uint16_t*)a.h};
+  return launch<0>(mA, mAs, mB, mBs, p, a.num_sms, st);
+}
+
+cudaError_t launch_tc_down(const TcArgs& a, cudaStream_t st) {
+  const GemmCommon& c = a.c;
+  if (c.max_tiles == 0) return cudaSuccess;
+  CUtensorMap mA, mAs, mB, mBs;
+  bool ok = map_rows(&mA, a.h, c.F, c.R, c.Fmax, BM);
+  ok = ok && map_down(&mB, a.down, c.F, c.d, c.E);
+  if (c.Fs > 0) {
+    ok = ok && map_rows(&mAs, (const uint16_t*)a.h + (int64_t)c.R * c.Fmax, c.Fs, c.T, c.Fmax, BM);
+    ok = ok && map_down(&mBs, a.sh_down, c.Fs, c.d, 1);
+  } else {
+    mAs = mA;
+    mBs = mB;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  TcParams p{c, nullptr, (const uint16_t*)a.down_bias, a.roww, (uint16_t*)a.Y};
+  return launch<1>(mA, mAs, mB, mBs, p, a.num_sms, st);
+}
+
+}  // namespace moe

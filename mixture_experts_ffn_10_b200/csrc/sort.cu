@@ -1,0 +1,210 @@
+// sort.cu -- expert histogram, exclusive scans and the stable token permutation
+// that turns the routing [T, k] into expert-contiguous rows, and the gather of
+// the input rows into that order.
+//
+// Rows of expert e are offsets[e] .. offsets[e+1]-1, token-ascending; the shared
+// expert (when present) is segment E with one row per token at R + t.  The same
+// pass computes, per GEMM, the prefix of tiles per segment that the grouped
+// GEMMs walk on the device (no host round trip).
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+// Per-chunk expert histogram: hist[b][e] = #(t in chunk b, j) with idx[t][j] == e.
+__global__ void __launch_bounds__(256) hist_kernel(SortArgs a) {
+  extern __shared__ int32_t sh[];
+  const int b = blockIdx.x;
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) sh[e] = 0;
+  __syncthreads();
+  const int t0 = b * kChunkTokens;
+  const int t1 = min(a.T, t0 + kChunkTokens);
+  for (int n = threadIdx.x; n < (t1 - t0) * a.k; n += blockDim.x) {
+    const int e = a.idx[(int64_t)t0 * a.k + n];
+    if (e >= 0 && e < a.E) atomicAdd(&sh[e], 1);
+    else set_status(a.status, MOE_ERR_SHAPE);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) a.hist[(int64_t)b * a.E + e] = sh[e];
+}
+
+// Block-wide exclusive scan of up to 1024 * kItems values held in shared memory.
+template <int kItems>
+__device__ void block_exclusive_scan(int32_t* v, int n, int32_t* total, int32_t* warp_tot) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  int32_t loc[kItems];
+  int32_t run = 0;
+#pragma unroll
+  for (int i = 0; i < kItems; i++) {
+    const int idx = tid * kItems + i;
+    loc[i] = idx < n ? v[idx] : 0;
+    run += loc[i];
+  }
+  int32_t incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) warp_tot[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    const int nw = blockDim.x >> 5;
+    int32_t wv = lane < nw ? warp_tot[lane] : 0, wi = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t u = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += u;
+    }
+    if (lane < nw) warp_tot[lane] = wi - wv;
+    if (lane == nw - 1) *total = wi;
+  }
+  __syncthreads();
+  int32_t base = warp_tot[wid] + incl - run;
+#pragma unroll
+  for (int i = 0; i < kItems; i++) {
+    const int idx = tid * kItems + i;
+    if (idx < n) v[idx] = base;
+    base += loc[i];
+  }
+  __syncthreads();
+}
+
+// One block of 1024 threads: per-expert chunk prefixes, segment offsets, tile prefixes.
+__global__ void __launch_bounds__(1024) scan_kernel(SortArgs a) {
+  __shared__ int32_t cnt[kMaxE + 1];
+  __shared__ int32_t tg[kMaxE + 1];
+  __shared__ int32_t td[kMaxE + 1];
+  __shared__ int32_t warp_tot[32];
+  __shared__ int32_t tot;
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    int32_t run = 0;
+    for (int b = 0; b < a.nchunks; b++) {
+      int32_t* p = &a.hist[(int64_t)b * a.E + e];
+      const int32_t h = *p;
+      *p = run;
+      run += h;
+    }
+    cnt[e] = run;
+  }
+  if (threadIdx.x == 0 && a.NS > a.E) cnt[a.E] = a.shared_rows;
+  __syncthreads();
+  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) {
+    const bool sh = s >= a.E;
+    const int32_t mt = (cnt[s] + a.bm - 1) / a.bm;
+    a.cnt[s] = cnt[s];
+    tg[s] = mt * (sh ? a.nt_gu_shared : a.nt_gu_routed);
+    td[s] = mt * (sh ? a.nt_dn_shared : a.nt_dn_routed);
+  }
+  __syncthreads();
+  block_exclusive_scan<2>(cnt, a.NS, &tot, warp_tot);
+  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.off[s] = cnt[s];
+  if (threadIdx.x == 0) {
+    a.off[a.NS] = tot;
+    if (tot != a.R + a.shared_rows) set_status(a.status, MOE_ERR_SHAPE);
+  }
+  block_exclusive_scan<2>(tg, a.NS, &tot, warp_tot);
+  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.tile_gu[s] = tg[s];
+  if (threadIdx.x == 0) a.tile_gu[a.NS] = tot;
+  block_exclusive_scan<2>(td, a.NS, &tot, warp_tot);
+  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.tile_dn[s] = td[s];
+  if (threadIdx.x == 0) a.tile_dn[a.NS] = tot;
+}
+
+// One warp per chunk walks its (t, j) entries in order, so rows inside an expert
+// stay token-ascending: row = off[e] + (earlier chunks) + (earlier in this chunk).
+constexpr int kScatterWarps = 4;
+__global__ void __launch_bounds__(kScatterWarps * 32) scatter_kernel(SortArgs a) {
+  extern __shared__ int32_t run_all[];  // [kScatterWarps][E]
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int b = blockIdx.x * kScatterWarps + wid;
+  int32_t* run = run_all + wid * a.E;
+  for (int e = lane; e < a.E; e += 32) run[e] = 0;
+  __syncwarp();
+  if (b >= a.nchunks) return;
+  const int t0 = b * kChunkTokens;
+  const int n_ent = (min(a.T, t0 + kChunkTokens) - t0) * a.k;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < n_ent; base += 32) {
+    const int n = base + lane;
+    const bool valid = n < n_ent;
+    const int64_t slot = (int64_t)t0 * a.k + n;
+    int e = valid ? a.idx[slot] : -1;
+    if (e < 0 || e >= a.E) e = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lt_mask);
+    if (e >= 0) {
+      const int32_t row = a.off[e] + a.hist[(int64_t)b * a.E + e] + run[e] + rank;
+      if (row >= 0 && row < a.R) {
+        const int t = t0 + n / a.k;
+        a.pos[slot] = row;
+        a.perm[row] = t;
+        a.roww[row] = a.w[slot];
+      } else {
+        set_status(a.status, MOE_ERR_SHAPE);
+      }
+    }
+    __syncwarp();
+    if (e >= 0 && rank == 0) run[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// xg[r] = x[perm[r]] (times roww[r] for weigh-inputs), one warp per row, 16-byte vectors.
+template <typename T>
+__global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= a.R) return;
+  const int t = a.perm[r];
+  if (t < 0 || t >= a.T) {
+    if (lane == 0) set_status(a.status, MOE_ERR_SHAPE);
+    return;
+  }
+  constexpr int kVec = 16 / sizeof(T);
+  const int nv = a.d / kVec;
+  const uint4* src = reinterpret_cast<const uint4*>((const T*)a.x + (int64_t)t * a.d);
+  uint4* dst = reinterpret_cast<uint4*>((T*)a.xg + r * a.d);
+  if (!a.weigh_inputs) {
+    for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+    return;
+  }
+  const float w = a.roww[r];
+  for (int v = lane; v < nv; v += 32) {
+    uint4 q = __ldg(src + v);
+    if constexpr (sizeof(T) == 2) {
+      uint32_t* u = reinterpret_cast<uint32_t*>(&q);
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const float lo = bf16_to_f32(u[i] & 0xffff) * w, hi = bf16_to_f32(u[i] >> 16) * w;
+        u[i] = pack_bf16x2(lo, hi);
+      }
+    } else {
+      float* f = reinterpret_cast<float*>(&q);
+#pragma unroll
+      for (int i = 0; i < 4; i++) f[i] *= w;
+    }
+    dst[v] = q;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_sort(const SortArgs& a, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  hist_kernel<<<a.nchunks, 256, a.E * sizeof(int32_t), st>>>(a);
+  scan_kernel<<<1, 1024, 0, st>>>(a);
+  const int blocks = (a.nchunks + kScatterWarps - 1) / kScatterWarps;
+  scatter_kernel<<<blocks, kScatterWarps * 32, kScatterWarps * a.E * sizeof(int32_t), st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const GatherArgs& a, cudaStream_t st) {
+  if (a.R == 0) return cudaSuccess;
+  const int blocks = (a.R + 7) / 8;
+  if (a.bf16) gather_kernel<uint16_t><<<blocks, 256, 0, st>>>(a);
+  else gather_kernel<float><<<blocks, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,134 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+include/moe.h declares, and rejects bad arguments on the host before any launch."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from mixture_experts_ffn_10_b200 import build
+    build.build()
+    import mixture_experts_ffn_10_b200 as m
+    return m
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "moe.h")) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    assert _declared() == sorted(["moe_options_init", "moe_workspace_size", "moe_forward",
+                                  "moe_route", "moe_forward_events", "moe_last_error",
+                                  "moe_debug_status", "moe_version"])
+
+
+def test_library_exports_every_declared_symbol(moe):
+    lib = C.CDLL(moe.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(moe.EXPORTED) == set(_declared())
+
+
+def test_struct_sizes_match_the_header(moe):
+    # int64 x 6 + int32 x 4; 12 x 4-byte fields; 17 pointers
+    assert C.sizeof(moe.moe_shape) == 64
+    assert C.sizeof(moe.moe_options) == 48
+    assert C.sizeof(moe.moe_tensors) == 17 * 8
+
+
+def test_options_defaults(moe):
+    o = moe.moe_options_init()
+    assert (o.score, o.renormalize, o.routed_scale, o.n_group, o.weigh_inputs) == (0, 0, 1.0, 0, 0)
+    assert (o.act, o.alpha, o.beta, o.limit, o.gu_layout, o.shared_gate) == (0, 1.0, 0.0, 0.0, 0, 0)
+    assert moe.moe_version().startswith("moe_b200")
+
+
+def _valid(moe, **kw):
+    args = dict(T=64, d=128, F=256, E=8, k=2, Fs=0, act_dtype="bf16", w_dtype="bf16",
+                logit_dtype="bf16")
+    args.update(kw)
+    return moe.make_shape(**args)
+
+
+def test_workspace_size_grows_with_tokens(moe):
+    o = moe.make_options(renormalize=True)
+    a = moe.moe_workspace_size(_valid(moe, T=64), o)
+    b = moe.moe_workspace_size(_valid(moe, T=128), o)
+    assert 0 < a < b and a % 256 == 0
+    assert moe.moe_workspace_size(_valid(moe, k=9), o) == 0
+    assert "k" in moe.moe_last_error()
+
+
+FAKE = 1 << 20  # a non-NULL, 256-aligned address: validation never dereferences it
+
+
+def _tensors(moe, **kw):
+    t = moe.moe_tensors()
+    for n in ("x", "router_logits", "gate_up", "down", "y"):
+        setattr(t, n, FAKE)
+    for n, v in kw.items():
+        setattr(t, n, v)
+    return t
+
+
+@pytest.mark.parametrize("shape_kw,opt_kw,tens_kw,code", [
+    (dict(k=0), {}, {}, 2),
+    (dict(k=9), {}, {}, 2),
+    (dict(d=12), {}, {}, 2),
+    (dict(T=-1), {}, {}, 2),
+    (dict(act_dtype="f32", w_dtype="bf16"), {}, {}, 3),
+    (dict(E=2048, k=2), {}, {}, 5),
+    (dict(k=33, E=64), {}, {}, 5),
+    (dict(w_dtype="mxfp4", d=80), {}, {}, 2),
+    ({}, dict(n_group=3, topk_group=1), {}, 9),
+    ({}, dict(n_group=4, topk_group=5), {}, 9),
+    (dict(E=8, k=4), dict(n_group=4, topk_group=1), {}, 9),
+    ({}, dict(limit=-1.0), {}, 9),
+    ({}, dict(routed_scale=float("inf")), {}, 9),
+    ({}, dict(shared_gate=True), {}, 9),
+    ({}, {}, dict(x=None), 1),
+    ({}, {}, dict(router_logits=None), 1),
+    ({}, {}, dict(gate_up=FAKE + 8), 4),
+    ({}, {}, dict(y=FAKE), 9),
+    (dict(Fs=64), {}, {}, 1),
+])
+def test_validation_rejects_before_launch(moe, shape_kw, opt_kw, tens_kw, code):
+    s = _valid(moe, **shape_kw)
+    o = moe.make_options(**opt_kw)
+    t = _tensors(moe, **tens_kw)
+    if tens_kw.get("y") == FAKE:
+        t.x = FAKE  # y aliases x
+    rc = moe.moe_forward(s, o, t, FAKE, 1 << 40, None)
+    assert rc == code, (rc, moe.moe_last_error())
+    assert moe.moe_last_error()
+
+
+def test_workspace_checks(moe):
+    s, o = _valid(moe), moe.make_options()
+    t = _tensors(moe)
+    t.y = FAKE * 2
+    need = moe.moe_workspace_size(s, o)
+    assert moe.moe_forward(s, o, t, None, need, None) == moe.MOE_ERR_WORKSPACE
+    assert moe.moe_forward(s, o, t, FAKE, need - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert moe.moe_forward(s, o, t, FAKE + 16, need, None) == moe.MOE_ERR_WORKSPACE
+
+
+def test_zero_tokens_is_a_no_op(moe):
+    s, o = _valid(moe, T=0), moe.make_options()
+    t = _tensors(moe)
+    t.y = FAKE * 2
+    assert moe.moe_forward(s, o, t, FAKE, moe.moe_workspace_size(s, o), None) == moe.MOE_OK
+
+
+def test_route_needs_outputs(moe):
+    s, o = _valid(moe), moe.make_options()
+    t = moe.moe_tensors()
+    t.router_logits = FAKE
+    assert moe.moe_route(s, o, t, FAKE, 1 << 40, None) == moe.MOE_ERR_NULL

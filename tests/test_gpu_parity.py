@@ -1,0 +1,147 @@
+"""GPU parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Sizes span several GEMM tiles with ragged tails in every dimension; each case
+compares the routing bit-exactly and every output element within the
+tolerance (1e-4 relative for fp32, 2e-2 for bf16, of max|y|).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import CONFIGS, make_inputs, small
+
+from gpu_cases import check_output, check_routing, host, parity, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+MIX = small(CONFIGS["mixtral_bf16"], name="mixtral_small", T=300, d=256, F=384)
+DSK = small(CONFIGS["deepseek_bf16"], name="deepseek_small", T=130, d=256, F=128, E=64, k=8, Fs=192)
+GPT = small(CONFIGS["gptoss_mxfp4"], name="gptoss_bf16_small", w_dtype="bf16", T=200, d=320, F=352,
+            E=8, k=4)
+DEC = small(CONFIGS["decode_T1"], name="decode_small", d=512, F=256, E=32)
+TINY = CONFIGS["tiny_fp32"]
+
+CASES = {
+    "tiny_fp32": TINY,
+    "tiny_fp32_options": small(TINY, name="tiny_fp32_options", gu_layout="interleaved", expert_bias=True,
+                               router_bias=True, Fs=64, shared_gate=True, shared_output=True,
+                               score="sigmoid", selection_bias_std=0.1, routed_scale=1.5),
+    "mixtral_small": MIX,
+    "deepseek_small": DSK,
+    "gptoss_bf16_small": GPT,
+    "decode_small_T1": DEC,
+    "decode_small_T5": small(DEC, name="decode_small_T5", T=5),
+    "shared_gate_and_output": small(DSK, name="shared_gate_and_output", shared_gate=True, shared_output=True),
+    "weigh_inputs": small(MIX, name="weigh_inputs", weigh_inputs=True, renormalize=False),
+    "no_renorm": small(MIX, name="no_renorm", renormalize=False, E=16, k=4),
+    "gelu_erf": small(MIX, name="gelu_erf", act="gelu_erf", beta=0.5),
+    "gelu_tanh": small(MIX, name="gelu_tanh", act="gelu_tanh"),
+    "relu": small(MIX, name="relu", act="relu", expert_bias=True),
+    "identity": small(MIX, name="identity", act="identity", beta=0.25),
+    "f32_logits": small(MIX, name="f32_logits", logit_dtype="f32", router_bias=True),
+    "T1": small(MIX, name="T1", T=1),
+    "T3": small(MIX, name="T3", T=3),
+    "T17": small(MIX, name="T17", T=17),
+    "E5": small(MIX, name="E5", E=5, k=3),
+    "E37": small(MIX, name="E37", E=37, k=3, T=90),
+    "mostly_empty_experts": small(MIX, name="mostly_empty_experts", E=64, k=2, T=3),
+    "k1": small(MIX, name="k1", k=1),
+    "k_equals_E": small(MIX, name="k_equals_E", E=4, k=4, renormalize=False),
+    "ragged_d_F": small(MIX, name="ragged_d_F", d=72, F=40, Fs=24, T=70),
+    "many_experts": small(MIX, name="many_experts", E=256, k=8, T=64, d=128, F=64),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_forward_matches_oracle(name):
+    parity(CASES[name])
+
+
+@pytest.mark.parametrize("E,k,G,TG", [(64, 8, 8, 4), (32, 4, 4, 2), (40, 6, 5, 3), (256, 8, 8, 4)])
+def test_routing_with_ties_and_groups(E, k, G, TG):
+    # bf16 logits on a coarse grid produce many exact ties in keys and group scores
+    cfg = small(DSK, name="route_ties", E=E, k=k, n_group=G, topk_group=TG, T=257, score="sigmoid",
+                selection_bias_std=0.0)
+    g = torch.Generator().manual_seed(E + k)
+    logits = (torch.randint(-4, 5, (cfg.T, E), generator=g).float() * 0.25).to(torch.bfloat16)
+    import mixture_experts_ffn_10_b200 as m
+    inputs = {"logits": logits.cuda()}
+    idx, w = m.route(cfg, inputs)
+    torch.cuda.synchronize()
+    check_routing(oracle.Problem(cfg, host(inputs)), idx, w)
+
+
+@pytest.mark.parametrize("score,sel", [("softmax", 0.0), ("softmax", 0.05), ("sigmoid", 0.1)])
+def test_routing_scores(score, sel):
+    cfg = small(MIX, name="route_scores", E=96, k=6, T=513, score=score, selection_bias_std=sel,
+                router_bias=True, renormalize=score == "sigmoid", routed_scale=2.5)
+    import mixture_experts_ffn_10_b200 as m
+    inputs = make_inputs(cfg, "cuda", with_weights=False)
+    idx, w = m.route(cfg, inputs)
+    torch.cuda.synchronize()
+    check_routing(oracle.Problem(cfg, host(inputs)), idx, w)
+
+
+def test_renormalize_clamp_on_gpu():
+    cfg = small(MIX, name="clamp", E=16, k=4, T=4, score="sigmoid")
+    logits = torch.full((4, 16), -20.0).to(torch.bfloat16)
+    import mixture_experts_ffn_10_b200 as m
+    inputs = {"logits": logits.cuda()}
+    idx, w = m.route(cfg, inputs)
+    torch.cuda.synchronize()
+    check_routing(oracle.Problem(cfg, host(inputs)), idx, w)
+
+
+@pytest.mark.parametrize("cfg", [MIX, TINY], ids=["bf16", "f32"])
+def test_bitwise_deterministic(cfg):
+    inputs = make_inputs(cfg, "cuda")
+    y1, i1, w1 = run_gpu(cfg, inputs)
+    y2, i2, w2 = run_gpu(cfg, inputs)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(i1, i2) and torch.equal(w1, w2)
+
+
+@pytest.mark.parametrize("cfg", [MIX, small(TINY, Fs=32)], ids=["bf16", "f32"])
+def test_interleaved_layout_is_bitwise_equal_to_concat(cfg):
+    inputs = make_inputs(cfg, "cuda")
+    y1, _, _ = run_gpu(cfg, inputs)
+    F = cfg.F
+    perm = torch.stack([torch.arange(F), torch.arange(F) + F], 1).reshape(-1).cuda()
+    il = dict(inputs)
+    il["gate_up"] = inputs["gate_up"][:, perm].contiguous()
+    if cfg.Fs:
+        Fs = cfg.Fs
+        ps = torch.stack([torch.arange(Fs), torch.arange(Fs) + Fs], 1).reshape(-1).cuda()
+        il["shared_gate_up"] = inputs["shared_gate_up"][ps].contiguous()
+    y2, _, _ = run_gpu(small(cfg, gu_layout="interleaved"), il)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_routed_scale_on_gpu():
+    base = small(MIX, score="sigmoid", renormalize=True)
+    inputs = make_inputs(base, "cuda")
+    y1, _, _ = run_gpu(base, inputs)
+    y2, _, _ = run_gpu(small(base, routed_scale=2.0), inputs)
+    torch.cuda.synchronize()
+    # scaling by a power of two is exact through every bf16 rounding step
+    assert torch.equal(y2.float(), 2.0 * y1.float())
+
+
+def test_shared_output_added_on_gpu():
+    cfg = small(MIX, shared_output=True)
+    inputs = make_inputs(cfg, "cuda")
+    y, _, _ = run_gpu(cfg, inputs)
+    p = oracle.Problem(cfg, host(inputs))
+    torch.cuda.synchronize()
+    check_output(cfg, y, p.forward(), "shared_output")
+
+
+def test_zero_tokens_no_op_on_gpu():
+    import mixture_experts_ffn_10_b200 as m
+    cfg = small(MIX, T=0)
+    inputs = make_inputs(cfg, "cuda")
+    y = m.forward(cfg, inputs)
+    torch.cuda.synchronize()
+    assert y.shape == (0, cfg.d)
