@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Benchmark of the top-k routed MoE FFN forward on B200 (one JSON line on rank 0).
+
+A step is one moe_forward (route -> sort -> gather -> gate_up GEMM -> down GEMM
+-> combine) over one batch of T seeded synthetic tokens.  Default workload: the
+Mixtral-shaped bf16 prefill layer (T=4096, d=4096, F=14336, E=8, k=2).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl own|reference]
+
+Timing: W warm-up steps, then K steps timed on the device with CUDA events
+recorded by the library on the launching stream at every stage boundary; the
+L2 is flushed (512 MiB write) before every timed step, outside the events.
+Under torchrun each rank runs an independent replica (no collective on the data
+path); the reported time is the max over ranks and `value` counts the tokens of
+all ranks.  `e2e` repeats the measurement through the same C-ABI call with the
+step's x and logits copied from pinned host memory and y copied back inside the
+timed region.  `--impl reference` times the CPU oracle on the host cores
+instead (the only other place this script runs it).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s; achieved TFLOP/s or HBM GB/s as % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 8  # route, hist, scan, scatter, gather, gate_up GEMM, down GEMM, combine
+# ncu dram bytes (read + write) per launch of the dominant kernel, per workload, from the
+# profile summaries under profiles/ (None until captured for the current kernel version).
+NCU_TRAFFIC = {}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_name(cfg):
+    s = f"{cfg.name}: T={cfg.T} d={cfg.d} F={cfg.F} E={cfg.E} k={cfg.k}"
+    if cfg.Fs:
+        s += f" Fs={cfg.Fs}"
+    return s + f" {cfg.act_dtype}/{cfg.w_dtype} {cfg.score}"
+
+
+def config_dict(cfg, extra=None):
+    d = {"workload": workload_name(cfg), "T": cfg.T, "d": cfg.d, "F": cfg.F, "E": cfg.E, "k": cfg.k,
+         "Fs": cfg.Fs, "global_batch": cfg.T, "parallelism": "replicas",
+         "l2": "flushed (512 MiB write) before every timed step"}
+    if extra:
+        d.update(extra)
+    return d
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, phys_index):
+        self.idx = str(phys_index)
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "50"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        self.p.wait()
+        self.f.seek(0)
+        rows = [r.split(", ") for r in self.f.read().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        rows = [r for r in rows if len(r) >= 9 and r[0].strip() == self.idx]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = max(float(r[2]) for r in rows)
+        loaded = [r for r in rows if float(r[3]) > 300.0] or rows  # power draw marks load
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in loaded for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        sm_loaded = [float(r[1]) for r in loaded]
+        return {"sm_mhz": statistics.median(sm_loaded) if sm_loaded else None, "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
+                "sm_mhz_min": min(sm) if sm else None}
+
+
+def physical_gpu_index(local):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",")]
+        if local < len(ids) and ids[local].isdigit():
+            return int(ids[local])
+    return local
+
+
+# ---------------------------------------------------------------------------- oracle arm
+def oracle_sample(cfg, inputs_host, budget_s=15.0, max_tokens=None):
+    """Time the oracle on a bounded sample of tokens; returns (tokens/s, n, seconds, threads)."""
+    import numpy as np
+
+    import oracle
+    oracle.build()
+    p = oracle.Problem(cfg, inputs_host)
+    threads = oracle.max_threads()
+    t0 = time.perf_counter()
+    p.forward(np.array([0], dtype=np.int64), nthreads=1)
+    t1 = max(time.perf_counter() - t0, 1e-4)
+    n = int(max(threads, min(cfg.T, budget_s / t1 * threads)))
+    n = min(n, cfg.T if max_tokens is None else max_tokens)
+    toks = np.arange(n, dtype=np.int64) % cfg.T
+    t0 = time.perf_counter()
+    p.forward(toks, nthreads=threads)
+    dt = time.perf_counter() - t0
+    return n / dt, n, dt, threads
+
+
+def host_inputs(inputs):
+    return {k: (None if v is None else v.detach().cpu()) for k, v in inputs.items()}
+
+
+def run_reference(args, cfg):
+    import torch
+
+    from workloads import make_inputs
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    hin = host_inputs(make_inputs(cfg, dev))
+    import numpy as np
+
+    import oracle
+    oracle.build()
+    p = oracle.Problem(cfg, hin)
+    threads = oracle.max_threads()
+    # size one step's sample to about a second of the host's cores
+    t0 = time.perf_counter()
+    p.forward(np.array([0], dtype=np.int64), nthreads=1)
+    t1 = max(time.perf_counter() - t0, 1e-4)
+    n = int(min(cfg.T, max(threads, 1.0 / t1 * threads)))
+    toks = np.arange(n, dtype=np.int64)
+    for _ in range(args.warmup):
+        p.forward(toks, nthreads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        p.forward(toks, nthreads=threads)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
+           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+           "config": config_dict(cfg, {"sample_tokens_per_step": n}),
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                            "sample": f"{n} of {cfg.T} tokens per step, whole layer per token"},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------- own arm
+def stage_model(cfg, distinct):
+    """Algorithmic FLOPs and bytes per launch of each GEMM stage."""
+    ab = 2 if cfg.act_dtype == "bf16" else 4
+    R = cfg.T * cfg.k
+    if cfg.w_dtype == "mxfp4":
+        wbytes = lambda n: n / 2 + n / 32  # noqa: E731
+    else:
+        wbytes = lambda n: n * ab  # noqa: E731
+    gu_w = distinct * wbytes(2 * cfg.F * cfg.d) + 2 * cfg.Fs * cfg.d * ab
+    dn_w = distinct * wbytes(cfg.d * cfg.F) + cfg.d * cfg.Fs * ab
+    return {
+        "gate_up": {"flops": 2.0 * (R * cfg.d * 2 * cfg.F + cfg.T * cfg.d * 2 * cfg.Fs),
+                    "bytes": gu_w + (R + (cfg.T if cfg.Fs else 0)) * (cfg.d + cfg.F) * ab},
+        "down": {"flops": 2.0 * (R * cfg.d * cfg.F + cfg.T * cfg.d * cfg.Fs),
+                 "bytes": dn_w + (R + (cfg.T if cfg.Fs else 0)) * (cfg.F + cfg.d) * ab},
+    }
+
+
+def run_own(args, cfg):
+    import torch
+
+    import mixture_experts_ffn_10_b200 as moe
+    from workloads import algorithmic_bytes, flops, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    stream = torch.cuda.Stream()
+    inputs = make_inputs(cfg, "cuda")
+    shape, opts = moe.shape_of(cfg), moe.options_of(cfg)
+    ws = moe.Workspace(moe.moe_workspace_size(shape, opts))
+    y = torch.empty_like(inputs["x"])
+    idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    tens = moe.tensors_of(inputs, y, idx, None)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    nev = moe.MOE_STAGE_EVENTS
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    for row in events:
+        for ev in row:
+            ev.record(stream)  # creates the underlying cudaEvent_t
+    handles = [[ev.cuda_event for ev in row] for row in events]
+    sptr = stream.cuda_stream
+
+    def step(ev=None):
+        if ev is None:
+            rc = moe.moe_forward(shape, opts, tens, ws.ptr, ws.nbytes, sptr)
+        else:
+            rc = moe.moe_forward_events(shape, opts, tens, ws.ptr, ws.nbytes, sptr, ev)
+        if rc != 0:
+            raise moe.MoeError(rc, moe.moe_last_error())
+
+    sampler = ClockSampler(physical_gpu_index(local))
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
+    torch.cuda.synchronize()
+    status = moe.moe_debug_status(ws.ptr, sptr)
+    if status != 0:
+        raise RuntimeError(f"device status {moe.STATUS_NAMES.get(status, status)}")
+
+    # ------------------------------------------------------------ device-timed steps
+    barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.zero_()
+            step(handles[i])
+    torch.cuda.synchronize()
+    barrier()
+    stage_ms = [0.0] * (nev - 1)
+    total_ms = 0.0
+    for row in events:
+        total_ms += row[0].elapsed_time(row[-1])
+        for s in range(nev - 1):
+            stage_ms[s] += row[s].elapsed_time(row[s + 1])
+    stage_ms = [v / args.steps for v in stage_ms]
+    total_ms = max_over_ranks(total_ms)
+    ms_per_step = total_ms / args.steps
+    value = world * cfg.T * args.steps / (total_ms / 1e3)
+
+    # ------------------------------------------------------------ end to end (host buffers)
+    x_h = inputs["x"].cpu().pin_memory()
+    l_h = inputs["logits"].cpu().pin_memory()
+    y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    x_d, l_d = inputs["x"], inputs["logits"]
+    e2e_steps = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            x_d.copy_(x_h, non_blocking=True)
+            l_d.copy_(l_h, non_blocking=True)
+            step()
+            y_h.copy_(y, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = world * cfg.T * e2e_steps / (e2e_ms / 1e3)
+    clocks = sampler.stop()
+
+    # ------------------------------------------------------------ roofline of the dominant kernel
+    distinct = int(torch.unique(idx).numel())
+    pk, pk_src = peaks()
+    model = stage_model(cfg, distinct)
+    names = list(moe.STAGES)
+    gemm_ms = {"gate_up": stage_ms[names.index("gate_up")], "down": stage_ms[names.index("down")]}
+    dom = max(gemm_ms, key=gemm_ms.get)
+    t_dom = gemm_ms[dom] / 1e3
+    m = model[dom]
+    t_tc, t_hbm = m["flops"] / (pk["bf16_tflops"] * 1e12), m["bytes"] / (pk["hbm_gbs"] * 1e9)
+    if t_tc >= t_hbm:
+        achieved, peak, unit, bound = m["flops"] / t_dom / 1e12, pk["bf16_tflops"], "TFLOP/s", "tensor"
+    else:
+        achieved, peak, unit, bound = m["bytes"] / t_dom / 1e9, pk["hbm_gbs"], "GB/s", "hbm"
+    roofline = {"bound": bound, "kernel": f"{dom} grouped GEMM", "achieved": achieved, "peak": peak,
+                "unit": unit, "frac": achieved / peak, "peak_source": f"{pk_src} (burst)",
+                "traffic": NCU_TRAFFIC.get((cfg.name, dom)),
+                "algorithmic_per_launch": m["flops"] if bound == "tensor" else m["bytes"]}
+    layer_flops = flops(cfg)
+    layer_bytes = algorithmic_bytes(cfg, distinct)
+    t_step = ms_per_step / 1e3
+    layer = {"tflops": layer_flops / t_step / 1e12, "tensor_frac": layer_flops / t_step / 1e12 / pk["bf16_tflops"],
+             "hbm_gbs": layer_bytes / t_step / 1e9, "hbm_frac": layer_bytes / t_step / 1e9 / pk["hbm_gbs"],
+             "tensor_frac_vendor_2250": layer_flops / t_step / 1e12 / 2250.0,
+             "hbm_frac_vendor_8000": layer_bytes / t_step / 1e9 / 8000.0,
+             "distinct_experts": distinct, "flops": layer_flops, "bytes": layer_bytes}
+
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": cfg.act_dtype if cfg.w_dtype != "mxfp4" else "bf16 (mxfp4 weights)",
+           "data": "synthetic (seeded; random-init weights)",
+           "config": config_dict(cfg, {"parallelism": f"replicas x{world}"}),
+           "roofline": roofline, "layer": layer,
+           "stage_ms": dict(zip(names, stage_ms)),
+           "e2e": {"value": e2e_value, "unit": "tokens/s",
+                   "h2d_bytes_per_step": x_h.numel() * x_h.element_size() + l_h.numel() * l_h.element_size(),
+                   "d2h_bytes_per_step": y_h.numel() * y_h.element_size()},
+           "gpu_launches": KERNELS_PER_STEP * args.steps,
+           "clocks": clocks}
+
+    # ------------------------------------------------------------ CPU baseline (rank 0, N=1)
+    if world == 1 and not args.no_cpu_baseline:
+        hin = host_inputs(inputs)
+        v, n, dt, threads = oracle_sample(cfg, hin, budget_s=args.cpu_budget)
+        out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                               "sample": f"{n} of {cfg.T} tokens (whole layer per token), {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--config", default="mixtral_bf16")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle wall time")
+    ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
+                    help="override a workload field (profiling / sweeps), e.g. --set T=1024")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    from workloads import CONFIGS, small
+    cfg = CONFIGS[args.config]
+    for kv in args.set:
+        k, v = kv.split("=", 1)
+        cur = getattr(cfg, k)
+        cfg = small(cfg, **{k: type(cur)(v) if not isinstance(cur, bool) else v in ("1", "true", "True")})
+    if args.set:
+        cfg = small(cfg, name=cfg.name + "[" + ",".join(args.set) + "]")
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_own(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
