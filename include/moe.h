@@ -196,6 +196,27 @@ MOE_API int moe_forward_events(const moe_shape *shape, const moe_options *opts, 
                                void *workspace, size_t workspace_bytes, void *stream,
                                void *const *events, int n_events);
 
+/*
+ * moe_forward without a caller workspace, for callers that cannot allocate
+ * device memory (a plugin inside a runtime that owns all device memory and
+ * offers no allocator; a request path that must not call cudaMalloc).  It is
+ * not an operation of the pages (they have no counterpart): the forward is
+ * the same as moe_forward, run on a static scratch array of
+ * MOE_NOALLOC_WORKSPACE_BYTES inside the library, held by every GPU that
+ * loads the library until the process exits.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Problems whose moe_workspace_size() exceeds the array are rejected with
+ *     MOE_ERR_WORKSPACE (nothing is launched); use moe_forward for them.
+ *   - All calls share the array: calls that overlap on the GPU (other streams
+ *     or threads) race and give wrong results; serialise them.
+ *   - It calls no cudaMalloc or cudaFree.  Other errors as moe_forward.
+ */
+#define MOE_NOALLOC_WORKSPACE_BYTES (64u << 20)
+MOE_API int moe_forward_noalloc(const moe_shape *shape, const moe_options *opts, const moe_tensors *t,
+                                void *stream);
+
 /* Message of the last failed call on this thread ("" if none). */
 MOE_API const char *moe_last_error(void);
 

@@ -72,6 +72,9 @@ _lib.moe_forward_events.argtypes = [_P(moe_shape), _P(moe_options), _P(moe_tenso
                                    C.c_size_t, C.c_void_p, _P(C.c_void_p), C.c_int]
 _lib.moe_forward_events.restype = C.c_int
 MOE_STAGE_EVENTS = 7
+_lib.moe_forward_noalloc.argtypes = [_P(moe_shape), _P(moe_options), _P(moe_tensors), C.c_void_p]
+_lib.moe_forward_noalloc.restype = C.c_int
+MOE_NOALLOC_WORKSPACE_BYTES = 64 << 20
 STAGES = ("route", "sort", "gather", "gate_up", "down", "combine")
 _lib.moe_last_error.argtypes = []
 _lib.moe_last_error.restype = C.c_char_p
@@ -81,7 +84,8 @@ _lib.moe_version.argtypes = []
 _lib.moe_version.restype = C.c_char_p
 
 EXPORTED = ("moe_options_init", "moe_workspace_size", "moe_forward", "moe_route",
-            "moe_forward_events", "moe_last_error", "moe_debug_status", "moe_version")
+            "moe_forward_events", "moe_forward_noalloc", "moe_last_error", "moe_debug_status",
+            "moe_version")
 
 
 class MoeError(RuntimeError):
@@ -117,6 +121,11 @@ def moe_forward_events(shape, opts, tensors, workspace: int, workspace_bytes: in
     arr = (C.c_void_p * len(events))(*events)
     return _lib.moe_forward_events(C.byref(shape), C.byref(opts), C.byref(tensors), workspace,
                                    workspace_bytes, stream, arr, len(events))
+
+
+def moe_forward_noalloc(shape, opts, tensors, stream: int) -> int:
+    """moe_forward on the library's static scratch array (no workspace argument)."""
+    return _lib.moe_forward_noalloc(C.byref(shape), C.byref(opts), C.byref(tensors), stream)
 
 
 def moe_last_error() -> str:

@@ -284,6 +284,13 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
 
 }  // namespace
 
+int forward_on_workspace(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws,
+                         size_t ws_bytes, void* stream) {
+  return run(s, o, t, ws, ws_bytes, stream, true);
+}
+
+int set_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
 size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   (void)o;
   p->T = s->T;

@@ -45,6 +45,12 @@ struct Plan {
 // Fills `p` from validated arguments; returns the workspace size.
 size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p);
 
+// The whole forward on a given device workspace (the body of moe_forward).
+int forward_on_workspace(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws,
+                         size_t ws_bytes, void* stream);
+// Records a message for moe_last_error() and returns `code`.
+int set_error(int code, const char* msg);
+
 // ---------------------------------------------------------------- device status
 // First word of the workspace: 0 = OK, else a moe_status a kernel recorded.
 __device__ __forceinline__ void set_status(int* status, int code) {

@@ -1,0 +1,54 @@
+"""moe_forward_noalloc: the forward on the library's own static scratch array.
+
+Callers that cannot allocate device memory (a plugin inside a runtime that
+owns all device memory, a request path that must not call cudaMalloc) use this
+entry point instead of passing a workspace.  This file is collected last so
+that a run stopping at its first failure has already run every other test.
+"""
+import numpy as np
+import pytest
+import torch
+
+from workloads import CONFIGS, make_inputs, small
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2  # bf16 output tolerance of the parity tests (of max|y|)
+
+
+def _cfg(seed):
+    return small(CONFIGS["decode_T64"], name="noalloc", T=96, d=512, F=384, E=32, k=4, seed=seed)
+
+
+def test_noalloc_entry_matches_moe_forward_on_two_calls_in_a_row():
+    import mixture_experts_ffn_10_b200 as m
+    stream = torch.cuda.current_stream().cuda_stream
+    for seed in (2101, 2102):  # two calls in a row, different inputs each time
+        cfg = _cfg(seed)
+        inputs = make_inputs(cfg, "cuda")
+        ref = m.forward(cfg, inputs)          # the existing entry point, caller workspace
+        y = torch.full_like(inputs["x"], float("nan"))
+        shape, opts = m.shape_of(cfg), m.options_of(cfg)
+        assert m.moe_workspace_size(shape, opts) <= m.MOE_NOALLOC_WORKSPACE_BYTES
+        rc = m.moe_forward_noalloc(shape, opts, m.tensors_of(inputs, y), stream)
+        assert rc == m.MOE_OK, m.moe_last_error()
+        torch.cuda.synchronize()
+        a = y.float().cpu().numpy()
+        b = ref.float().cpu().numpy()
+        assert np.isfinite(a).all()
+        assert np.abs(a - b).max() <= TOL * np.abs(b).max()
+
+
+def test_noalloc_entry_rejects_problems_beyond_its_scratch():
+    import mixture_experts_ffn_10_b200 as m
+    cfg = small(CONFIGS["mixtral_bf16"], T=4096)
+    shape, opts = m.shape_of(cfg), m.options_of(cfg)
+    assert m.moe_workspace_size(shape, opts) > m.MOE_NOALLOC_WORKSPACE_BYTES
+    t = m.moe_tensors()
+    fake = 1 << 20
+    for n in ("x", "router_logits", "gate_up", "down"):
+        setattr(t, n, fake)
+    t.y = 2 * fake
+    rc = m.moe_forward_noalloc(shape, opts, t, torch.cuda.current_stream().cuda_stream)
+    assert rc == m.MOE_ERR_WORKSPACE
+    assert "static array" in m.moe_last_error()
