@@ -59,7 +59,8 @@ int check_shape_opts(const moe_shape* s, const moe_options* o) {
     return fail(MOE_ERR_SHAPE, "d, F and Fs must be multiples of 8 (16-byte rows)");
   if (s->w_dtype == MOE_MXFP4 && (s->d % 32 || s->F % 32))
     return fail(MOE_ERR_SHAPE, "MXFP4 experts need d and F multiples of 32 (block size)");
-  if (s->w_dtype == MOE_MXFP4) return fail(MOE_ERR_UNSUPPORTED, "MXFP4 expert weights are not built in this version");
+  if (s->w_dtype == MOE_MXFP4 && s->Fs > 0)
+    return fail(MOE_ERR_UNSUPPORTED, "a shared expert next to MXFP4 routed experts is not built");
   const int64_t rows = s->T * s->k + (s->Fs > 0 ? s->T : 0);
   if (s->T > (1ll << 26) || rows >= (1ll << 31))
     return fail(MOE_ERR_SHAPE, "T*k + T must stay below 2^31 rows (T=%lld)", (long long)s->T);
@@ -249,11 +250,16 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
     ta.h = at<void>(ws, p.o_h);
     ta.Y = at<void>(ws, p.o_y);
     ta.num_sms = num_sms_of_current_device();
+    ta.gate_up_scales = t->gate_up_scales;
+    ta.down_scales = t->down_scales;
+    const bool fp4 = s->w_dtype == MOE_MXFP4;
     ta.c = gu;
-    if ((e = launch_tc_gate_up(ta, st)) != cudaSuccess) return cuda_fail(e, "tensor-core gate_up GEMM");
+    e = fp4 ? launch_fp4_gate_up(ta, st) : launch_tc_gate_up(ta, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core gate_up GEMM");
     if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     ta.c = dn;
-    if ((e = launch_tc_down(ta, st)) != cudaSuccess) return cuda_fail(e, "tensor-core down GEMM");
+    e = fp4 ? launch_fp4_down(ta, st) : launch_tc_down(ta, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core down GEMM");
   } else {
     SimtArgs sm{};
     sm.x = (const float*)t->x;
@@ -308,7 +314,12 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   p->w_dtype = s->w_dtype;
   p->logit_dtype = s->logit_dtype;
   p->tc = s->act_dtype == MOE_BF16;
-  if (p->tc) {
+  if (s->w_dtype == MOE_MXFP4) {
+    p->bm = kFp4BM;
+    p->nt_gu_routed = (int)cdiv(s->F, kFp4GuBN);
+    p->nt_dn_routed = (int)cdiv(s->d, kFp4DnBN);
+    p->nt_gu_shared = p->nt_dn_shared = 0;
+  } else if (p->tc) {
     p->bm = kTcBM;
     p->nt_gu_routed = (int)cdiv(s->F, kTcGuBN);
     p->nt_gu_shared = (int)cdiv(s->Fs, kTcGuBN);

@@ -201,8 +201,16 @@ struct TcArgs {
   void* h;                  // [rows, Fmax] bf16
   void* Y;                  // [rows, d] bf16
   int num_sms;
+  const uint8_t* gate_up_scales;  // MXFP4 only: e8m0 [E, 2F, d/32]
+  const uint8_t* down_scales;     // MXFP4 only: e8m0 [E, d, F/32]
 };
 cudaError_t launch_tc_gate_up(const TcArgs& a, cudaStream_t st);
 cudaError_t launch_tc_down(const TcArgs& a, cudaStream_t st);
+// MXFP4 expert stacks (gate_up / down are e2m1 codes); no shared expert.
+cudaError_t launch_fp4_gate_up(const TcArgs& a, cudaStream_t st);
+cudaError_t launch_fp4_down(const TcArgs& a, cudaStream_t st);
+constexpr int kFp4BM = 256;       // rows per MXFP4 tile (two M=128 halves share each decoded stage)
+constexpr int kFp4GuBN = 64;      // h features per MXFP4 gate_up tile (64 gate + 64 up rows)
+constexpr int kFp4DnBN = 128;     // output features per MXFP4 down tile
 
 }  // namespace moe

@@ -20,11 +20,8 @@
 // fetched through a 4-D tensor map view of the stack that hides the layout:
 // concat [E][2][F][d] or interleaved [E][F][2][d].  So accumulator column j
 // (< 128) is gate feature f0 + j and column 128 + j its up partner.
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 #include "sm100.cuh"
+#include "tmap.cuh"
 
 namespace moe {
 namespace {
@@ -52,27 +49,6 @@ struct TcParams {
   const float* roww;             // [R]
   uint16_t* out;                 // h [rows, Fmax] or Y [rows, d]
 };
-
-struct Tile {
-  int seg, m0, n_blk, rows;
-};
-
-__device__ __forceinline__ Tile decode_tile(const GemmCommon& c, int tile) {
-  int lo = 0, hi = c.NS - 1;  // last segment s with tiles[s] <= tile
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (c.tiles[mid] <= tile) lo = mid;
-    else hi = mid - 1;
-  }
-  Tile t;
-  t.seg = lo;
-  t.rows = c.cnt[lo];
-  const int mt = (t.rows + BM - 1) / BM;
-  const int local = tile - c.tiles[lo];
-  t.n_blk = local / mt;
-  t.m0 = (local % mt) * BM;
-  return t;
-}
 
 template <int MODE>
 __device__ __forceinline__ int k_extent(const GemmCommon& c, bool shared) {
@@ -130,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const Tile t = decode_tile(c, tile);
+        const Tile t = decode_tile<BM>(c, tile);
         const bool sh = t.seg >= c.E;
         const int nkb = (k_extent<MODE>(c, sh) + BK - 1) / BK;
         const int arow = sh ? t.m0 : c.off[t.seg] + t.m0;
@@ -174,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, tcount++) {
-        const Tile t = decode_tile(c, tile);
+        const Tile t = decode_tile<BM>(c, tile);
         const bool sh = t.seg >= c.E;
         const int nkb = (k_extent<MODE>(c, sh) + BK - 1) / BK;
         const int acc = tcount & 1;
@@ -209,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r_in_tile = q * 32 + lane;
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, tcount++) {
-      const Tile t = decode_tile(c, tile);
+      const Tile t = decode_tile<BM>(c, tile);
       const bool sh = t.seg >= c.E;
       const int acc = tcount & 1;
       if (!mbar_wait(&tfull[acc], (tcount >> 1) & 1, abort_flag, c.status)) break;
@@ -311,29 +287,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
-// bf16 tensor map, dims[0] innermost (elements), strides in bytes for dims 1.., box dims.
+// bf16 tensor map with the 128-byte swizzle the UMMA descriptors expect.
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
               const uint32_t* box) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
-                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // rows x K matrix with row pitch `pitch` elements; box 64 x box_rows.

@@ -20,6 +20,7 @@ DSK = small(CONFIGS["deepseek_bf16"], name="deepseek_small", T=130, d=256, F=128
 GPT = small(CONFIGS["gptoss_mxfp4"], name="gptoss_bf16_small", w_dtype="bf16", T=200, d=320, F=352,
             E=8, k=4)
 DEC = small(CONFIGS["decode_T1"], name="decode_small", d=512, F=256, E=32)
+FP4 = small(CONFIGS["gptoss_mxfp4"], name="gptoss_mxfp4_small", T=200, d=320, F=352, E=8, k=4)
 TINY = CONFIGS["tiny_fp32"]
 
 CASES = {
@@ -50,6 +51,10 @@ CASES = {
     "k_equals_E": small(MIX, name="k_equals_E", E=4, k=4, renormalize=False),
     "ragged_d_F": small(MIX, name="ragged_d_F", d=72, F=40, Fs=24, T=70),
     "many_experts": small(MIX, name="many_experts", E=256, k=8, T=64, d=128, F=64),
+    "gptoss_mxfp4_small": FP4,
+    "mxfp4_concat": small(FP4, name="mxfp4_concat", gu_layout="concat", limit=0.0, alpha=1.0),
+    "mxfp4_T1_many_experts": small(FP4, name="mxfp4_T1_many_experts", T=1, E=32, k=4),
+    "mxfp4_big_rows": small(FP4, name="mxfp4_big_rows", T=700, E=4, k=2, d=256, F=256),
 }
 
 
@@ -145,3 +150,31 @@ def test_zero_tokens_no_op_on_gpu():
     y = m.forward(cfg, inputs)
     torch.cuda.synchronize()
     assert y.shape == (0, cfg.d)
+
+
+def _dequant_mxfp4(q, s):
+    """bf16 weights equal to an MXFP4 stack, decoded with the oracle's own e2m1/e8m0 decoders."""
+    table = torch.tensor([oracle.decode_e2m1(c) for c in range(16)], dtype=torch.float64)
+    q = q.cpu().to(torch.int64)
+    codes = torch.stack([q & 0xF, q >> 4], -1).reshape(*q.shape[:-1], q.shape[-1] * 2)
+    scale = torch.tensor([oracle.decode_e8m0(v) for v in range(256)], dtype=torch.float64)[s.cpu().to(torch.int64)]
+    w = table[codes] * scale.repeat_interleave(32, -1)
+    out = w.to(torch.bfloat16)
+    assert torch.equal(out.double(), w)  # every MXFP4 value is exact in bf16
+    return out
+
+
+@pytest.mark.parametrize("layout", ["interleaved", "concat"])
+def test_mxfp4_path_equals_bf16_path_on_dequantized_weights(layout):
+    cfg = small(FP4, gu_layout=layout)
+    inputs = make_inputs(cfg, "cuda")
+    y4, i4, _ = run_gpu(cfg, inputs)
+    deq = dict(inputs)
+    deq["gate_up"] = _dequant_mxfp4(inputs["gate_up"], inputs["gate_up_scales"]).cuda()
+    deq["down"] = _dequant_mxfp4(inputs["down"], inputs["down_scales"]).cuda()
+    deq["gate_up_scales"] = deq["down_scales"] = None
+    yb, ib, _ = run_gpu(small(cfg, w_dtype="bf16"), deq)
+    torch.cuda.synchronize()
+    assert torch.equal(i4, ib)
+    a, b = y4.float(), yb.float()
+    assert (a - b).abs().max().item() <= 1e-2 * b.abs().max().item()
