@@ -13,15 +13,19 @@
 // weight stage, halving the decode work per FLOP.  Warp roles:
 //   warp 0      TMA: activations 256 x 64 (bf16, 128B swizzle) and codes 128 x 32 B
 //   warp 1      TMEM owner and MMA issuer (M=128 N=128 K=16 per half)
-//   warps 2-5   epilogue (bias + activation, or bias x routing weight; bf16 stores)
-//   warps 6-13  converters: codes + scale -> bf16 in the 128B-swizzled K-major layout
-//               the MMA descriptor reads, then a proxy fence and a barrier arrive.
-// Decode: a code's 3 magnitude bits select the two bytes of its unscaled bf16 value
-// through byte permutes of two 8-entry byte tables, the sign bit is moved to bit 15,
-// and one bf16x2 multiply by 2^(s-127) applies the block scale.  Exact (both factors
-// have at most two significant bits) for scale bytes 8..252.
+//   warps 2-9   epilogue (bias + activation, or bias x routing weight; bf16 stores);
+//               warps 2-5 drain the first M half, warps 6-9 the second
+//   warps 10-25 converters: codes + scale -> bf16 in the 128B-swizzled K-major layout
+//               the MMA descriptor reads, then a proxy fence and one arrive per warp.
+// Decode: the hardware conversion cvt.rn.f16x2.e2m1x2 turns each code byte into two
+// exact f16 values; shifting an f16's exponent and mantissa right by 3 bits (sign
+// kept) gives a bf16 of the same value times 2^-112, and one bf16x2 multiply by
+// 2^(s-15) applies the block scale and undoes the bias.  Exact (both factors have
+// at most two significant bits, the product stays normal) for scale bytes 2..142;
+// larger scale bytes take a second multiply.
 #include <cuda_bf16.h>
 
+#include "epilogue.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
 
@@ -41,13 +45,13 @@ constexpr int W_BYTES = BNB * BK * 2;   // 16 KiB decoded bf16
 constexpr int STAGE_BYTES = A_BYTES + Q_BYTES + W_BYTES;
 constexpr int ACC_COLS = 2 * BNB;       // two halves
 constexpr int TMEM_COLS = 2 * ACC_COLS; // double-buffered
-constexpr int kEpiWarps = 4;
-constexpr int kCvtWarps = 8;
-constexpr int kCvtThreads = kCvtWarps * 32;  // one (row, 32-element block) per thread and stage
+constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant: one per M half
+constexpr int kCvtWarps = 16;
+constexpr int kCvtThreads = kCvtWarps * 32;  // 16 elements (8 code bytes) per thread and stage
 constexpr int kThreads = 64 + (kEpiWarps + kCvtWarps) * 32;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr uint32_t IDESC = idesc_bf16_f32(HALF, BNB);
-static_assert(kCvtThreads == BNB * (BK / 32), "one converter thread per (row, block)");
+static_assert(kCvtThreads == BNB * (BK / 16), "one converter thread per (row, 16 elements)");
 
 struct Fp4Params {
   GemmCommon c;
@@ -78,38 +82,44 @@ __device__ __forceinline__ int weight_row(const GemmCommon& c, int n_blk, int r,
   return o;
 }
 
-// 8 e2m1 codes (one 32-bit word, element j in bits 4j..4j+3) -> 4 bf16x2 words, scaled.
-__device__ __forceinline__ void decode8(uint32_t w, __nv_bfloat162 scale2, uint32_t (&out)[4]) {
-  // unscaled bf16 of magnitude code 0..7: {0, .5, 1, 1.5, 2, 3, 4, 6}
-  constexpr uint32_t kHi0 = 0x3F3F3F00u, kHi1 = 0x40404040u;  // high bytes, codes 0-3 / 4-7
-  constexpr uint32_t kLo0 = 0xC0800000u, kLo1 = 0xC0804000u;  // low bytes
-  const uint32_t m = w & 0x77777777u;
-  const uint32_t sel_a = m, sel_b = m >> 16;
-  const uint32_t hi_a = __byte_perm(kHi0, kHi1, sel_a), lo_a = __byte_perm(kLo0, kLo1, sel_a);
-  const uint32_t hi_b = __byte_perm(kHi0, kHi1, sel_b), lo_b = __byte_perm(kLo0, kLo1, sel_b);
-  uint32_t p[4];
-  p[0] = __byte_perm(lo_a, hi_a, 0x5140);
-  p[1] = __byte_perm(lo_a, hi_a, 0x7362);
-  p[2] = __byte_perm(lo_b, hi_b, 0x5140);
-  p[3] = __byte_perm(lo_b, hi_b, 0x7362);
-  // sign of element j (bit 4j+3) -> bit 15 (even j) or bit 31 (odd j) of its pair
-  p[0] |= ((w << 12) & 0x8000u) | ((w << 24) & 0x80000000u);
-  p[1] |= ((w << 4) & 0x8000u) | ((w << 16) & 0x80000000u);
-  p[2] |= ((w >> 4) & 0x8000u) | ((w << 8) & 0x80000000u);
-  p[3] |= ((w >> 12) & 0x8000u) | (w & 0x80000000u);
-#pragma unroll
-  for (int i = 0; i < 4; i++) {
-    __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&p[i]);
-    v = __hmul2(v, scale2);
-    out[i] = *reinterpret_cast<uint32_t*>(&v);
-  }
+// 8 e2m1 codes (one 32-bit word, element j in bits 4j..4j+3) -> 4 f16x2 words
+// (element 2i in the low half of word i), exact.
+__device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t (&h)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
 }
 
-// bf16x2 holding 2^(s-127) twice (s = 0 is the subnormal 2^-127, 255 is NaN).
-__device__ __forceinline__ __nv_bfloat162 scale_pair(uint32_t s) {
-  const uint32_t b = s == 0 ? 0x0040u : (s == 255 ? 0x7FC0u : (s << 7));
-  const uint32_t pr = b | (b << 16);
-  return *reinterpret_cast<const __nv_bfloat162*>(&pr);
+// f16x2 of e2m1 values -> bf16x2 of the same values times 2^-112 (exponent and
+// mantissa bits moved down by 3, signs kept; the low 3 mantissa bits are zero).
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2_biased(uint32_t h) {
+  return ((h >> 3) & 0x0FFF0FFFu) | (h & 0x80008000u);
+}
+
+// bf16x2 multiplier that applies 2^(s-127) to a value biased by 2^-112: 2^(s-15).
+// For s > 142 that factor is not a bf16; `extra` then holds the remaining 2^(s-142).
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t s, uint32_t* extra) {
+  uint32_t e = s + 112;   // bf16 exponent field of 2^(s-15)
+  *extra = 0;
+  if (s == 255) e = 255;  // NaN scale propagates
+  else if (e > 254) {
+    *extra = (s - 142 + 127) << 7;  // 2^(s-142)
+    *extra |= *extra << 16;
+    e = 254;                          // 2^127
+  }
+  const uint32_t b = (e << 7) | (s == 255 ? 0x40u : 0u);
+  return b | (b << 16);
+}
+
+__device__ __forceinline__ uint32_t bmul(uint32_t a, uint32_t b) {
+  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a), y = *reinterpret_cast<__nv_bfloat162*>(&b);
+  x = __hmul2(x, y);
+  return *reinterpret_cast<uint32_t*>(&x);
 }
 
 template <int MODE>
@@ -133,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; s++) {
       mbar_init(&full[s], 1);
-      mbar_init(&conv[s], kCvtThreads);
+      mbar_init(&conv[s], kCvtWarps);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; b++) {
@@ -161,33 +171,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      auto issue = [&](const Tile& t, int kb, uint64_t* bar, uint8_t* sa) {
+        const int arow = c.off[t.seg] + t.m0;
+        uint8_t* sq = sa + A_BYTES;
+        const int ka = kb * BK, kq = kb * (BK / 2);
+        tma_load_2d(&tmA, bar, sa, ka, arow);
+        if (MODE == 0) {
+          const int f0 = t.n_blk * (BNB / 2);
+          const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
+          for (int half = 0; half < 2; half++) {
+            const int c1 = il ? half : f0, c2 = il ? f0 : half;
+            tma_load_4d(&tmQ, bar, sq + half * (Q_BYTES / 2), kq, c1, c2, t.seg);
+          }
+        } else {
+          tma_load_3d(&tmQ, bar, sq, kq, t.n_blk * BNB, t.seg);
+        }
+      };
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         const Tile t = decode_tile<BM>(c, tile);
-        const int arow = c.off[t.seg] + t.m0;
         for (int kb = 0; kb < nkb; kb++, it++) {
           const int s = it % STAGES;
           if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, c.status)) {
             ok = false;
             break;
           }
-          uint8_t* sa = smem + s * STAGE_BYTES;
-          uint8_t* sq = sa + A_BYTES;
           mbar_arrive_expect_tx(&full[s], A_BYTES + Q_BYTES);
-          tma_load_2d(&tmA, &full[s], sa, kb * BK, arow);
-          if (MODE == 0) {
-            const int f0 = t.n_blk * (BNB / 2);
-            if (c.gu_layout == MOE_GU_INTERLEAVED) {
-              tma_load_4d(&tmQ, &full[s], sq, kb * (BK / 2), 0, f0, t.seg);
-              tma_load_4d(&tmQ, &full[s], sq + Q_BYTES / 2, kb * (BK / 2), 1, f0, t.seg);
-            } else {
-              tma_load_4d(&tmQ, &full[s], sq, kb * (BK / 2), f0, 0, t.seg);
-              tma_load_4d(&tmQ, &full[s], sq + Q_BYTES / 2, kb * (BK / 2), f0, 1, t.seg);
-            }
-          } else {
-            tma_load_3d(&tmQ, &full[s], sq, kb * (BK / 2), t.n_blk * BNB, t.seg);
-          }
+          issue(t, kb, &full[s], smem + s * STAGE_BYTES);
         }
       }
       for (uint32_t j = (it > (uint32_t)STAGES ? it - STAGES : 0); j < it; j++) {
@@ -236,24 +247,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 2 + kEpiWarps) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;
+    const int q = warp & 3;                 // TMEM lane quadrant this warp may read
+    const int h = (warp - 2) / 4;           // M half this warp drains
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, tcount++) {
       const Tile t = decode_tile<BM>(c, tile);
       const int acc = tcount & 1;
       if (!mbar_wait(&tfull[acc], (tcount >> 1) & 1, abort_flag, c.status)) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int h = 0; h < 2; h++) {
-        const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS + h * BNB;
-        const int row = t.m0 + h * HALF + q * 32 + lane;
-        const bool valid = row < t.rows;
-        if (!__any_sync(0xffffffffu, valid)) continue;
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS + h * BNB;
+      const int row = t.m0 + h * HALF + q * 32 + lane;
+      const bool valid = row < t.rows;
+      if (__any_sync(0xffffffffu, valid)) {
         const int64_t grow = (int64_t)c.off[t.seg] + row;
         if (MODE == 0) {
-          const int F = c.F;
           const int f0 = t.n_blk * (BNB / 2);
-          const uint16_t* bias = p.gate_up_bias ? p.gate_up_bias + (int64_t)t.seg * 2 * F : nullptr;
+          const uint16_t* bias = p.gate_up_bias ? p.gate_up_bias + (int64_t)t.seg * 2 * c.F : nullptr;
           const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
           uint16_t* out = p.out + grow * c.Fmax;
 #pragma unroll 1
@@ -263,35 +272,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld16(tb + BNB / 2 + ch * 16, u);
             tmem_ld_wait();
             const int fb = f0 + ch * 16;
-            if (valid && fb < F) {
-              uint32_t packed[8];
-#pragma unroll
-              for (int i = 0; i < 16; i += 2) {
-                float hv[2];
-#pragma unroll
-                for (int h2 = 0; h2 < 2; h2++) {
-                  const int f = fb + i + h2;
-                  float gv = __uint_as_float(g[i + h2]), uv = __uint_as_float(u[i + h2]);
-                  if (bias && f < F) {
-                    gv += bf16_to_f32(bias[il ? 2 * f : f]);
-                    uv += bf16_to_f32(bias[il ? 2 * f + 1 : F + f]);
-                  }
-                  hv[h2] = gated_act(c.act, gv, uv);
-                }
-                packed[i / 2] = pack_bf16x2(hv[0], hv[1]);
-              }
-              if (fb + 16 <= F) {
-                uint4* dst = reinterpret_cast<uint4*>(out + fb);
-                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-              } else {
-                for (int i = 0; i < 16 && fb + i < F; i++)
-                  out[fb + i] = (uint16_t)(packed[i / 2] >> (16 * (i & 1)));
-              }
-            }
+            if (valid && fb < c.F) gate_up_chunk(g, u, bias, fb, c.F, il, c.act, out);
           }
         } else {
-          const int N = c.d;
           const int n0 = t.n_blk * BNB;
           const uint16_t* bias = p.down_bias ? p.down_bias + (int64_t)t.seg * c.d : nullptr;
           const float w = (c.weigh_inputs || !valid) ? 1.f : p.roww[grow];
@@ -302,28 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld16(tb + ch * 16, v);
             tmem_ld_wait();
             const int ob = n0 + ch * 16;
-            if (valid && ob < N) {
-              uint32_t packed[8];
-#pragma unroll
-              for (int i = 0; i < 16; i += 2) {
-                float o[2];
-#pragma unroll
-                for (int h2 = 0; h2 < 2; h2++) {
-                  float a = __uint_as_float(v[i + h2]);
-                  if (bias && ob + i + h2 < N) a += bf16_to_f32(bias[ob + i + h2]);
-                  o[h2] = a * w;
-                }
-                packed[i / 2] = pack_bf16x2(o[0], o[1]);
-              }
-              if (ob + 16 <= N) {
-                uint4* dst = reinterpret_cast<uint4*>(out + ob);
-                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-              } else {
-                for (int i = 0; i < 16 && ob + i < N; i++)
-                  out[ob + i] = (uint16_t)(packed[i / 2] >> (16 * (i & 1)));
-              }
-            }
+            if (valid && ob < c.d) down_chunk(v, bias, ob, c.d, w, out);
           }
         }
       }
@@ -332,10 +294,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ converters
-    const int u = threadIdx.x - 64 - kEpiWarps * 32;  // 0 .. kCvtThreads-1
-    const int r = u % BNB;                           // weight row inside the tile
-    const int b = u / BNB;                           // 32-element block inside the stage
-    const int kblocks = K / 32;                      // scale bytes per weight row
+    // Lane layout: 8 weight rows x 4 quarters (16 elements each) per warp, so the
+    // 8-byte code loads cover 256 contiguous bytes and the swizzled 16-byte stores
+    // of a quarter-warp hit distinct banks.
+    const int cw = warp - 2 - kEpiWarps;         // 0 .. kCvtWarps-1
+    const int r = cw * 8 + (lane >> 2);          // weight row inside the tile
+    const int g = lane & 3;                      // quarter of the 64-element stage
+    const int b = g >> 1;                        // 32-element scale block
+    const int kblocks = K / 32;                  // scale bytes per weight row
     const int rows_per_e = MODE == 0 ? 2 * c.F : c.d;
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -358,19 +324,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         uint8_t* base = smem + st * STAGE_BYTES;
-        const uint4 q = *reinterpret_cast<const uint4*>(base + A_BYTES + r * (BK / 2) + b * 16);
+        const uint2 q = *reinterpret_cast<const uint2*>(base + A_BYTES + r * (BK / 2) + g * 8);
         uint8_t* wrow = base + A_BYTES + Q_BYTES + r * (BK * 2);
-        const __nv_bfloat162 sc = scale_pair(s0);
-        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+        uint32_t extra;
+        const uint32_t sc = scale_bf16x2(s0, &extra);
+        const uint32_t words[2] = {q.x, q.y};
 #pragma unroll
-        for (int wi = 0; wi < 4; wi++) {
-          uint32_t o[4];
-          decode8(words[wi], sc, o);
-          const int chunk = b * 4 + wi;  // 16-byte chunk of the 128-byte row
+        for (int wi = 0; wi < 2; wi++) {
+          uint32_t h[4], o[4];
+          e2m1x8_to_f16x8(words[wi], h);
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            o[i] = bmul(f16x2_to_bf16x2_biased(h[i]), sc);
+            if (extra) o[i] = bmul(o[i], extra);
+          }
+          const int chunk = g * 2 + wi;  // 16-byte chunk (8 elements) of the 128-byte row
           *reinterpret_cast<uint4*>(wrow + ((chunk ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         fence_proxy_async_smem();
-        mbar_arrive(&conv[st]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&conv[st]);
         s0 = s1;
         s1 = s2;
         s2 = s3;

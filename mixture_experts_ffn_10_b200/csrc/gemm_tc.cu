@@ -14,12 +14,14 @@
 //              swizzle) per stage into a 4-stage shared-memory ring;
 //   warp 1     TMEM allocator and MMA issuer: tcgen05.mma M=128 N=256 K=16,
 //              fp32 accumulators in TMEM, two accumulator buffers of 256 columns;
-//   warps 2-5  epilogue: tcgen05.ld the accumulator rows, bias + activation (or
+//   warps 2-9  epilogue: tcgen05.ld the accumulator rows, bias + activation (or
 //              bias x routing weight), bf16 stores; overlaps the next tile's MMAs.
+//              Warps w and w+4 share a TMEM lane quadrant and alternate chunks.
 // For gate_up the B tile is 128 gate rows followed by the 128 matching up rows,
 // fetched through a 4-D tensor map view of the stack that hides the layout:
 // concat [E][2][F][d] or interleaved [E][F][2][d].  So accumulator column j
 // (< 128) is gate feature f0 + j and column 128 + j its up partner.
+#include "epilogue.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
 
@@ -37,7 +39,7 @@ constexpr int B_BYTES = BNB * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, splitting the column chunks
 constexpr int kThreads = 64 + kEpiWarps * 32;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BNB);
@@ -103,38 +105,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t it = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const Tile t = decode_tile<BM>(c, tile);
+      auto issue = [&](const Tile& t, int kb, uint64_t* bar, uint8_t* sa) {
         const bool sh = t.seg >= c.E;
-        const int nkb = (k_extent<MODE>(c, sh) + BK - 1) / BK;
         const int arow = sh ? t.m0 : c.off[t.seg] + t.m0;
         const CUtensorMap* mA = sh ? &tmAs : &tmA;
         const CUtensorMap* mB = sh ? &tmBs : &tmB;
         const int e = sh ? 0 : t.seg;
+        const int k0 = kb * BK;
+        tma_load_2d(mA, bar, sa, k0, arow);
+        if (MODE == 0) {
+          const int f0 = t.n_blk * (BNB / 2);
+          const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
+          for (int half = 0; half < 2; half++) {
+            const int c1 = il ? half : f0, c2 = il ? f0 : half;
+            tma_load_4d(mB, bar, sa + A_BYTES + half * (B_BYTES / 2), k0, c1, c2, e);
+          }
+        } else {
+          tma_load_3d(mB, bar, sa + A_BYTES, k0, t.n_blk * BNB, e);
+        }
+      };
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const Tile t = decode_tile<BM>(c, tile);
+        const int nkb = (k_extent<MODE>(c, t.seg >= c.E) + BK - 1) / BK;
         for (int kb = 0; kb < nkb; kb++, it++) {
           const int s = it % STAGES;
           if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, c.status)) {
             ok = false;
             break;
           }
-          uint8_t* sa = smem + s * STAGE_BYTES;
-          uint8_t* sb = sa + A_BYTES;
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-          tma_load_2d(mA, &full[s], sa, kb * BK, arow);
-          if (MODE == 0) {
-            const int f0 = t.n_blk * (BNB / 2);
-            if (c.gu_layout == MOE_GU_INTERLEAVED) {
-              tma_load_4d(mB, &full[s], sb, kb * BK, 0, f0, e);
-              tma_load_4d(mB, &full[s], sb + B_BYTES / 2, kb * BK, 1, f0, e);
-            } else {
-              tma_load_4d(mB, &full[s], sb, kb * BK, f0, 0, e);
-              tma_load_4d(mB, &full[s], sb + B_BYTES / 2, kb * BK, f0, 1, e);
-            }
-          } else {
-            tma_load_3d(mB, &full[s], sb, kb * BK, t.n_blk * BNB, e);
-          }
+          issue(t, kb, &full[s], smem + s * STAGE_BYTES);
         }
       }
       // every load issued into a stage has landed before the CTA may exit
@@ -181,7 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // this warp may read TMEM lanes 32q .. 32q+31
+    const int q = warp & 3;            // this warp may read TMEM lanes 32q .. 32q+31
+    const int part = (warp - 2) / 4;   // which alternate column chunks this warp drains
     const int r_in_tile = q * 32 + lane;
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, tcount++) {
@@ -202,73 +205,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
           uint16_t* out = p.out + grow * c.Fmax;
 #pragma unroll 1
-          for (int ch = 0; ch < (BNB / 2) / 16; ch++) {
+          for (int ch = part; ch < (BNB / 2) / 16; ch += 2) {
             uint32_t g[16], u[16];
             tmem_ld16(tb + ch * 16, g);
             tmem_ld16(tb + BNB / 2 + ch * 16, u);
             tmem_ld_wait();
             const int fb = f0 + ch * 16;
-            if (valid && fb < F) {
-              uint32_t packed[8];
-#pragma unroll
-              for (int i = 0; i < 16; i += 2) {
-                float hv[2];
-#pragma unroll
-                for (int h2 = 0; h2 < 2; h2++) {
-                  const int f = fb + i + h2;
-                  float gv = __uint_as_float(g[i + h2]), uv = __uint_as_float(u[i + h2]);
-                  if (bias && f < F) {
-                    gv += bf16_to_f32(bias[il ? 2 * f : f]);
-                    uv += bf16_to_f32(bias[il ? 2 * f + 1 : F + f]);
-                  }
-                  hv[h2] = gated_act(c.act, gv, uv);
-                }
-                packed[i / 2] = pack_bf16x2(hv[0], hv[1]);
-              }
-              if (fb + 16 <= F) {
-                uint4* dst = reinterpret_cast<uint4*>(out + fb);
-                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-              } else {
-                for (int i = 0; i < 16 && fb + i < F; i++)
-                  out[fb + i] = (uint16_t)(packed[i / 2] >> (16 * (i & 1)));
-              }
-            }
+            if (valid && fb < F) gate_up_chunk(g, u, bias, fb, F, il, c.act, out);
           }
         } else {
-          const int N = c.d;
           const int n0 = t.n_blk * BNB;
           const uint16_t* bias = (!sh && p.down_bias) ? p.down_bias + (int64_t)t.seg * c.d : nullptr;
           const float w = (sh || c.weigh_inputs || !valid) ? 1.f : p.roww[grow];
           uint16_t* out = p.out + grow * c.d;
 #pragma unroll 1
-          for (int ch = 0; ch < BNB / 16; ch++) {
+          for (int ch = part; ch < BNB / 16; ch += 2) {
             uint32_t v[16];
             tmem_ld16(tb + ch * 16, v);
             tmem_ld_wait();
             const int ob = n0 + ch * 16;
-            if (valid && ob < N) {
-              uint32_t packed[8];
-#pragma unroll
-              for (int i = 0; i < 16; i += 2) {
-                float o[2];
-#pragma unroll
-                for (int h2 = 0; h2 < 2; h2++) {
-                  float a = __uint_as_float(v[i + h2]);
-                  if (bias && ob + i + h2 < N) a += bf16_to_f32(bias[ob + i + h2]);
-                  o[h2] = a * w;
-                }
-                packed[i / 2] = pack_bf16x2(o[0], o[1]);
-              }
-              if (ob + 16 <= N) {
-                uint4* dst = reinterpret_cast<uint4*>(out + ob);
-                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-              } else {
-                for (int i = 0; i < 16 && ob + i < N; i++)
-                  out[ob + i] = (uint16_t)(packed[i / 2] >> (16 * (i & 1)));
-              }
-            }
+            if (valid && ob < c.d) down_chunk(v, bias, ob, c.d, w, out);
           }
         }
       }
