@@ -7,9 +7,12 @@ Mixtral-shaped bf16 prefill layer (T=4096, d=4096, F=14336, E=8, k=2).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl own|reference]
 
-Timing: W warm-up steps, then K steps timed on the device with CUDA events
-recorded by the library on the launching stream at every stage boundary; the
-L2 is flushed (512 MiB write) before every timed step, outside the events.
+Timing: W warm-up steps, then K steps timed on the device with one CUDA event
+pair per step on the launching stream, each step a replay of a CUDA graph of
+the moe_forward call (--no-graph: eager calls); the L2 is flushed (512 MiB
+write) before every timed step, outside the events.  A second pass of K eager
+steps has the library record an event at every stage boundary; it gives the
+per-kernel times behind the roofline figure.
 Under torchrun each rank runs an independent replica (no collective on the data
 path); the reported time is the max over ranks and `value` counts the tokens of
 all ranks.  `e2e` repeats the measurement through the same C-ABI call with the
@@ -47,6 +50,21 @@ def peaks():
             d = json.load(f)
         return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def max_over_ranks(v: float, dist=None, device="cpu") -> float:
+    """The max of a per-rank value over all ranks (identity without a process group)."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_throughput(world: int, tokens_per_rank: int, steps: int, max_ms: float) -> float:
+    """Tokens/s of the whole job: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (max_ms / 1e3)
 
 
 def workload_name(cfg):
@@ -219,13 +237,6 @@ def run_own(args, cfg):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     stream = torch.cuda.Stream()
     inputs = make_inputs(cfg, "cuda")
     shape, opts = moe.shape_of(cfg), moe.options_of(cfg)
@@ -261,24 +272,51 @@ def run_own(args, cfg):
         raise RuntimeError(f"device status {moe.STATUS_NAMES.get(status, status)}")
 
     # ------------------------------------------------------------ device-timed steps
+    # Pass 1 (the reported time): one event pair per step around the forward,
+    # replayed from a CUDA graph of the C-ABI call unless --no-graph.
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        torch.cuda.synchronize()
+    t0s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t1s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for i in range(args.steps):
             flush.zero_()
-            step(handles[i])
+            t0s[i].record(stream)
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
+            t1s[i].record(stream)
     torch.cuda.synchronize()
     barrier()
+    total_ms = sum(a.elapsed_time(b) for a, b in zip(t0s, t1s))
+    status = moe.moe_debug_status(ws.ptr, sptr)
+    if status != 0:
+        raise RuntimeError(f"device status {moe.STATUS_NAMES.get(status, status)}")
+
+    # Pass 2 (per-kernel breakdown for the roofline): the library records an event at
+    # every stage boundary on the launching stream, eager launches.
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.zero_()
+            step(handles[i])
+    torch.cuda.synchronize()
     stage_ms = [0.0] * (nev - 1)
-    total_ms = 0.0
+    eager_ms = 0.0
     for row in events:
-        total_ms += row[0].elapsed_time(row[-1])
+        eager_ms += row[0].elapsed_time(row[-1])
         for s in range(nev - 1):
             stage_ms[s] += row[s].elapsed_time(row[s + 1])
     stage_ms = [v / args.steps for v in stage_ms]
-    total_ms = max_over_ranks(total_ms)
+    total_ms = max_over_ranks(total_ms, dist, "cuda")
     ms_per_step = total_ms / args.steps
-    value = world * cfg.T * args.steps / (total_ms / 1e3)
+    value = whole_job_throughput(world, cfg.T, args.steps, total_ms)
 
     # ------------------------------------------------------------ end to end (host buffers)
     x_h = inputs["x"].cpu().pin_memory()
@@ -299,8 +337,8 @@ def run_own(args, cfg):
         e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * cfg.T * e2e_steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
+    e2e_value = whole_job_throughput(world, cfg.T, e2e_steps, e2e_ms)
     clocks = sampler.stop()
 
     # ------------------------------------------------------------ roofline of the dominant kernel
@@ -330,13 +368,17 @@ def run_own(args, cfg):
              "hbm_frac_vendor_8000": layer_bytes / t_step / 1e9 / 8000.0,
              "distinct_experts": distinct, "flops": layer_flops, "bytes": layer_bytes}
 
+    if graph is not None:
+        del graph
     out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": cfg.act_dtype if cfg.w_dtype != "mxfp4" else "bf16 (mxfp4 weights)",
            "data": "synthetic (seeded; random-init weights)",
-           "config": config_dict(cfg, {"parallelism": f"replicas x{world}"}),
+           "config": config_dict(cfg, {"parallelism": f"replicas x{world}",
+                                       "launch": "cuda graph of moe_forward" if not args.no_graph else "eager moe_forward"}),
            "roofline": roofline, "layer": layer,
            "stage_ms": dict(zip(names, stage_ms)),
+           "eager_ms_per_step_with_stage_events": eager_ms / args.steps,
            "e2e": {"value": e2e_value, "unit": "tokens/s",
                    "h2d_bytes_per_step": x_h.numel() * x_h.element_size() + l_h.numel() * l_h.element_size(),
                    "d2h_bytes_per_step": y_h.numel() * y_h.element_size()},
@@ -364,6 +406,7 @@ def main():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--config", default="mixtral_bf16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of a CUDA graph replay")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle wall time")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a workload field (profiling / sweeps), e.g. --set T=1024")

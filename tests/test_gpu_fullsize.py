@@ -1,0 +1,82 @@
+"""Parity at the full workload sizes the benchmark times (same entry point and launch).
+
+Every token's routing is compared bit-exactly with the oracle; outputs are
+compared element by element on a sample of tokens (first, last and seeded
+random ones), which the oracle computes one by one; and the forward is run
+twice to check bitwise determinism at full size.  Weights of experts the
+sampled tokens do not use are never copied to the host (the host arrays are
+lazily zero-filled).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import CONFIGS, make_inputs
+
+from gpu_cases import TOL, W_RTOL, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+FULL = ["tiny_fp32", "mixtral_bf16", "gptoss_mxfp4", "deepseek_bf16", "decode_T1", "decode_T8",
+        "decode_T64", "decode_T256"]
+N_SAMPLE = 6
+
+
+def _np(t):
+    t = t.detach()
+    if t.dtype == torch.bfloat16:
+        t = t.view(torch.int16)
+    return t
+
+
+def _host_sparse(inputs, experts):
+    """Host copies: small tensors whole, expert stacks only for `experts` (rest lazily zero)."""
+    out = {}
+    for k, v in inputs.items():
+        if v is None:
+            out[k] = None
+            continue
+        a = _np(v)
+        if k in ("gate_up", "down", "gate_up_scales", "down_scales"):
+            dt = {torch.int16: np.uint16, torch.uint8: np.uint8, torch.float32: np.float32}[a.dtype]
+            h = np.zeros(tuple(a.shape), dtype=dt)  # calloc: untouched experts cost no memory
+            for e in experts:
+                h[e] = a[e].cpu().numpy().view(dt)
+            out[k] = h
+        else:
+            h = a.cpu().numpy()
+            out[k] = h.view(np.uint16) if a.dtype == torch.int16 else h
+    return out
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_parity(name):
+    cfg = CONFIGS[name]
+    torch.manual_seed(0)
+    inputs = make_inputs(cfg, "cuda")
+    y, idx, w = run_gpu(cfg, inputs)
+    y2, idx2, _ = run_gpu(cfg, inputs)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2) and torch.equal(idx, idx2), "not bitwise reproducible at full size"
+
+    # routing of every token
+    idx_h, w_h = idx.cpu().numpy(), w.cpu().numpy()
+    routing_only = {k: inputs[k] for k in ("logits", "router_bias", "selection_bias")}
+    pr = oracle.Problem(cfg, {k: (None if v is None else v.cpu()) for k, v in routing_only.items()})
+    rng = np.random.default_rng(cfg.seed)
+    sample = sorted({0, cfg.T - 1, *rng.integers(0, cfg.T, N_SAMPLE - 2).tolist()})
+    for t in range(cfg.T):
+        ri, rw, _, _ = pr.route(t)
+        assert np.array_equal(idx_h[t], ri), f"token {t}: {idx_h[t]} vs {ri}"
+        assert np.all(np.abs(w_h[t] - rw) <= W_RTOL * np.abs(rw) + 1e-30)
+
+    # outputs of the sampled tokens
+    experts = sorted({int(e) for t in sample for e in idx_h[t]})
+    p = oracle.Problem(cfg, _host_sparse(inputs, experts))
+    ref = p.forward(np.array(sample, dtype=np.int64))
+    got = y[sample].float().cpu().double().numpy()
+    scale = np.abs(ref).max()
+    err = np.abs(got - ref).max()
+    assert np.isfinite(got).all()
+    assert err <= TOL[cfg.act_dtype] * scale, f"{name}: max err {err:.3e} > {TOL[cfg.act_dtype] * scale:.3e}"

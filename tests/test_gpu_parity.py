@@ -178,3 +178,31 @@ def test_mxfp4_path_equals_bf16_path_on_dequantized_weights(layout):
     assert torch.equal(i4, ib)
     a, b = y4.float(), yb.float()
     assert (a - b).abs().max().item() <= 1e-2 * b.abs().max().item()
+
+
+@pytest.mark.parametrize("cfg", [MIX, FP4, small(DSK, shared_gate=True)], ids=["bf16", "mxfp4", "shared"])
+def test_forward_captured_in_a_cuda_graph_matches_eager(cfg):
+    import mixture_experts_ffn_10_b200 as m
+    inputs = make_inputs(cfg, "cuda")
+    shape, opts = m.shape_of(cfg), m.options_of(cfg)
+    ws = m.Workspace(m.moe_workspace_size(shape, opts))
+    y = torch.empty_like(inputs["x"])
+    tens = m.tensors_of(inputs, y)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):  # warm-up call outside the capture
+        assert m.moe_forward(shape, opts, tens, ws.ptr, ws.nbytes, s.cuda_stream) == 0
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        assert m.moe_forward(shape, opts, tens, ws.ptr, ws.nbytes, s.cuda_stream) == 0
+    # new inputs in the same buffers, then replay
+    other = make_inputs(small(cfg, seed=cfg.seed + 77), "cuda", with_weights=False)
+    inputs["x"].copy_(other["x"])
+    inputs["logits"].copy_(other["logits"])
+    g.replay()
+    torch.cuda.synchronize()
+    y_graph = y.clone()
+    y_eager = m.forward(cfg, inputs)
+    torch.cuda.synchronize()
+    assert torch.equal(y_graph, y_eager)
+    del g
