@@ -37,7 +37,6 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer tokens/s; achieved TFLOP/s or HBM GB/s as % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 8  # route, hist, scan, scatter, gather, gate_up GEMM, down GEMM, combine
 # ncu dram bytes (read + write) per launch of the dominant kernel, per workload, from the
 # profile summaries under profiles/ (None until captured for the current kernel version).
 NCU_TRAFFIC = {}
@@ -382,7 +381,7 @@ def run_own(args, cfg):
            "e2e": {"value": e2e_value, "unit": "tokens/s",
                    "h2d_bytes_per_step": x_h.numel() * x_h.element_size() + l_h.numel() * l_h.element_size(),
                    "d2h_bytes_per_step": y_h.numel() * y_h.element_size()},
-           "gpu_launches": KERNELS_PER_STEP * args.steps,
+           "gpu_launches": moe.moe_forward_kernel_count(shape, opts) * args.steps,
            "clocks": clocks}
 
     # ------------------------------------------------------------ CPU baseline (rank 0, N=1)

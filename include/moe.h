@@ -217,6 +217,10 @@ MOE_API int moe_forward_events(const moe_shape *shape, const moe_options *opts, 
 MOE_API int moe_forward_noalloc(const moe_shape *shape, const moe_options *opts, const moe_tensors *t,
                                 void *stream);
 
+/* Number of CUDA kernels one moe_forward of this problem launches (-1 if the
+ * arguments are invalid; 0 for T == 0).  For launch accounting. */
+MOE_API int moe_forward_kernel_count(const moe_shape *shape, const moe_options *opts);
+
 /* Message of the last failed call on this thread ("" if none). */
 MOE_API const char *moe_last_error(void);
 

@@ -75,6 +75,8 @@ MOE_STAGE_EVENTS = 7
 _lib.moe_forward_noalloc.argtypes = [_P(moe_shape), _P(moe_options), _P(moe_tensors), C.c_void_p]
 _lib.moe_forward_noalloc.restype = C.c_int
 MOE_NOALLOC_WORKSPACE_BYTES = 64 << 20
+_lib.moe_forward_kernel_count.argtypes = [_P(moe_shape), _P(moe_options)]
+_lib.moe_forward_kernel_count.restype = C.c_int
 STAGES = ("route", "sort", "gather", "gate_up", "down", "combine")
 _lib.moe_last_error.argtypes = []
 _lib.moe_last_error.restype = C.c_char_p
@@ -84,8 +86,8 @@ _lib.moe_version.argtypes = []
 _lib.moe_version.restype = C.c_char_p
 
 EXPORTED = ("moe_options_init", "moe_workspace_size", "moe_forward", "moe_route",
-            "moe_forward_events", "moe_forward_noalloc", "moe_last_error", "moe_debug_status",
-            "moe_version")
+            "moe_forward_events", "moe_forward_noalloc", "moe_forward_kernel_count",
+            "moe_last_error", "moe_debug_status", "moe_version")
 
 
 class MoeError(RuntimeError):
@@ -126,6 +128,10 @@ def moe_forward_events(shape, opts, tensors, workspace: int, workspace_bytes: in
 def moe_forward_noalloc(shape, opts, tensors, stream: int) -> int:
     """moe_forward on the library's static scratch array (no workspace argument)."""
     return _lib.moe_forward_noalloc(C.byref(shape), C.byref(opts), C.byref(tensors), stream)
+
+
+def moe_forward_kernel_count(shape, opts) -> int:
+    return _lib.moe_forward_kernel_count(C.byref(shape), C.byref(opts))
 
 
 def moe_last_error() -> str:

@@ -8,6 +8,7 @@
 // or a bias without its slot; a dtype it cannot serve is Unsupported), mapped
 // to status codes.
 #include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -227,13 +228,18 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
   gc.act = ActParams{o->act, o->alpha, o->beta, o->limit};
   gc.weigh_inputs = o->weigh_inputs;
   gc.status = status;
+  gc.splits = 1;
+  gc.partial = at<float>(ws, p.o_part);
+  gc.partial_pitch = (int)p.partial_pitch;
   // Upper bound of the M tiles: every non-empty expert adds at most one partial tile.
   const int64_t mt_routed = p.R / p.bm + std::min<int64_t>(p.E, p.R);
   const int64_t mt_shared = p.Fs > 0 ? cdiv(p.T, p.bm) : 0;
   GemmCommon gu = gc, dn = gc;
   gu.tiles = sa.tile_gu;
+  gu.splits = p.splits_gu;
   gu.max_tiles = (int)(mt_routed * p.nt_gu_routed + mt_shared * p.nt_gu_shared);
   dn.tiles = sa.tile_dn;
+  dn.splits = p.splits_dn;
   dn.max_tiles = (int)(mt_routed * p.nt_dn_routed + mt_shared * p.nt_dn_shared);
 
   if (p.tc) {
@@ -256,10 +262,14 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
     ta.c = gu;
     e = fp4 ? launch_fp4_gate_up(ta, st) : launch_tc_gate_up(ta, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core gate_up GEMM");
+    if (gu.splits > 1 && (e = launch_splitk_gate_up_reduce(ta, st)) != cudaSuccess)
+      return cuda_fail(e, "split-K gate_up reduction");
     if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     ta.c = dn;
     e = fp4 ? launch_fp4_down(ta, st) : launch_tc_down(ta, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core down GEMM");
+    if (dn.splits > 1 && (e = launch_splitk_down_reduce(ta, st)) != cudaSuccess)
+      return cuda_fail(e, "split-K down reduction");
   } else {
     SimtArgs sm{};
     sm.x = (const float*)t->x;
@@ -330,6 +340,20 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
     p->nt_gu_shared = (int)cdiv(s->Fs, 32);
     p->nt_dn_routed = p->nt_dn_shared = (int)cdiv(s->d, 64);
   }
+  // split-K for the bf16 tensor-core GEMMs when even the largest possible tile
+  // count leaves SMs idle (small token counts)
+  p->splits_gu = p->splits_dn = 1;
+  p->partial_pitch = 0;
+  if (p->tc && s->w_dtype == MOE_BF16 && p->R <= kSplitMaxRows) {
+    const int sms = num_sms_of_current_device();
+    const int64_t m_bound = std::min<int64_t>(p->E, p->R) + p->R / kTcBM;
+    const int64_t m_shared = p->Fs > 0 ? cdiv(p->T, kTcBM) : 0;
+    const int nkb_dn = (int)std::min<int64_t>(cdiv(p->F, 64), p->Fs > 0 ? cdiv(p->Fs, 64) : INT32_MAX);
+    p->splits_gu = choose_splits(m_bound * p->nt_gu_routed + m_shared * p->nt_gu_shared, (int)cdiv(p->d, 64), sms);
+    p->splits_dn = choose_splits(m_bound * p->nt_dn_routed + m_shared * p->nt_dn_shared, nkb_dn, sms);
+    if (p->splits_gu > 1 || p->splits_dn > 1)
+      p->partial_pitch = (int64_t)std::max({p->nt_gu_routed, p->nt_gu_shared, p->nt_dn_routed}) * 256;
+  }
   const size_t elt = p->tc ? 2 : 4;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -352,6 +376,8 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   p->o_x = take(p->R * p->d * elt);
   p->o_h = take(p->rows * p->Fmax * elt);
   p->o_y = take(p->rows * p->d * elt);
+  p->o_part = take((size_t)std::max(p->splits_gu, p->splits_dn) * p->rows * p->partial_pitch * 4 *
+                   (p->partial_pitch > 0 ? 1 : 0));
   p->total = off;
   return off;
 }
@@ -391,6 +417,15 @@ int moe_route(const moe_shape* s, const moe_options* o, const moe_tensors* t, vo
 int moe_forward_events(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws, size_t ws_bytes,
                        void* stream, void* const* events, int n_events) {
   return moe::run(s, o, t, ws, ws_bytes, stream, true, events, n_events);
+}
+
+int moe_forward_kernel_count(const moe_shape* s, const moe_options* o) {
+  if (moe::check_shape_opts(s, o) != MOE_OK) return -1;
+  if (s->T == 0) return 0;
+  moe::Plan p;
+  moe::make_plan(s, o, &p);
+  // route, histogram, scan, scatter, gather, gate_up, down, combine (+ split-K reductions)
+  return 8 + (p.splits_gu > 1) + (p.splits_dn > 1);
 }
 
 const char* moe_last_error(void) { return moe::g_err.c_str(); }

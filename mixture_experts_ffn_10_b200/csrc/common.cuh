@@ -19,6 +19,7 @@ constexpr int kSimtBM = 64;       // rows per SIMT GEMM tile
 constexpr int kTcBM = 128;        // rows per tensor-core GEMM tile (UMMA M)
 constexpr int kTcGuBN = 128;      // h features per gate_up tile (gate rows + up rows = 256)
 constexpr int kTcDnBN = 256;      // output features per down tile
+constexpr int kSplitMaxRows = 4096;  // split-K only for problems with at most this many routed rows
 
 // ---------------------------------------------------------------- workspace plan
 // Segments: experts 0..E-1 (routed rows, sorted by expert, token-ascending
@@ -37,9 +38,11 @@ struct Plan {
   bool tc;            // tensor-core path (bf16 activations) vs SIMT fp32 path
   int bm;             // GEMM tile rows
   int nt_gu_routed, nt_gu_shared, nt_dn_routed, nt_dn_shared;  // N tiles per segment
+  int splits_gu, splits_dn;  // split-K factors of the two GEMMs (1 = none)
+  int64_t partial_pitch;     // floats per row of the split-K partial buffer
   // byte offsets into the workspace
   size_t o_status, o_idx, o_w, o_hist, o_cnt, o_off, o_tgu, o_tdn, o_pos, o_perm, o_roww,
-      o_sgate, o_x, o_h, o_y, total;
+      o_sgate, o_x, o_h, o_y, o_part, total;
 };
 
 // Fills `p` from validated arguments; returns the workspace size.
@@ -168,6 +171,12 @@ struct GemmCommon {
   ActParams act;
   int weigh_inputs;
   int* status;
+  // split-K: each tile's K range is cut into `splits` parts whose fp32 partial
+  // accumulators go to partial[split][row][n_blk * 256 + col] (pitch floats per
+  // row); a reduce kernel then sums them in split order and runs the epilogue.
+  int splits;
+  float* partial;
+  int partial_pitch;
 };
 
 struct SimtArgs {
@@ -206,6 +215,11 @@ struct TcArgs {
 };
 cudaError_t launch_tc_gate_up(const TcArgs& a, cudaStream_t st);
 cudaError_t launch_tc_down(const TcArgs& a, cudaStream_t st);
+// Split-K reductions (partials -> epilogue) for the bf16 tensor-core GEMMs.
+cudaError_t launch_splitk_gate_up_reduce(const TcArgs& a, cudaStream_t st);
+cudaError_t launch_splitk_down_reduce(const TcArgs& a, cudaStream_t st);
+// Split count for a GEMM of at most `tiles` tiles of `nkb` k-blocks on `sms` SMs.
+int choose_splits(int64_t tiles, int nkb, int sms);
 // MXFP4 expert stacks (gate_up / down are e2m1 codes); no shared expert.
 cudaError_t launch_fp4_gate_up(const TcArgs& a, cudaStream_t st);
 cudaError_t launch_fp4_down(const TcArgs& a, cudaStream_t st);

@@ -100,7 +100,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = c.tiles[c.NS];
+  // Work units: (tile, split).  Split sp of a tile covers k-blocks
+  // [sp * nkb / S, (sp + 1) * nkb / S) of the tile's K range.
+  const int S = c.splits;
+  const int total = c.tiles[c.NS] * S;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -126,10 +129,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const Tile t = decode_tile<BM>(c, tile);
+      for (int unit = blockIdx.x; ok && unit < total; unit += gridDim.x) {
+        const Tile t = decode_tile<BM>(c, unit / S);
         const int nkb = (k_extent<MODE>(c, t.seg >= c.E) + BK - 1) / BK;
-        for (int kb = 0; kb < nkb; kb++, it++) {
+        const int sp = unit % S, kb1 = (sp + 1) * nkb / S;
+        for (int kb = sp * nkb / S; kb < kb1; kb++, it++) {
           const int s = it % STAGES;
           if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, c.status)) {
             ok = false;
@@ -151,15 +155,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, tcount++) {
-        const Tile t = decode_tile<BM>(c, tile);
+      for (int unit = blockIdx.x; ok && unit < total; unit += gridDim.x, tcount++) {
+        const Tile t = decode_tile<BM>(c, unit / S);
         const bool sh = t.seg >= c.E;
         const int nkb = (k_extent<MODE>(c, sh) + BK - 1) / BK;
+        const int sp = unit % S, kb0 = sp * nkb / S, kb1 = (sp + 1) * nkb / S;
         const int acc = tcount & 1;
         if (!mbar_wait(&tempty[acc], ((tcount >> 1) & 1) ^ 1, abort_flag, c.status)) break;
         tc_fence_after();
         const uint32_t dt = tmem_base + acc * ACC_COLS;
-        for (int kb = 0; kb < nkb; kb++, it++) {
+        for (int kb = kb0; kb < kb1; kb++, it++) {
           const int s = it % STAGES;
           if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag, c.status)) {
             ok = false;
@@ -170,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t ad = sdesc_k_sw128(sa), bd = sdesc_k_sw128(sa + A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; kk++)
-            mma_bf16(dt, ad + 2 * kk, bd + 2 * kk, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            mma_bf16(dt, ad + 2 * kk, bd + 2 * kk, IDESC, (kb > kb0 || kk > 0) ? 1u : 0u);
           mma_commit(&empty[s]);
         }
         if (ok) mma_commit(&tfull[acc]);
@@ -187,8 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int part = (warp - 2) / 4;   // which alternate column chunks this warp drains
     const int r_in_tile = q * 32 + lane;
     uint32_t tcount = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, tcount++) {
-      const Tile t = decode_tile<BM>(c, tile);
+    for (int unit = blockIdx.x; unit < total; unit += gridDim.x, tcount++) {
+      const Tile t = decode_tile<BM>(c, unit / S);
       const bool sh = t.seg >= c.E;
       const int acc = tcount & 1;
       if (!mbar_wait(&tfull[acc], (tcount >> 1) & 1, abort_flag, c.status)) break;
@@ -197,7 +202,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = t.m0 + r_in_tile;
       const bool valid = row < t.rows;
       const int64_t grow = (int64_t)c.off[t.seg] + row;
-      if (__any_sync(0xffffffffu, valid)) {
+      if (S > 1) {
+        // split-K: this unit's fp32 partial accumulator row goes to the partial buffer
+        if (__any_sync(0xffffffffu, valid)) {
+          float* prow = c.partial + ((int64_t)(unit % S) * (c.R + (c.Fs > 0 ? c.T : 0)) + grow) * c.partial_pitch +
+                        t.n_blk * ACC_COLS;
+#pragma unroll 1
+          for (int ch = part; ch < ACC_COLS / 16; ch += 2) {
+            uint32_t v[16];
+            tmem_ld16(tb + ch * 16, v);
+            tmem_ld_wait();
+            if (valid) {
+              float4* dst = reinterpret_cast<float4*>(prow + ch * 16);
+#pragma unroll
+              for (int i = 0; i < 4; i++)
+                dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                     __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            }
+          }
+        }
+      } else if (__any_sync(0xffffffffu, valid)) {
         if (MODE == 0) {
           const int F = sh ? c.Fs : c.F;
           const int f0 = t.n_blk * (BNB / 2);
@@ -286,7 +310,8 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMa
   cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int grid = p.c.max_tiles < num_sms ? p.c.max_tiles : num_sms;
+  const int units = p.c.max_tiles * p.c.splits;
+  const int grid = units < num_sms ? units : num_sms;
   tc_gemm_kernel<MODE><<<grid, kThreads, SMEM_BYTES, st>>>(a, as, b, bs, p);
   return cudaGetLastError();
 }

@@ -26,7 +26,8 @@ def _declared():
 def test_header_declares_the_entry_points():
     assert _declared() == sorted(["moe_options_init", "moe_workspace_size", "moe_forward",
                                   "moe_route", "moe_forward_events", "moe_forward_noalloc",
-                                  "moe_last_error", "moe_debug_status", "moe_version"])
+                                  "moe_forward_kernel_count", "moe_last_error", "moe_debug_status",
+                                  "moe_version"])
 
 
 def test_library_exports_every_declared_symbol(moe):

@@ -51,6 +51,10 @@ CASES = {
     "k_equals_E": small(MIX, name="k_equals_E", E=4, k=4, renormalize=False),
     "ragged_d_F": small(MIX, name="ragged_d_F", d=72, F=40, Fs=24, T=70),
     "many_experts": small(MIX, name="many_experts", E=256, k=8, T=64, d=128, F=64),
+    "tiny_batch_shared_expert": small(DSK, name="tiny_batch_shared_expert", T=4, shared_gate=True,
+                                      expert_bias=True),
+    "tiny_batch_interleaved": small(MIX, name="tiny_batch_interleaved", T=8, gu_layout="interleaved",
+                                    act="gelu_tanh", expert_bias=True, weigh_inputs=True),
     "gptoss_mxfp4_small": FP4,
     "mxfp4_concat": small(FP4, name="mxfp4_concat", gu_layout="concat", limit=0.0, alpha=1.0),
     "mxfp4_T1_many_experts": small(FP4, name="mxfp4_T1_many_experts", T=1, E=32, k=4),
