@@ -348,8 +348,8 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
     const int sms = num_sms_of_current_device();
     const int64_t m_bound = std::min<int64_t>(p->E, p->R) + p->R / kTcBM;
     const int64_t m_shared = p->Fs > 0 ? cdiv(p->T, kTcBM) : 0;
-    const int nkb_dn = (int)std::min<int64_t>(cdiv(p->F, 64), p->Fs > 0 ? cdiv(p->Fs, 64) : INT32_MAX);
-    p->splits_gu = choose_splits(m_bound * p->nt_gu_routed + m_shared * p->nt_gu_shared, (int)cdiv(p->d, 64), sms);
+    const int nkb_dn = (int)std::min<int64_t>(cdiv(p->F, kTcBK), p->Fs > 0 ? cdiv(p->Fs, kTcBK) : INT32_MAX);
+    p->splits_gu = choose_splits(m_bound * p->nt_gu_routed + m_shared * p->nt_gu_shared, (int)cdiv(p->d, kTcBK), sms);
     p->splits_dn = choose_splits(m_bound * p->nt_dn_routed + m_shared * p->nt_dn_shared, nkb_dn, sms);
     if (p->splits_gu > 1 || p->splits_dn > 1)
       p->partial_pitch = (int64_t)std::max({p->nt_gu_routed, p->nt_gu_shared, p->nt_dn_routed}) * 256;

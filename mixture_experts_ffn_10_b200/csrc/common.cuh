@@ -19,6 +19,7 @@ constexpr int kSimtBM = 64;       // rows per SIMT GEMM tile
 constexpr int kTcBM = 128;        // rows per tensor-core GEMM tile (UMMA M)
 constexpr int kTcGuBN = 128;      // h features per gate_up tile (gate rows + up rows = 256)
 constexpr int kTcDnBN = 256;      // output features per down tile
+constexpr int kTcBK = 64;         // K elements per pipeline stage of the bf16 tensor-core GEMMs
 constexpr int kSplitMaxRows = 4096;  // split-K only for problems with at most this many routed rows
 
 // ---------------------------------------------------------------- workspace plan

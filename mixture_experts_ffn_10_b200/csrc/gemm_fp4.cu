@@ -11,12 +11,14 @@
 // Tile: 256 activation rows (two M=128 halves) x 128 weight rows x K, fp32 in TMEM
 // (2 halves x 128 columns, double-buffered).  Both halves share each decoded
 // weight stage, halving the decode work per FLOP.  Warp roles:
-//   warp 0      TMA: activations 256 x 64 (bf16, 128B swizzle) and codes 128 x 32 B
+//   warp 0      TMA producer of activations 256 x 64 (bf16, 128B swizzle)
 //   warp 1      TMEM owner and MMA issuer (M=128 N=128 K=16 per half)
+//   warp 26     TMA producer of the codes, 128 x 32 bytes, running up to 6 stages ahead
 //   warps 2-9   epilogue (bias + activation, or bias x routing weight; bf16 stores);
 //               warps 2-5 drain the first M half, warps 6-9 the second
-//   warps 10-25 converters: codes + scale -> bf16 in the 128B-swizzled K-major layout
-//               the MMA descriptor reads, then a proxy fence and one arrive per warp.
+//   warps 10-25 converters in four groups, group g owning stages it % 4 == g:
+//               codes + scale -> bf16 in the 128B-swizzled K-major layout the MMA
+//               descriptor reads, then a proxy fence and one arrive per warp.
 // Decode: the hardware conversion cvt.rn.f16x2.e2m1x2 turns each code byte into two
 // exact f16 values; shifting an f16's exponent and mantissa right by 3 bits (sign
 // kept) gives a bf16 of the same value times 2^-112, and one bf16x2 multiply by
@@ -38,20 +40,25 @@ constexpr int BM = kFp4BM;              // 256 = 2 x 128
 constexpr int HALF = 128;
 constexpr int BK = 64;                  // K elements per stage
 constexpr int BNB = 128;                // weight rows per tile
-constexpr int STAGES = 4;
+// Three rings, so that decoding never holds an activation slot:
+constexpr int AST = 4;                  // activations: 256 x 64 bf16, freed by the MMA
+constexpr int QST = 6;                  // e2m1 codes: 128 x 32 bytes, freed once converted
+constexpr int WST = 4;                  // decoded bf16 weights: 128 x 64, freed by the MMA
 constexpr int A_BYTES = BM * BK * 2;    // 32 KiB
-constexpr int Q_BYTES = BNB * BK / 2;   // 4 KiB of codes
-constexpr int W_BYTES = BNB * BK * 2;   // 16 KiB decoded bf16
-constexpr int STAGE_BYTES = A_BYTES + Q_BYTES + W_BYTES;
+constexpr int Q_BYTES = BNB * BK / 2;   // 4 KiB
+constexpr int W_BYTES = BNB * BK * 2;   // 16 KiB
+constexpr int RING_BYTES = AST * A_BYTES + WST * W_BYTES + QST * Q_BYTES;
 constexpr int ACC_COLS = 2 * BNB;       // two halves
 constexpr int TMEM_COLS = 2 * ACC_COLS; // double-buffered
 constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant: one per M half
 constexpr int kCvtWarps = 16;
-constexpr int kCvtThreads = kCvtWarps * 32;  // 16 elements (8 code bytes) per thread and stage
-constexpr int kThreads = 64 + (kEpiWarps + kCvtWarps) * 32;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int kCvtGroups = 4;                // converter groups, each owning every 4th stage
+constexpr int kCvtGroupWarps = kCvtWarps / kCvtGroups;
+constexpr int kThreads = 64 + (kEpiWarps + kCvtWarps + 1) * 32;  // + the codes producer warp
+constexpr int SMEM_BYTES = RING_BYTES + 1024 + 512;
 constexpr uint32_t IDESC = idesc_bf16_f32(HALF, BNB);
-static_assert(kCvtThreads == BNB * (BK / 16), "one converter thread per (row, 16 elements)");
+static_assert(kCvtGroupWarps * 32 == BNB, "one converter thread per weight row in a group");
+static_assert(WST % kCvtGroups == 0, "a group's stages map to its own decoded-weight slots");
 
 struct Fp4Params {
   GemmCommon c;
@@ -128,10 +135,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const Fp4Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint64_t* conv = full + STAGES;
-  uint64_t* empty = conv + STAGES;
-  uint64_t* tfull = empty + STAGES;
+  uint8_t* ringA = smem;                                   // AST x 32 KiB (1024-aligned)
+  uint8_t* ringW = ringA + AST * A_BYTES;                  // WST x 16 KiB (1024-aligned)
+  uint8_t* ringQ = ringW + WST * W_BYTES;                  // QST x 4 KiB
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + RING_BYTES);
+  uint64_t* emptyA = fullA + AST;
+  uint64_t* fullW = emptyA + AST;
+  uint64_t* emptyW = fullW + WST;
+  uint64_t* fullQ = emptyW + WST;
+  uint64_t* emptyQ = fullQ + QST;
+  uint64_t* tfull = emptyQ + QST;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -139,12 +152,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const GemmCommon& c = p.c;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kCodesWarp = 2 + kEpiWarps + kCvtWarps;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; s++) {
-      mbar_init(&full[s], 1);
-      mbar_init(&conv[s], kCvtWarps);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < AST; s++) {
+      mbar_init(&fullA[s], 1);
+      mbar_init(&emptyA[s], 1);
+    }
+    for (int s = 0; s < WST; s++) {
+      mbar_init(&fullW[s], kCvtGroupWarps);
+      mbar_init(&emptyW[s], 1);
+    }
+    for (int s = 0; s < QST; s++) {
+      mbar_init(&fullQ[s], 1);
+      mbar_init(&emptyQ[s], kCvtGroupWarps);
     }
     for (int b = 0; b < 2; b++) {
       mbar_init(&tfull[b], 1);
@@ -168,42 +189,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int K = k_extent<MODE>(c);
   const int nkb = (K + BK - 1) / BK;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == kCodesWarp) {
+    // ------------------------------------------------------------ TMA producers
     if (lane == 0) {
-      auto issue = [&](const Tile& t, int kb, uint64_t* bar, uint8_t* sa) {
-        const int arow = c.off[t.seg] + t.m0;
-        uint8_t* sq = sa + A_BYTES;
-        const int ka = kb * BK, kq = kb * (BK / 2);
-        tma_load_2d(&tmA, bar, sa, ka, arow);
-        if (MODE == 0) {
-          const int f0 = t.n_blk * (BNB / 2);
-          const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
-          for (int half = 0; half < 2; half++) {
-            const int c1 = il ? half : f0, c2 = il ? f0 : half;
-            tma_load_4d(&tmQ, bar, sq + half * (Q_BYTES / 2), kq, c1, c2, t.seg);
-          }
-        } else {
-          tma_load_3d(&tmQ, bar, sq, kq, t.n_blk * BNB, t.seg);
-        }
-      };
+      const bool codes = warp == kCodesWarp;
+      const int depth = codes ? QST : AST;
+      uint64_t* full = codes ? fullQ : fullA;
+      uint64_t* empty = codes ? emptyQ : emptyA;
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         const Tile t = decode_tile<BM>(c, tile);
         for (int kb = 0; kb < nkb; kb++, it++) {
-          const int s = it % STAGES;
-          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, c.status)) {
+          const int s = it % depth;
+          if (!mbar_wait(&empty[s], ((it / depth) & 1) ^ 1, abort_flag, c.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], A_BYTES + Q_BYTES);
-          issue(t, kb, &full[s], smem + s * STAGE_BYTES);
+          if (!codes) {
+            mbar_arrive_expect_tx(&full[s], A_BYTES);
+            tma_load_2d(&tmA, &full[s], ringA + s * A_BYTES, kb * BK, c.off[t.seg] + t.m0);
+          } else {
+            uint8_t* sq = ringQ + s * Q_BYTES;
+            mbar_arrive_expect_tx(&full[s], Q_BYTES);
+            const int kq = kb * (BK / 2);
+            if (MODE == 0) {
+              const int f0 = t.n_blk * (BNB / 2);
+              const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
+              for (int half = 0; half < 2; half++)
+                tma_load_4d(&tmQ, &full[s], sq + half * (Q_BYTES / 2), kq, il ? half : f0, il ? f0 : half, t.seg);
+            } else {
+              tma_load_3d(&tmQ, &full[s], sq, kq, t.n_blk * BNB, t.seg);
+            }
+          }
         }
       }
-      for (uint32_t j = (it > (uint32_t)STAGES ? it - STAGES : 0); j < it; j++) {
+      // every load issued into a slot has landed before the CTA may exit
+      for (uint32_t j = (it > (uint32_t)depth ? it - depth : 0); j < it; j++) {
         const uint64_t t0 = global_timer();
-        while (!mbar_try_wait(&full[j % STAGES], (j / STAGES) & 1) && global_timer() - t0 < kTimeoutNs) {
+        while (!mbar_try_wait(&full[j % depth], (j / depth) & 1) && global_timer() - t0 < kTimeoutNs) {
         }
       }
     }
@@ -220,23 +244,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t dt = tmem_base + acc * ACC_COLS;
         for (int kb = 0; kb < nkb; kb++, it++) {
-          const int s = it % STAGES;
-          if (!mbar_wait(&conv[s], (it / STAGES) & 1, abort_flag, c.status)) {
+          const int sa = it % AST, sw = it % WST;
+          if (!mbar_wait(&fullA[sa], (it / AST) & 1, abort_flag, c.status) ||
+              !mbar_wait(&fullW[sw], (it / WST) & 1, abort_flag, c.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
-          const uint64_t bd = sdesc_k_sw128(sa + A_BYTES + Q_BYTES);
+          const uint64_t bd = sdesc_k_sw128(smem_u32(ringW + sw * W_BYTES));
 #pragma unroll
           for (int h = 0; h < 2; h++) {
             if (h == 1 && !two) break;
-            const uint64_t ad = sdesc_k_sw128(sa + h * (HALF * BK * 2));
+            const uint64_t ad = sdesc_k_sw128(smem_u32(ringA + sa * A_BYTES + h * (HALF * BK * 2)));
 #pragma unroll
             for (int kk = 0; kk < BK / 16; kk++)
               mma_bf16(dt + h * BNB, ad + 2 * kk, bd + 2 * kk, IDESC, (kb | kk) != 0 ? 1u : 0u);
           }
-          mma_commit(&empty[s]);
+          mma_commit(&emptyA[sa]);
+          mma_commit(&emptyW[sw]);
         }
         if (ok) mma_commit(&tfull[acc]);
       }
@@ -292,62 +317,73 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
-  } else {
+  } else if (warp < kCodesWarp) {
     // ------------------------------------------------------------ converters
-    // Lane layout: 8 weight rows x 4 quarters (16 elements each) per warp, so the
-    // 8-byte code loads cover 256 contiguous bytes and the swizzled 16-byte stores
-    // of a quarter-warp hit distinct banks.
+    // Four groups of four warps; group g converts the stages it with it % 4 == g,
+    // so four stages are in conversion at once.  In a group, thread = weight row:
+    // it loads the row's 32 code bytes, decodes 64 elements with the row's two
+    // block scales and writes the 128-byte row in the swizzled layout (the 8
+    // consecutive rows of a quarter-warp hit distinct banks).
     const int cw = warp - 2 - kEpiWarps;         // 0 .. kCvtWarps-1
-    const int r = cw * 8 + (lane >> 2);          // weight row inside the tile
-    const int g = lane & 3;                      // quarter of the 64-element stage
-    const int b = g >> 1;                        // 32-element scale block
+    const int group = cw / kCvtGroupWarps;       // 0 .. kCvtGroups-1
+    const int r = (cw % kCvtGroupWarps) * 32 + lane;  // weight row inside the tile
     const int kblocks = K / 32;                  // scale bytes per weight row
     const int rows_per_e = MODE == 0 ? 2 * c.F : c.d;
-    uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    uint32_t it = 0;  // stage index of the tile's first k-block
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, it += nkb) {
       const Tile t = decode_tile<BM>(c, tile);
       bool rvalid;
       const int wr = weight_row<MODE>(c, t.n_blk, r, &rvalid);
       const uint8_t* srow = p.scales + ((int64_t)t.seg * rows_per_e + wr) * kblocks;
-      // scale bytes of this thread's block for k-blocks kb .. kb+3, loaded ahead
-      auto load_scale = [&](int kb) -> uint32_t {
-        const int col = kb * 2 + b;
-        return (rvalid && kb < nkb && col < kblocks) ? (uint32_t)__ldg(srow + col) : 127u;
+      auto load_scales = [&](int kb) -> uint32_t {  // the row's two block scales of k-block kb
+        if (!rvalid || kb >= nkb) return 127u | (127u << 8);
+        const int col = kb * 2;
+        const uint32_t lo = col < kblocks ? __ldg(srow + col) : 127u;
+        const uint32_t hi = col + 1 < kblocks ? __ldg(srow + col + 1) : 127u;
+        return lo | (hi << 8);
       };
-      uint32_t s0 = load_scale(0), s1 = load_scale(1), s2 = load_scale(2), s3 = load_scale(3);
+      int kb = (int)((group - (int)(it % kCvtGroups) + kCvtGroups) % kCvtGroups);
+      uint32_t sc = load_scales(kb);
       bool ok = true;
-      for (int kb = 0; kb < nkb; kb++, it++) {
-        const uint32_t s4 = load_scale(kb + 4);
-        const int st = it % STAGES;
-        if (!mbar_wait(&full[st], (it / STAGES) & 1, abort_flag, c.status)) {
+      for (; kb < nkb; kb += kCvtGroups) {
+        const uint32_t next = load_scales(kb + kCvtGroups);
+        const uint32_t st = it + kb;
+        const int sq = st % QST, sw = st % WST;
+        if (!mbar_wait(&fullQ[sq], (st / QST) & 1, abort_flag, c.status)) {
           ok = false;
           break;
         }
-        uint8_t* base = smem + st * STAGE_BYTES;
-        const uint2 q = *reinterpret_cast<const uint2*>(base + A_BYTES + r * (BK / 2) + g * 8);
-        uint8_t* wrow = base + A_BYTES + Q_BYTES + r * (BK * 2);
-        uint32_t extra;
-        const uint32_t sc = scale_bf16x2(s0, &extra);
-        const uint32_t words[2] = {q.x, q.y};
+        const uint4* qrow = reinterpret_cast<const uint4*>(ringQ + sq * Q_BYTES + r * (BK / 2));
+        const uint4 q0 = qrow[0], q1 = qrow[1];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&emptyQ[sq]);  // codes are in registers: the slot may refill
+        if (!mbar_wait(&emptyW[sw], ((st / WST) & 1) ^ 1, abort_flag, c.status)) {
+          ok = false;
+          break;
+        }
+        uint8_t* wrow = ringW + sw * W_BYTES + r * (BK * 2);
+        const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-        for (int wi = 0; wi < 2; wi++) {
-          uint32_t h[4], o[4];
-          e2m1x8_to_f16x8(words[wi], h);
+        for (int blk = 0; blk < 2; blk++) {
+          uint32_t extra;
+          const uint32_t scale = scale_bf16x2((sc >> (8 * blk)) & 0xFF, &extra);
 #pragma unroll
-          for (int i = 0; i < 4; i++) {
-            o[i] = bmul(f16x2_to_bf16x2_biased(h[i]), sc);
-            if (extra) o[i] = bmul(o[i], extra);
+          for (int wi = 0; wi < 4; wi++) {
+            uint32_t h[4], o[4];
+            e2m1x8_to_f16x8(words[blk * 4 + wi], h);
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+              o[i] = bmul(f16x2_to_bf16x2_biased(h[i]), scale);
+              if (extra) o[i] = bmul(o[i], extra);
+            }
+            const int chunk = blk * 4 + wi;  // 16-byte chunk (8 elements) of the 128-byte row
+            *reinterpret_cast<uint4*>(wrow + ((chunk ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
           }
-          const int chunk = g * 2 + wi;  // 16-byte chunk (8 elements) of the 128-byte row
-          *reinterpret_cast<uint4*>(wrow + ((chunk ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&conv[st]);
-        s0 = s1;
-        s1 = s2;
-        s2 = s3;
-        s3 = s4;
+        if (lane == 0) mbar_arrive(&fullW[sw]);
+        sc = next;
       }
       if (!ok) break;
     }

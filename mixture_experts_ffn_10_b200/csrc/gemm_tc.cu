@@ -31,9 +31,16 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = kTcBM;            // 128
-constexpr int BK = 64;               // one 128-byte swizzle row of bf16
+#ifndef MOE_TC_BK
+#define MOE_TC_BK 64
+#endif
+constexpr int BK = MOE_TC_BK;        // K per stage: 64 (128-byte rows, 4 stages); 32 (64-byte rows, 8 stages) measured slower
 constexpr int BNB = 256;             // B rows per tile
-constexpr int STAGES = 4;
+constexpr int STAGES = BK == 32 ? 8 : 4;
+constexpr CUtensorMapSwizzle kSwizzle = BK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+  return BK == 32 ? sdesc_k_sw64(saddr) : sdesc_k_sw128(saddr);
+}
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BNB * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -172,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
-          const uint64_t ad = sdesc_k_sw128(sa), bd = sdesc_k_sw128(sa + A_BYTES);
+          const uint64_t ad = sdesc(sa), bd = sdesc(sa + A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; kk++)
             mma_bf16(dt, ad + 2 * kk, bd + 2 * kk, IDESC, (kb > kb0 || kk > 0) ? 1u : 0u);
@@ -267,11 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- host side
 
-// bf16 tensor map with the 128-byte swizzle the UMMA descriptors expect.
+// bf16 tensor map with the swizzle the UMMA descriptors expect.
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
               const uint32_t* box) {
-  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides, box,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides, box, kSwizzle);
 }
 
 // rows x K matrix with row pitch `pitch` elements; box 64 x box_rows.
