@@ -14,9 +14,8 @@
 //              swizzle) per stage into a 4-stage shared-memory ring;
 //   warp 1     TMEM allocator and MMA issuer: tcgen05.mma M=128 N=256 K=16,
 //              fp32 accumulators in TMEM, two accumulator buffers of 256 columns;
-//   warps 2-9  epilogue: tcgen05.ld the accumulator rows, bias + activation (or
+//   warps 2-5  epilogue: tcgen05.ld the accumulator rows, bias + activation (or
 //              bias x routing weight), bf16 stores; overlaps the next tile's MMAs.
-//              Warps w and w+4 share a TMEM lane quadrant and alternate chunks.
 // For gate_up the B tile is 128 gate rows followed by the 128 matching up rows,
 // fetched through a 4-D tensor map view of the stack that hides the layout:
 // concat [E][2][F][d] or interleaved [E][F][2][d].  So accumulator column j
@@ -46,7 +45,11 @@ constexpr int B_BYTES = BNB * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
-constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, splitting the column chunks
+#ifndef MOE_TC_EPI_WARPS
+#define MOE_TC_EPI_WARPS 4
+#endif
+constexpr int kEpiWarps = MOE_TC_EPI_WARPS;  // 4, or 8 = two per TMEM lane quadrant splitting the chunks
+constexpr int kEpiGroups = kEpiWarps / 4;
 constexpr int kThreads = 64 + kEpiWarps * 32;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BNB);
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float* prow = c.partial + ((int64_t)(unit % S) * (c.R + (c.Fs > 0 ? c.T : 0)) + grow) * c.partial_pitch +
                         t.n_blk * ACC_COLS;
 #pragma unroll 1
-          for (int ch = part; ch < ACC_COLS / 16; ch += 2) {
+          for (int ch = part; ch < ACC_COLS / 16; ch += kEpiGroups) {
             uint32_t v[16];
             tmem_ld16(tb + ch * 16, v);
             tmem_ld_wait();
@@ -236,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
           uint16_t* out = p.out + grow * c.Fmax;
 #pragma unroll 1
-          for (int ch = part; ch < (BNB / 2) / 16; ch += 2) {
+          for (int ch = part; ch < (BNB / 2) / 16; ch += kEpiGroups) {
             uint32_t g[16], u[16];
             tmem_ld16(tb + ch * 16, g);
             tmem_ld16(tb + BNB / 2 + ch * 16, u);
@@ -250,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float w = (sh || c.weigh_inputs || !valid) ? 1.f : p.roww[grow];
           uint16_t* out = p.out + grow * c.d;
 #pragma unroll 1
-          for (int ch = part; ch < BNB / 16; ch += 2) {
+          for (int ch = part; ch < BNB / 16; ch += kEpiGroups) {
             uint32_t v[16];
             tmem_ld16(tb + ch * 16, v);
             tmem_ld_wait();
