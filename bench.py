@@ -39,7 +39,12 @@ METRIC = "MoE layer tokens/s; achieved TFLOP/s or HBM GB/s as % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu dram bytes (read + write) per launch of the dominant kernel, per workload, from the
 # profile summaries under profiles/ (None until captured for the current kernel version).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {  # profiles/tc_gemm_mixtral_shape_E2.md, profiles/tc_fp4_gptoss.md
+    ("mixtral_bf16", "gate_up"): 1951094016 + 229368064,
+    ("mixtral_bf16", "down"): 1437665024 + 73983744,
+    ("gptoss_mxfp4", "gate_up"): 330280192 + 39711488,
+    ("gptoss_mxfp4", "down"): 188636416 + 26926080,
+}
 
 
 def peaks():
@@ -354,8 +359,10 @@ def run_own(args, cfg):
         achieved, peak, unit, bound = m["flops"] / t_dom / 1e12, pk["bf16_tflops"], "TFLOP/s", "tensor"
     else:
         achieved, peak, unit, bound = m["bytes"] / t_dom / 1e9, pk["hbm_gbs"], "GB/s", "hbm"
+    sustained = pk["bf16_tflops_sustained"] if bound == "tensor" else None
     roofline = {"bound": bound, "kernel": f"{dom} grouped GEMM", "achieved": achieved, "peak": peak,
                 "unit": unit, "frac": achieved / peak, "peak_source": f"{pk_src} (burst)",
+                "frac_vs_sustained_peak": (achieved / sustained) if sustained else None,
                 "traffic": NCU_TRAFFIC.get((cfg.name, dom)),
                 "algorithmic_per_launch": m["flops"] if bound == "tensor" else m["bytes"]}
     layer_flops = flops(cfg)
