@@ -168,6 +168,11 @@ MOE_API size_t moe_workspace_size(const moe_shape *shape, const moe_options *opt
  * Errors: MOE_ERR_NULL / SHAPE / DTYPE / ALIGN / ARG / UNSUPPORTED / WORKSPACE
  * before any launch; MOE_ERR_CUDA if a launch fails.  T == 0 is a no-op.
  * Results are bitwise reproducible run to run for the same inputs.
+ * Kernel choice: with bf16 weights and on average >= 512 routed rows per
+ * expert (and T*k > 4096) the GEMMs run on CTA pairs (256-row tiles over two
+ * SMs); the environment variable MOE_B200_PAIR_GEMM=0 or =1, read at every
+ * call, forces the single-CTA or the pair kernels.  Set it before
+ * moe_workspace_size: the two choices may need different workspace sizes.
  */
 MOE_API int moe_forward(const moe_shape *shape, const moe_options *opts, const moe_tensors *t,
                 void *workspace, size_t workspace_bytes, void *stream);

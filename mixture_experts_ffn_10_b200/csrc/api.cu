@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -260,13 +261,13 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
     ta.down_scales = t->down_scales;
     const bool fp4 = s->w_dtype == MOE_MXFP4;
     ta.c = gu;
-    e = fp4 ? launch_fp4_gate_up(ta, st) : launch_tc_gate_up(ta, st);
+    e = fp4 ? launch_fp4_gate_up(ta, st) : p.pair ? launch_tc2_gate_up(ta, st) : launch_tc_gate_up(ta, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core gate_up GEMM");
     if (gu.splits > 1 && (e = launch_splitk_gate_up_reduce(ta, st)) != cudaSuccess)
       return cuda_fail(e, "split-K gate_up reduction");
     if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     ta.c = dn;
-    e = fp4 ? launch_fp4_down(ta, st) : launch_tc_down(ta, st);
+    e = fp4 ? launch_fp4_down(ta, st) : p.pair ? launch_tc2_down(ta, st) : launch_tc_down(ta, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core down GEMM");
     if (dn.splits > 1 && (e = launch_splitk_down_reduce(ta, st)) != cudaSuccess)
       return cuda_fail(e, "split-K down reduction");
@@ -307,6 +308,16 @@ int forward_on_workspace(const moe_shape* s, const moe_options* o, const moe_ten
 
 int set_error(int code, const char* msg) { return fail(code, "%s", msg); }
 
+// CTA-pair GEMMs for large batches: every expert then has several 256-row
+// tiles on average, and the pair kernel needs a third less TMA traffic per SM.
+// MOE_B200_PAIR_GEMM=0 or 1 overrides the choice (bf16 weights only).
+bool use_pair_gemm(int64_t R, int64_t E) {
+  const char* env = std::getenv("MOE_B200_PAIR_GEMM");
+  if (env && env[0] == '0') return false;
+  if (env && env[0] == '1') return true;
+  return R > kSplitMaxRows && R >= (int64_t)kPairMinRows * E;
+}
+
 size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   (void)o;
   p->T = s->T;
@@ -324,13 +335,14 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   p->w_dtype = s->w_dtype;
   p->logit_dtype = s->logit_dtype;
   p->tc = s->act_dtype == MOE_BF16;
+  p->pair = p->tc && s->w_dtype == MOE_BF16 && use_pair_gemm(p->R, s->E);
   if (s->w_dtype == MOE_MXFP4) {
     p->bm = kFp4BM;
     p->nt_gu_routed = (int)cdiv(s->F, kFp4GuBN);
     p->nt_dn_routed = (int)cdiv(s->d, kFp4DnBN);
     p->nt_gu_shared = p->nt_dn_shared = 0;
   } else if (p->tc) {
-    p->bm = kTcBM;
+    p->bm = p->pair ? kPairBM : kTcBM;
     p->nt_gu_routed = (int)cdiv(s->F, kTcGuBN);
     p->nt_gu_shared = (int)cdiv(s->Fs, kTcGuBN);
     p->nt_dn_routed = p->nt_dn_shared = (int)cdiv(s->d, kTcDnBN);
@@ -344,7 +356,7 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   // count leaves SMs idle (small token counts)
   p->splits_gu = p->splits_dn = 1;
   p->partial_pitch = 0;
-  if (p->tc && s->w_dtype == MOE_BF16 && p->R <= kSplitMaxRows) {
+  if (p->tc && s->w_dtype == MOE_BF16 && !p->pair && p->R <= kSplitMaxRows) {
     const int sms = num_sms_of_current_device();
     const int64_t m_bound = std::min<int64_t>(p->E, p->R) + p->R / kTcBM;
     const int64_t m_shared = p->Fs > 0 ? cdiv(p->T, kTcBM) : 0;

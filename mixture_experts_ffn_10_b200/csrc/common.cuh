@@ -17,6 +17,8 @@ constexpr int kMaxGroups = 32;    // groups (one lane each)
 constexpr int kChunkTokens = 64;  // tokens per histogram / scatter chunk
 constexpr int kSimtBM = 64;       // rows per SIMT GEMM tile
 constexpr int kTcBM = 128;        // rows per tensor-core GEMM tile (UMMA M)
+constexpr int kPairBM = 256;      // rows per CTA-pair tile (UMMA M over two SMs)
+constexpr int kPairMinRows = 512; // CTA pairs when routed rows per expert average at least this
 constexpr int kTcGuBN = 128;      // h features per gate_up tile (gate rows + up rows = 256)
 constexpr int kTcDnBN = 256;      // output features per down tile
 constexpr int kTcBK = 64;         // K elements per pipeline stage of the bf16 tensor-core GEMMs
@@ -37,6 +39,7 @@ struct Plan {
   int64_t nchunks;    // ceil(T / kChunkTokens)
   int act_dtype, w_dtype, logit_dtype;
   bool tc;            // tensor-core path (bf16 activations) vs SIMT fp32 path
+  bool pair;          // bf16 GEMMs on CTA pairs (256-row tiles)
   int bm;             // GEMM tile rows
   int nt_gu_routed, nt_gu_shared, nt_dn_routed, nt_dn_shared;  // N tiles per segment
   int splits_gu, splits_dn;  // split-K factors of the two GEMMs (1 = none)
@@ -216,6 +219,8 @@ struct TcArgs {
 };
 cudaError_t launch_tc_gate_up(const TcArgs& a, cudaStream_t st);
 cudaError_t launch_tc_down(const TcArgs& a, cudaStream_t st);
+cudaError_t launch_tc2_gate_up(const TcArgs& a, cudaStream_t st);  // CTA-pair variants
+cudaError_t launch_tc2_down(const TcArgs& a, cudaStream_t st);
 // Split-K reductions (partials -> epilogue) for the bf16 tensor-core GEMMs.
 cudaError_t launch_splitk_gate_up_reduce(const TcArgs& a, cudaStream_t st);
 cudaError_t launch_splitk_down_reduce(const TcArgs& a, cudaStream_t st);

@@ -52,6 +52,17 @@ def _host_sparse(inputs, experts):
 
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_parity(name):
+    _full_size(name)
+
+
+def test_full_size_mixtral_single_cta_gemm(monkeypatch):
+    """The large-batch workload again with the single-CTA GEMMs forced (the library
+    picks the CTA-pair GEMMs for it by default)."""
+    monkeypatch.setenv("MOE_B200_PAIR_GEMM", "0")
+    _full_size("mixtral_bf16")
+
+
+def _full_size(name):
     cfg = CONFIGS[name]
     torch.manual_seed(0)
     inputs = make_inputs(cfg, "cuda")
