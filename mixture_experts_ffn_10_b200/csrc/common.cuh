@@ -39,7 +39,7 @@ struct Plan {
   int64_t nchunks;    // ceil(T / kChunkTokens)
   int act_dtype, w_dtype, logit_dtype;
   bool tc;            // tensor-core path (bf16 activations) vs SIMT fp32 path
-  bool pair;          // bf16 GEMMs on CTA pairs (256-row tiles)
+  bool pair;          // bf16 GEMMs on CTA pairs (256 x 256 tiles over two SMs)
   int bm;             // GEMM tile rows
   int nt_gu_routed, nt_gu_shared, nt_dn_routed, nt_dn_shared;  // N tiles per segment
   int splits_gu, splits_dn;  // split-K factors of the two GEMMs (1 = none)

@@ -8,26 +8,26 @@
 // with W[e][r][k] = e2m1(code[e][r][k]) * 2^(scale[e][r][k/32] - 127) (OCP MX v1.0:
 // e2m1 two per byte, even k in the low nibble; e8m0 scale per 32 elements of K).
 //
-// Tile: 256 activation rows (two M=128 halves) x 128 weight rows x K, fp32 in TMEM
-// (2 halves x 128 columns, double-buffered).  Both halves share each decoded
-// weight stage, halving the decode work per FLOP.  Warp roles:
+// Tile: 256 activation rows x 128 weight rows x K, computed transposed: the
+// decoded weights are the MMA's A operand (M = 128 weight rows) and the
+// activation rows its B operand (N = the tile's token rows rounded up to 16, at
+// most 256), so one M=128 N<=256 instruction per K step reads 4 KiB of weights
+// and at most 8 KiB of activations.  The tensor pipe's shared-memory operand
+// reads, not the data movement, bound this kernel, and an M=128 N=256 step needs
+// a quarter less of them per FLOP than two M=128 N=128 halves sharing the
+// weights.  TMEM: 128 lanes (weight rows) x 256 columns (tokens), double-buffered.
+// Warp roles:
 //   warp 0      TMA producer of activations 256 x 64 (bf16, 128B swizzle)
-//   warp 1      TMEM owner and MMA issuer (M=128 N=128 K=16 per half)
+//   warp 1      TMEM owner and MMA issuer (M=128 N<=256 K=16)
 //   warp 26     TMA producer of the codes, 128 x 32 bytes, running up to 6 stages ahead
-//   warps 2-9   epilogue (bias + activation, or bias x routing weight; bf16 stores);
-//               warps 2-5 drain the first M half, warps 6-9 the second
+//   warps 2-9   epilogue: two warps per TMEM lane quadrant, alternate 16-token chunks;
+//               for gate_up, weight rows 2j and 2j+1 are the gate and up rows of one
+//               feature, so neighbouring lanes pair up with one shuffle
 //   warps 10-25 converters in four groups, group g owning stages it % 4 == g:
 //               codes + scale -> bf16 in the 128B-swizzled K-major layout the MMA
-//               descriptor reads, then a proxy fence and one arrive per warp.
-// Decode: the hardware conversion cvt.rn.f16x2.e2m1x2 turns each code byte into two
-// exact f16 values; shifting an f16's exponent and mantissa right by 3 bits (sign
-// kept) gives a bf16 of the same value times 2^-112, and one bf16x2 multiply by
-// 2^(s-15) applies the block scale and undoes the bias.  Exact (both factors have
-// at most two significant bits, the product stays normal) for scale bytes 2..142;
-// larger scale bytes take a second multiply.
-#include <cuda_bf16.h>
-
+//               descriptor reads (mxfp4.cuh), then a proxy fence and one arrive per warp.
 #include "epilogue.cuh"
+#include "mxfp4.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
 
@@ -35,9 +35,9 @@ namespace moe {
 namespace {
 
 using namespace sm100;
+using namespace mxfp4;
 
 constexpr int BM = kFp4BM;              // 256 = 2 x 128
-constexpr int HALF = 128;
 constexpr int BK = 64;                  // K elements per stage
 constexpr int BNB = 128;                // weight rows per tile
 // Three rings, so that decoding never holds an activation slot:
@@ -48,15 +48,15 @@ constexpr int A_BYTES = BM * BK * 2;    // 32 KiB
 constexpr int Q_BYTES = BNB * BK / 2;   // 4 KiB
 constexpr int W_BYTES = BNB * BK * 2;   // 16 KiB
 constexpr int RING_BYTES = AST * A_BYTES + WST * W_BYTES + QST * Q_BYTES;
-constexpr int ACC_COLS = 2 * BNB;       // two halves
+constexpr int ACC_COLS = BM;            // one column per activation row
 constexpr int TMEM_COLS = 2 * ACC_COLS; // double-buffered
-constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant: one per M half
+constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, alternate token chunks
+constexpr int kEpiGroups = kEpiWarps / 4;
 constexpr int kCvtWarps = 16;
 constexpr int kCvtGroups = 4;                // converter groups, each owning every 4th stage
 constexpr int kCvtGroupWarps = kCvtWarps / kCvtGroups;
 constexpr int kThreads = 64 + (kEpiWarps + kCvtWarps + 1) * 32;  // + the codes producer warp
 constexpr int SMEM_BYTES = RING_BYTES + 1024 + 512;
-constexpr uint32_t IDESC = idesc_bf16_f32(HALF, BNB);
 static_assert(kCvtGroupWarps * 32 == BNB, "one converter thread per weight row in a group");
 static_assert(WST % kCvtGroups == 0, "a group's stages map to its own decoded-weight slots");
 
@@ -74,12 +74,14 @@ __device__ __forceinline__ int k_extent(const GemmCommon& c) {
   return MODE == 0 ? c.d : c.F;
 }
 
-// Row of the scale / code stack (inside expert e) that tile row r reads.
+// Row of the scale / code stack (inside expert e) that weight row r of the tile
+// (the MMA's M index) reads.  gate_up: rows 2j, 2j+1 = gate and up rows of
+// feature n_blk * 64 + j.
 template <int MODE>
 __device__ __forceinline__ int weight_row(const GemmCommon& c, int n_blk, int r, bool* valid) {
   if (MODE == 0) {
-    const int half = r / (BNB / 2);
-    const int f = n_blk * (BNB / 2) + r % (BNB / 2);
+    const int half = r & 1;
+    const int f = n_blk * (BNB / 2) + (r >> 1);
     *valid = f < c.F;
     if (c.gu_layout == MOE_GU_INTERLEAVED) return 2 * f + half;
     return half ? c.F + f : f;
@@ -87,46 +89,6 @@ __device__ __forceinline__ int weight_row(const GemmCommon& c, int n_blk, int r,
   const int o = n_blk * BNB + r;
   *valid = o < c.d;
   return o;
-}
-
-// 8 e2m1 codes (one 32-bit word, element j in bits 4j..4j+3) -> 4 f16x2 words
-// (element 2i in the low half of word i), exact.
-__device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t (&h)[4]) {
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-      : "r"(w));
-}
-
-// f16x2 of e2m1 values -> bf16x2 of the same values times 2^-112 (exponent and
-// mantissa bits moved down by 3, signs kept; the low 3 mantissa bits are zero).
-__device__ __forceinline__ uint32_t f16x2_to_bf16x2_biased(uint32_t h) {
-  return ((h >> 3) & 0x0FFF0FFFu) | (h & 0x80008000u);
-}
-
-// bf16x2 multiplier that applies 2^(s-127) to a value biased by 2^-112: 2^(s-15).
-// For s > 142 that factor is not a bf16; `extra` then holds the remaining 2^(s-142).
-__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t s, uint32_t* extra) {
-  uint32_t e = s + 112;   // bf16 exponent field of 2^(s-15)
-  *extra = 0;
-  if (s == 255) e = 255;  // NaN scale propagates
-  else if (e > 254) {
-    *extra = (s - 142 + 127) << 7;  // 2^(s-142)
-    *extra |= *extra << 16;
-    e = 254;                          // 2^127
-  }
-  const uint32_t b = (e << 7) | (s == 255 ? 0x40u : 0u);
-  return b | (b << 16);
-}
-
-__device__ __forceinline__ uint32_t bmul(uint32_t a, uint32_t b) {
-  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a), y = *reinterpret_cast<__nv_bfloat162*>(&b);
-  x = __hmul2(x, y);
-  return *reinterpret_cast<uint32_t*>(&x);
 }
 
 template <int MODE>
@@ -238,7 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, tcount++) {
         const Tile t = decode_tile<BM>(c, tile);
-        const bool two = t.rows - t.m0 > HALF;  // second half holds rows of this segment
+        const int live = t.rows - t.m0 < BM ? t.rows - t.m0 : BM;  // token rows of this tile
+        const uint32_t idesc = idesc_bf16_f32(BNB, (live + 15) & ~15);
         const int acc = tcount & 1;
         if (!mbar_wait(&tempty[acc], ((tcount >> 1) & 1) ^ 1, abort_flag, c.status)) break;
         tc_fence_after();
@@ -251,15 +214,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t bd = sdesc_k_sw128(smem_u32(ringW + sw * W_BYTES));
+          const uint64_t wd = sdesc_k_sw128(smem_u32(ringW + sw * W_BYTES));  // A: decoded weights
+          const uint64_t xd = sdesc_k_sw128(smem_u32(ringA + sa * A_BYTES));  // B: activations
 #pragma unroll
-          for (int h = 0; h < 2; h++) {
-            if (h == 1 && !two) break;
-            const uint64_t ad = sdesc_k_sw128(smem_u32(ringA + sa * A_BYTES + h * (HALF * BK * 2)));
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; kk++)
-              mma_bf16(dt + h * BNB, ad + 2 * kk, bd + 2 * kk, IDESC, (kb | kk) != 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BK / 16; kk++)
+            mma_bf16(dt, wd + 2 * kk, xd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           mma_commit(&emptyA[sa]);
           mma_commit(&emptyW[sw]);
         }
@@ -272,45 +231,68 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 2 + kEpiWarps) {
     // ------------------------------------------------------------ epilogue
+    // Lane r of the accumulator is weight row r (32q + lane), column j token m0 + j.
     const int q = warp & 3;                 // TMEM lane quadrant this warp may read
-    const int h = (warp - 2) / 4;           // M half this warp drains
+    const int part = (warp - 2) / 4;        // which alternate 16-token chunks it drains
+    const int r = q * 32 + lane;
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, tcount++) {
       const Tile t = decode_tile<BM>(c, tile);
       const int acc = tcount & 1;
-      if (!mbar_wait(&tfull[acc], (tcount >> 1) & 1, abort_flag, c.status)) break;
+      // warp-uniform: the TMEM loads below need every lane of the warp
+      const bool got = mbar_wait(&tfull[acc], (tcount >> 1) & 1, abort_flag, c.status);
+      if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS + h * BNB;
-      const int row = t.m0 + h * HALF + q * 32 + lane;
-      const bool valid = row < t.rows;
-      if (__any_sync(0xffffffffu, valid)) {
-        const int64_t grow = (int64_t)c.off[t.seg] + row;
-        if (MODE == 0) {
-          const int f0 = t.n_blk * (BNB / 2);
-          const uint16_t* bias = p.gate_up_bias ? p.gate_up_bias + (int64_t)t.seg * 2 * c.F : nullptr;
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
+      const int live = t.rows - t.m0;      // token rows of the tile (may exceed BM)
+      const int64_t grow0 = (int64_t)c.off[t.seg] + t.m0;
+      if (MODE == 0) {
+        // lanes 2j / 2j+1 hold the gate / up row of feature f; the even lane
+        // finishes the chunk's first 8 tokens, the odd lane the last 8
+        const int f = t.n_blk * (BNB / 2) + (r >> 1);
+        const bool odd = lane & 1;
+        float bg = 0.f, bu = 0.f;
+        if (p.gate_up_bias && f < c.F) {
+          const uint16_t* b = p.gate_up_bias + (int64_t)t.seg * 2 * c.F;
           const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
-          uint16_t* out = p.out + grow * c.Fmax;
+          bg = bf16_to_f32(b[il ? 2 * f : f]);
+          bu = bf16_to_f32(b[il ? 2 * f + 1 : c.F + f]);
+        }
 #pragma unroll 1
-          for (int ch = 0; ch < (BNB / 2) / 16; ch++) {
-            uint32_t g[16], u[16];
-            tmem_ld16(tb + ch * 16, g);
-            tmem_ld16(tb + BNB / 2 + ch * 16, u);
-            tmem_ld_wait();
-            const int fb = f0 + ch * 16;
-            if (valid && fb < c.F) gate_up_chunk(g, u, bias, fb, c.F, il, c.act, out);
+        for (int ch = part; ch < BM / 16 && ch * 16 < live; ch += kEpiGroups) {
+          uint32_t v[16];
+          tmem_ld16(tb + ch * 16, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 8; i++) {
+            // the even lane keeps its gate values of tokens 0..7 and receives the
+            // up values; the odd lane keeps up 8..15 and receives gate 8..15
+            const uint32_t give = odd ? v[i] : v[8 + i];
+            const uint32_t recv = __shfl_xor_sync(0xffffffffu, give, 1);
+            const float g = __uint_as_float(odd ? recv : v[i]);
+            const float u = __uint_as_float(odd ? v[8 + i] : recv);
+            const int tok = ch * 16 + (odd ? 8 : 0) + i;
+            if (tok < live && f < c.F)
+              p.out[(grow0 + tok) * c.Fmax + f] = f32_to_bf16_rn(gated_act_bf16(c.act, g + bg, u + bu));
           }
-        } else {
-          const int n0 = t.n_blk * BNB;
-          const uint16_t* bias = p.down_bias ? p.down_bias + (int64_t)t.seg * c.d : nullptr;
-          const float w = (c.weigh_inputs || !valid) ? 1.f : p.roww[grow];
-          uint16_t* out = p.out + grow * c.d;
+        }
+      } else {
+        const int o = t.n_blk * BNB + r;
+        const float b = (p.down_bias && o < c.d) ? bf16_to_f32(p.down_bias[(int64_t)t.seg * c.d + o]) : 0.f;
 #pragma unroll 1
-          for (int ch = 0; ch < BNB / 16; ch++) {
-            uint32_t v[16];
-            tmem_ld16(tb + ch * 16, v);
-            tmem_ld_wait();
-            const int ob = n0 + ch * 16;
-            if (valid && ob < c.d) down_chunk(v, bias, ob, c.d, w, out);
+        for (int ch = part; ch < BM / 16 && ch * 16 < live; ch += kEpiGroups) {
+          uint32_t v[16];
+          tmem_ld16(tb + ch * 16, v);
+          tmem_ld_wait();
+          // routing weights of the chunk's 16 tokens: lane i (and i + 16) loads token i's
+          const int my_tok = ch * 16 + (lane & 15);
+          const float my_w = (c.weigh_inputs || my_tok >= live) ? 1.f : p.roww[grow0 + my_tok];
+#pragma unroll
+          for (int i = 0; i < 16; i++) {
+            const float w = __shfl_sync(0xffffffffu, my_w, i);
+            const int tok = ch * 16 + i;
+            if (tok < live && o < c.d)
+              p.out[(grow0 + tok) * c.d + o] = f32_to_bf16_rn((__uint_as_float(v[i]) + b) * w);
           }
         }
       }
@@ -353,7 +335,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        const uint4* qrow = reinterpret_cast<const uint4*>(ringQ + sq * Q_BYTES + r * (BK / 2));
+        // code rows in the slot: gate_up 64 gate rows then their 64 up rows; down in order
+        const int qr = MODE == 0 ? (r & 1) * (BNB / 2) + (r >> 1) : r;
+        const uint4* qrow = reinterpret_cast<const uint4*>(ringQ + sq * Q_BYTES + qr * (BK / 2));
         const uint4 q0 = qrow[0], q1 = qrow[1];
         __syncwarp();
         if (lane == 0) mbar_arrive(&emptyQ[sq]);  // codes are in registers: the slot may refill
@@ -361,25 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        uint8_t* wrow = ringW + sw * W_BYTES + r * (BK * 2);
-        const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-        for (int blk = 0; blk < 2; blk++) {
-          uint32_t extra;
-          const uint32_t scale = scale_bf16x2((sc >> (8 * blk)) & 0xFF, &extra);
-#pragma unroll
-          for (int wi = 0; wi < 4; wi++) {
-            uint32_t h[4], o[4];
-            e2m1x8_to_f16x8(words[blk * 4 + wi], h);
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-              o[i] = bmul(f16x2_to_bf16x2_biased(h[i]), scale);
-              if (extra) o[i] = bmul(o[i], extra);
-            }
-            const int chunk = blk * 4 + wi;  // 16-byte chunk (8 elements) of the 128-byte row
-            *reinterpret_cast<uint4*>(wrow + ((chunk ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-          }
-        }
+        decode_row_sw128(q0, q1, sc, ringW + sw * W_BYTES + r * (BK * 2), r);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&fullW[sw]);

@@ -176,7 +176,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int nkb = (k_extent<MODE>(c, t.seg >= c.E) + BK - 1) / BK;
         const int sp = unit % S, kb0 = sp * nkb / S, kb1 = (sp + 1) * nkb / S;
         const int acc = tcount & 1;
-        if (!mbar_wait(&tempty[acc], ((tcount >> 1) & 1) ^ 1, abort_flag, c.status)) break;
+        // the odd CTA's epilogue warps arrive here with cluster-scope release
+        if (!mbar_wait_cluster(&tempty[acc], ((tcount >> 1) & 1) ^ 1, abort_flag, c.status)) break;
         tc_fence_after();
         const uint32_t dt = tmem_base + acc * ACC_COLS;
         for (int kb = kb0; kb < kb1; kb++, it++) {

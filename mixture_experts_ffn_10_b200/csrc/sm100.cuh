@@ -50,6 +50,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with acquire at cluster scope: pairs with release arrivals made by
+// threads of the other CTA of a pair.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `bar` with the given parity.  Gives up (returns false)
 // when *abort is set by another role, or after kTimeoutNs, in which case it sets
 // *abort and records MOE_ERR_TIMEOUT in the device status word.
@@ -59,6 +73,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   const uint64_t t0 = global_timer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer() - t0 > kTimeoutNs) {
+      *abort = 1;
+      set_status(status, MOE_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// mbar_wait for barriers that threads of the other CTA of a pair arrive on.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                  int* status) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
     if (*abort) return false;
     if (global_timer() - t0 > kTimeoutNs) {
       *abort = 1;

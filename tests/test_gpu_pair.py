@@ -1,4 +1,4 @@
-"""GPU parity of the CTA-pair bf16 GEMMs (256-row tiles computed by two SMs).
+"""GPU parity of the CTA-pair bf16 GEMMs (256 x 256 tiles computed by two SMs).
 
 The library picks the pair kernels by itself for large batches (on average 512
 or more routed rows per expert); MOE_B200_PAIR_GEMM=1 forces them, so that small
