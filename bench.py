@@ -10,9 +10,10 @@ Mixtral-shaped bf16 prefill layer (T=4096, d=4096, F=14336, E=8, k=2).
 Timing: W warm-up steps, then K steps timed on the device with one CUDA event
 pair per step on the launching stream, each step a replay of a CUDA graph of
 the moe_forward call (--no-graph: eager calls); the L2 is flushed (512 MiB
-write) before every timed step, outside the events.  A second pass of K eager
-steps has the library record an event at every stage boundary; it gives the
-per-kernel times behind the roofline figure.
+write) before every timed step, outside the events.  A second pass of K steps
+has the library record an event at every stage boundary (inside the replayed
+graph, so without host launch gaps); it gives the per-kernel times behind the
+roofline figure.
 Under torchrun each rank runs an independent replica (no collective on the data
 path); the reported time is the max over ranks and `value` counts the tokens of
 all ranks.  `e2e` repeats the measurement through the same C-ABI call with the
@@ -40,10 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu dram bytes (read + write) per launch of the dominant kernel, per workload, from the
 # profile summaries under profiles/ (None until captured for the current kernel version).
 NCU_TRAFFIC = {  # profiles/tc2_gemm_mixtral_shape_E2.md, profiles/tc_fp4_gptoss.md
-    ("mixtral_bf16", "gate_up"): 1990000000 + 234580000,
-    ("mixtral_bf16", "down"): 1410000000 + 70570000,
-    ("gptoss_mxfp4", "gate_up"): 330280192 + 39711488,
-    ("gptoss_mxfp4", "down"): 188636416 + 26926080,
+    ("mixtral_bf16", "gate_up"): 2710000000 + 245120000,
+    ("mixtral_bf16", "down"): 1550000000 + 70600000,
 }
 
 
@@ -305,19 +304,68 @@ def run_own(args, cfg):
         raise RuntimeError(f"device status {moe.STATUS_NAMES.get(status, status)}")
 
     # Pass 2 (per-kernel breakdown for the roofline): the library records an event at
-    # every stage boundary on the launching stream, eager launches.
+    # every stage boundary on the launching stream.  The call with its events is
+    # replayed from a CUDA graph as in pass 1 (the events become graph nodes), so the
+    # stage times hold no host launch gaps; --no-graph records them on eager calls.
+    stage_graph = None
+    if graph is not None:
+        stage_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(stage_graph, stream=stream):
+            step(handles[0])
+        torch.cuda.synchronize()
+    stage_ms = [0.0] * (nev - 1)
+    staged_ms = 0.0
+
+    def add_row(row):
+        nonlocal staged_ms
+        staged_ms += row[0].elapsed_time(row[-1])
+        for s in range(nev - 1):
+            stage_ms[s] += row[s].elapsed_time(row[s + 1])
+
     with torch.cuda.stream(stream):
         for i in range(args.steps):
             flush.zero_()
-            step(handles[i])
+            if stage_graph is not None:
+                stage_graph.replay()
+                torch.cuda.synchronize()
+                add_row(events[0])
+            else:
+                step(handles[i])
     torch.cuda.synchronize()
-    stage_ms = [0.0] * (nev - 1)
-    eager_ms = 0.0
-    for row in events:
-        eager_ms += row[0].elapsed_time(row[-1])
-        for s in range(nev - 1):
-            stage_ms[s] += row[s].elapsed_time(row[s + 1])
+    if stage_graph is None:
+        for row in events:
+            add_row(row)
     stage_ms = [v / args.steps for v in stage_ms]
+    stage_launch = "cuda graph" if stage_graph is not None else "eager"
+
+    # Pass 3 (the roofline's kernel time): the same call with only the two events
+    # around the dominant GEMM stage (GEMM + its split-K reduction, if any), so
+    # that no other event node adds to that stage's time.
+    names = list(moe.STAGES)
+    dom = max(("gate_up", "down"), key=lambda n: stage_ms[names.index(n)])
+    s_dom = names.index(dom)  # the stage spans events[s_dom] .. events[s_dom + 1]
+    dom_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for ev in dom_ev:
+        ev.record(stream)
+    dom_handles = [None] * nev
+    dom_handles[s_dom], dom_handles[s_dom + 1] = dom_ev[0].cuda_event, dom_ev[1].cuda_event
+    dom_graph = None
+    if graph is not None:
+        dom_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(dom_graph, stream=stream):
+            step(dom_handles)
+        torch.cuda.synchronize()
+    dom_ms = 0.0
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.zero_()
+            if dom_graph is not None:
+                dom_graph.replay()
+            else:
+                step(dom_handles)
+            torch.cuda.synchronize()
+            dom_ms += dom_ev[0].elapsed_time(dom_ev[1])
+    dom_ms /= args.steps
     total_ms = max_over_ranks(total_ms, dist, "cuda")
     ms_per_step = total_ms / args.steps
     value = whole_job_throughput(world, cfg.T, args.steps, total_ms)
@@ -349,10 +397,7 @@ def run_own(args, cfg):
     distinct = int(torch.unique(idx).numel())
     pk, pk_src = peaks()
     model = stage_model(cfg, distinct)
-    names = list(moe.STAGES)
-    gemm_ms = {"gate_up": stage_ms[names.index("gate_up")], "down": stage_ms[names.index("down")]}
-    dom = max(gemm_ms, key=gemm_ms.get)
-    t_dom = gemm_ms[dom] / 1e3
+    t_dom = dom_ms / 1e3
     m = model[dom]
     t_tc, t_hbm = m["flops"] / (pk["bf16_tflops"] * 1e12), m["bytes"] / (pk["hbm_gbs"] * 1e9)
     if t_tc >= t_hbm:
@@ -365,7 +410,10 @@ def run_own(args, cfg):
                 "frac_vs_sustained_peak": (achieved / sustained) if sustained else None,
                 # the figures belong to the kernels the library picks by itself
                 "traffic": None if os.environ.get("MOE_B200_PAIR_GEMM") else NCU_TRAFFIC.get((cfg.name, dom)),
-                "algorithmic_per_launch": m["flops"] if bound == "tensor" else m["bytes"]}
+                "algorithmic_per_launch": m["flops"] if bound == "tensor" else m["bytes"],
+                "kernel_ms": dom_ms,
+                "timed": "CUDA events around this stage only (GEMM + split-K reduction), "
+                         + ("graph replay" if dom_graph is not None else "eager calls") + ", L2 flushed"}
     layer_flops = flops(cfg)
     layer_bytes = algorithmic_bytes(cfg, distinct)
     t_step = ms_per_step / 1e3
@@ -377,6 +425,10 @@ def run_own(args, cfg):
 
     if graph is not None:
         del graph
+    if stage_graph is not None:
+        del stage_graph
+    if dom_graph is not None:
+        del dom_graph
     out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": cfg.act_dtype if cfg.w_dtype != "mxfp4" else "bf16 (mxfp4 weights)",
@@ -385,7 +437,8 @@ def run_own(args, cfg):
                                        "launch": "cuda graph of moe_forward" if not args.no_graph else "eager moe_forward"}),
            "roofline": roofline, "layer": layer,
            "stage_ms": dict(zip(names, stage_ms)),
-           "eager_ms_per_step_with_stage_events": eager_ms / args.steps,
+           "stage_timing": {"launch": stage_launch,
+                            "ms_per_step_with_stage_events": staged_ms / args.steps},
            "e2e": {"value": e2e_value, "unit": "tokens/s",
                    "h2d_bytes_per_step": x_h.numel() * x_h.element_size() + l_h.numel() * l_h.element_size(),
                    "d2h_bytes_per_step": y_h.numel() * y_h.element_size()},

@@ -194,7 +194,8 @@ MOE_API int moe_route(const moe_shape *shape, const moe_options *opts, const moe
  *   events[2] after sort/scan/scatter events[6] after the combine
  *   events[3] after the row gather
  * n_events <= MOE_STAGE_EVENTS; NULL entries are skipped.  Same results,
- * errors and workspace rules as moe_forward.
+ * errors and workspace rules as moe_forward.  Called under stream capture,
+ * the events become event-record nodes of the graph and time every replay.
  */
 #define MOE_STAGE_EVENTS 7
 MOE_API int moe_forward_events(const moe_shape *shape, const moe_options *opts, const moe_tensors *t,

@@ -147,8 +147,14 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
   if (n_events < 0 || n_events > MOE_STAGE_EVENTS) return fail(MOE_ERR_ARG, "n_events must be 0..%d", MOE_STAGE_EVENTS);
   if (p.T == 0) return MOE_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Under stream capture the events must become event-record nodes of the graph
+  // (external records), not capture dependencies, to time each replay.
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (events && cudaStreamIsCapturing(st, &capture) != cudaSuccess) return cuda_fail(cudaGetLastError(), "cudaStreamIsCapturing");
+  const unsigned record_flags = capture == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : 0u;
   auto mark = [&](int i) -> cudaError_t {
-    if (events && i < n_events && events[i]) return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
+    if (events && i < n_events && events[i])
+      return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), st, record_flags);
     return cudaSuccess;
   };
   int* status = at<int>(ws, p.o_status);

@@ -12,7 +12,8 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;
+constexpr int kBatch = 4;  // expert rows whose loads are issued together
 
 template <typename T>
 __device__ __forceinline__ void load8(const T* p, float* f) {
@@ -42,15 +43,27 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
 #pragma unroll
   for (int i = 0; i < 8; i++) acc[i] = 0.f;
   float v[8];
-  for (int j = 0; j < a.k; j++) {
-    const int64_t row = a.pos[(int64_t)t * a.k + j];
-    if (row < 0 || row >= a.R) {
-      set_status(a.status, MOE_ERR_SHAPE);
-      continue;
-    }
-    load8<T>(Y + row * a.d + c, v);
+  // batches of kBatch rows: all loads first, then the adds in slot order
+  for (int j0 = 0; j0 < a.k; j0 += kBatch) {
+    float b[kBatch][8];
 #pragma unroll
-    for (int i = 0; i < 8; i++) acc[i] += v[i];
+    for (int u = 0; u < kBatch; u++) {
+#pragma unroll
+      for (int i = 0; i < 8; i++) b[u][i] = 0.f;
+      const int j = j0 + u;
+      if (j < a.k) {
+        const int64_t row = a.pos[(int64_t)t * a.k + j];
+        if (row < 0 || row >= a.R) set_status(a.status, MOE_ERR_SHAPE);
+        else load8<T>(Y + row * a.d + c, b[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; u++) {
+      if (j0 + u < a.k) {
+#pragma unroll
+        for (int i = 0; i < 8; i++) acc[i] += b[u][i];
+      }
+    }
   }
   if (a.has_shared) {
     const float g = a.sgate ? a.sgate[t] : 1.f;

@@ -150,7 +150,9 @@ __global__ void __launch_bounds__(kScatterWarps * 32) scatter_kernel(SortArgs a)
   }
 }
 
-// xg[r] = x[perm[r]] (times roww[r] for weigh-inputs), one warp per row, 16-byte vectors.
+// xg[r] = x[perm[r]] (times roww[r] for weigh-inputs), 16-byte vectors: one warp
+// per row and slice of the row; slice blockIdx.y of gridDim.y (more than one only
+// when there are too few rows to fill the GPU).
 template <typename T>
 __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
   const int lane = threadIdx.x & 31;
@@ -163,14 +165,16 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
   }
   constexpr int kVec = 16 / sizeof(T);
   const int nv = a.d / kVec;
+  const int per = (nv + gridDim.y - 1) / gridDim.y;
+  const int v0 = blockIdx.y * per, v1 = min(nv, v0 + per);
   const uint4* src = reinterpret_cast<const uint4*>((const T*)a.x + (int64_t)t * a.d);
   uint4* dst = reinterpret_cast<uint4*>((T*)a.xg + r * a.d);
   if (!a.weigh_inputs) {
-    for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+    for (int v = v0 + lane; v < v1; v += 32) dst[v] = __ldg(src + v);
     return;
   }
   const float w = a.roww[r];
-  for (int v = lane; v < nv; v += 32) {
+  for (int v = v0 + lane; v < v1; v += 32) {
     uint4 q = __ldg(src + v);
     if constexpr (sizeof(T) == 2) {
       uint32_t* u = reinterpret_cast<uint32_t*>(&q);
@@ -202,8 +206,13 @@ cudaError_t launch_sort(const SortArgs& a, cudaStream_t st) {
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t st) {
   if (a.R == 0) return cudaSuccess;
   const int blocks = (a.R + 7) / 8;
-  if (a.bf16) gather_kernel<uint16_t><<<blocks, 256, 0, st>>>(a);
-  else gather_kernel<float><<<blocks, 256, 0, st>>>(a);
+  // few rows: split each row into slices of at least 32 vectors until ~512 blocks
+  const int nv = a.d / (a.bf16 ? 8 : 4);
+  int slices = 1;
+  while (blocks * slices * 2 <= 512 && nv / (slices * 2) >= 32) slices *= 2;
+  const dim3 grid(blocks, slices);
+  if (a.bf16) gather_kernel<uint16_t><<<grid, 256, 0, st>>>(a);
+  else gather_kernel<float><<<grid, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 
