@@ -114,8 +114,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync();  // barrier init and the TMEM address visible to both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int S = c.splits;
-  const int total = c.tiles[c.NS] * S;
+  const int S = 1;  // the plan never splits K for pair tiles (launch rejects it)
+  const int total = c.tiles[c.NS];
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -220,26 +220,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int row = t.m0 + r_in_tile;
       const bool valid = row < t.rows;
       const int64_t grow = (int64_t)c.off[t.seg] + row;
-      if (S > 1) {
-        // split-K: this unit's fp32 partial accumulator row goes to the partial buffer
-        if (__any_sync(0xffffffffu, valid)) {
-          float* prow = c.partial + ((int64_t)(unit % S) * (c.R + (c.Fs > 0 ? c.T : 0)) + grow) * c.partial_pitch +
-                        t.n_blk * ACC_COLS;
-#pragma unroll 1
-          for (int ch = 0; ch < ACC_COLS / 16; ch++) {
-            uint32_t v[16];
-            tmem_ld16(tb + ch * 16, v);
-            tmem_ld_wait();
-            if (valid) {
-              float4* dst = reinterpret_cast<float4*>(prow + ch * 16);
-#pragma unroll
-              for (int i = 0; i < 4; i++)
-                dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                     __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-            }
-          }
-        }
-      } else if (__any_sync(0xffffffffu, valid)) {
+      if (__any_sync(0xffffffffu, valid)) {
         if (MODE == 0) {
           const int F = sh ? c.Fs : c.F;
           const int f0 = t.n_blk * BNC;
@@ -349,7 +330,8 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMa
   cudaError_t e = cudaFuncSetAttribute(tc2_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int units = p.c.max_tiles * p.c.splits;
+  if (p.c.splits != 1) return cudaErrorInvalidValue;
+  const int units = p.c.max_tiles;
   const int mc = max_clusters<MODE>(num_sms);
   const int clusters = units < mc ? units : mc;
   tc2_gemm_kernel<MODE><<<2 * clusters, kThreads, SMEM_BYTES, st>>>(a, as, b, bs, p);

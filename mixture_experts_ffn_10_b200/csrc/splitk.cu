@@ -65,12 +65,18 @@ __global__ void __launch_bounds__(256) reduce_down_kernel(TcArgs a) {
 
 }  // namespace
 
+// Cost of a split factor in 64-deep K steps per CTA: the waves of work units
+// times (K steps per unit + kUnitOverhead for a unit's pipeline fill and
+// epilogue), plus kReduceCost for the reduction kernel when S > 1.
+constexpr int64_t kUnitOverhead = 2;
+constexpr int64_t kReduceCost = 4;
+
 int choose_splits(int64_t tiles, int nkb, int sms) {
   if (tiles <= 0 || tiles >= sms) return 1;
   int best = 1;
-  int64_t best_cost = ((tiles + sms - 1) / sms) * nkb;
+  int64_t best_cost = ((tiles + sms - 1) / sms) * (nkb + kUnitOverhead);
   for (int s = 2; s <= 8 && 2 * s <= nkb; s++) {
-    const int64_t cost = ((tiles * s + sms - 1) / sms) * ((nkb + s - 1) / s);
+    const int64_t cost = ((tiles * s + sms - 1) / sms) * ((nkb + s - 1) / s + kUnitOverhead) + kReduceCost;
     if (cost < best_cost) {
       best_cost = cost;
       best = s;
