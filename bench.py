@@ -43,6 +43,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {  # profiles/tc2_gemm_mixtral_shape_E2.md, profiles/tc_fp4_gptoss.md
     ("mixtral_bf16", "gate_up"): 2710000000 + 245120000,
     ("mixtral_bf16", "down"): 1550000000 + 70600000,
+    ("gptoss_mxfp4", "gate_up"): 329673728 + 38580992,
+    ("gptoss_mxfp4", "down"): 188522240 + 30254336,
 }
 
 
