@@ -210,3 +210,35 @@ def test_forward_captured_in_a_cuda_graph_matches_eager(cfg):
     torch.cuda.synchronize()
     assert torch.equal(y_graph, y_eager)
     del g
+
+
+def test_stage_events_inside_a_cuda_graph_time_every_replay():
+    """moe_forward_events under stream capture: the events become graph nodes, each
+    replay times the stages, and the output equals moe_forward's."""
+    import mixture_experts_ffn_10_b200 as m
+    cfg = MIX
+    inputs = make_inputs(cfg, "cuda")
+    shape, opts = m.shape_of(cfg), m.options_of(cfg)
+    ws = m.Workspace(m.moe_workspace_size(shape, opts))
+    y = torch.empty_like(inputs["x"])
+    tens = m.tensors_of(inputs, y)
+    s = torch.cuda.Stream()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(m.MOE_STAGE_EVENTS)]
+    for ev in evs:
+        ev.record(s)
+    handles = [ev.cuda_event for ev in evs]
+    with torch.cuda.stream(s):
+        assert m.moe_forward(shape, opts, tens, ws.ptr, ws.nbytes, s.cuda_stream) == 0
+    torch.cuda.synchronize()
+    y_plain = y.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        assert m.moe_forward_events(shape, opts, tens, ws.ptr, ws.nbytes, s.cuda_stream, handles) == 0
+    for _ in range(2):
+        y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_plain)
+        stages = [evs[i].elapsed_time(evs[i + 1]) for i in range(len(evs) - 1)]
+        assert all(t >= 0.0 for t in stages) and sum(stages) > 0.0
+    del g
