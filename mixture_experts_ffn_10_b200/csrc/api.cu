@@ -443,7 +443,7 @@ int moe_forward_kernel_count(const moe_shape* s, const moe_options* o) {
   moe::Plan p;
   moe::make_plan(s, o, &p);
   // route, histogram, scan, scatter, gather, gate_up, down, combine (+ split-K reductions)
-  return 8 + (p.splits_gu > 1) + (p.splits_dn > 1);
+  return (p.nchunks == 1 ? 6 : 8) + (p.splits_gu > 1) + (p.splits_dn > 1);
 }
 
 const char* moe_last_error(void) { return moe::g_err.c_str(); }

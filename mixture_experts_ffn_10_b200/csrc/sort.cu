@@ -70,6 +70,37 @@ __device__ void block_exclusive_scan(int32_t* v, int n, int32_t* total, int32_t*
   __syncthreads();
 }
 
+// Segment offsets and per-GEMM tile prefixes from the per-expert row counts in
+// cnt[0..E) (shared memory; a block of 1024 threads).  Leaves the segments'
+// first rows (exclusive prefix) in cnt.
+__device__ void segment_scan(const SortArgs& a, int32_t* cnt, int32_t* tg, int32_t* td, int32_t* warp_tot,
+                             int32_t* tot) {
+  if (threadIdx.x == 0 && a.NS > a.E) cnt[a.E] = a.shared_rows;
+  __syncthreads();
+  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) {
+    const bool sh = s >= a.E;
+    const int32_t mt = (cnt[s] + a.bm - 1) / a.bm;
+    a.cnt[s] = cnt[s];
+    tg[s] = mt * (sh ? a.nt_gu_shared : a.nt_gu_routed);
+    td[s] = mt * (sh ? a.nt_dn_shared : a.nt_dn_routed);
+  }
+  __syncthreads();
+  block_exclusive_scan<2>(cnt, a.NS, tot, warp_tot);
+  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.off[s] = cnt[s];
+  if (threadIdx.x == 0) {
+    a.off[a.NS] = *tot;
+    if (*tot != a.R + a.shared_rows) set_status(a.status, MOE_ERR_SHAPE);
+  }
+  __syncthreads();
+  block_exclusive_scan<2>(tg, a.NS, tot, warp_tot);
+  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.tile_gu[s] = tg[s];
+  if (threadIdx.x == 0) a.tile_gu[a.NS] = *tot;
+  __syncthreads();
+  block_exclusive_scan<2>(td, a.NS, tot, warp_tot);
+  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.tile_dn[s] = td[s];
+  if (threadIdx.x == 0) a.tile_dn[a.NS] = *tot;
+}
+
 // One block of 1024 threads: per-expert chunk prefixes, segment offsets, tile prefixes.
 __global__ void __launch_bounds__(1024) scan_kernel(SortArgs a) {
   __shared__ int32_t cnt[kMaxE + 1];
@@ -87,28 +118,65 @@ __global__ void __launch_bounds__(1024) scan_kernel(SortArgs a) {
     }
     cnt[e] = run;
   }
-  if (threadIdx.x == 0 && a.NS > a.E) cnt[a.E] = a.shared_rows;
-  __syncthreads();
-  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) {
-    const bool sh = s >= a.E;
-    const int32_t mt = (cnt[s] + a.bm - 1) / a.bm;
-    a.cnt[s] = cnt[s];
-    tg[s] = mt * (sh ? a.nt_gu_shared : a.nt_gu_routed);
-    td[s] = mt * (sh ? a.nt_dn_shared : a.nt_dn_routed);
+  segment_scan(a, cnt, tg, td, warp_tot, &tot);
+}
+
+// Stable in-order placement of the (t, j) entries n0 .. n0 + n_ent - 1 of one chunk by
+// one warp: row = first row of the expert + `before` (rows of earlier chunks, or null)
+// + run (earlier entries of this chunk; run[] zeroed, in shared memory).
+__device__ void scatter_chunk(const SortArgs& a, int t0, int n_ent, const int32_t* first_row,
+                              const int32_t* before, int32_t* run) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < n_ent; base += 32) {
+    const int n = base + lane;
+    const bool valid = n < n_ent;
+    const int64_t slot = (int64_t)t0 * a.k + n;
+    int e = valid ? a.idx[slot] : -1;
+    if (e < 0 || e >= a.E) e = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lt_mask);
+    if (e >= 0) {
+      const int32_t row = first_row[e] + (before ? before[e] : 0) + run[e] + rank;
+      if (row >= 0 && row < a.R) {
+        const int t = t0 + n / a.k;
+        a.pos[slot] = row;
+        a.perm[row] = t;
+        a.roww[row] = a.w[slot];
+      } else {
+        set_status(a.status, MOE_ERR_SHAPE);
+      }
+    }
+    __syncwarp();
+    if (e >= 0 && rank == 0) run[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// The whole sort for a single chunk of tokens (T <= kChunkTokens) in one block:
+// histogram in shared memory, the segment scan, and the in-order scatter.
+__global__ void __launch_bounds__(1024) sort_one_chunk_kernel(SortArgs a) {
+  __shared__ int32_t cnt[kMaxE + 1];
+  __shared__ int32_t tg[kMaxE + 1];
+  __shared__ int32_t td[kMaxE + 1];
+  __shared__ int32_t run[kMaxE];
+  __shared__ int32_t warp_tot[32];
+  __shared__ int32_t tot;
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    cnt[e] = 0;
+    run[e] = 0;
   }
   __syncthreads();
-  block_exclusive_scan<2>(cnt, a.NS, &tot, warp_tot);
-  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.off[s] = cnt[s];
-  if (threadIdx.x == 0) {
-    a.off[a.NS] = tot;
-    if (tot != a.R + a.shared_rows) set_status(a.status, MOE_ERR_SHAPE);
+  const int n_ent = a.T * a.k;
+  for (int n = threadIdx.x; n < n_ent; n += blockDim.x) {
+    const int e = a.idx[n];
+    if (e >= 0 && e < a.E) atomicAdd(&cnt[e], 1);
+    else set_status(a.status, MOE_ERR_SHAPE);
   }
-  block_exclusive_scan<2>(tg, a.NS, &tot, warp_tot);
-  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.tile_gu[s] = tg[s];
-  if (threadIdx.x == 0) a.tile_gu[a.NS] = tot;
-  block_exclusive_scan<2>(td, a.NS, &tot, warp_tot);
-  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.tile_dn[s] = td[s];
-  if (threadIdx.x == 0) a.tile_dn[a.NS] = tot;
+  __syncthreads();
+  segment_scan(a, cnt, tg, td, warp_tot, &tot);
+  __syncthreads();
+  if (threadIdx.x < 32) scatter_chunk(a, 0, n_ent, cnt, nullptr, run);
 }
 
 // One warp per chunk walks its (t, j) entries in order, so rows inside an expert
@@ -123,31 +191,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) scatter_kernel(SortArgs a)
   __syncwarp();
   if (b >= a.nchunks) return;
   const int t0 = b * kChunkTokens;
-  const int n_ent = (min(a.T, t0 + kChunkTokens) - t0) * a.k;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = 0; base < n_ent; base += 32) {
-    const int n = base + lane;
-    const bool valid = n < n_ent;
-    const int64_t slot = (int64_t)t0 * a.k + n;
-    int e = valid ? a.idx[slot] : -1;
-    if (e < 0 || e >= a.E) e = -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & lt_mask);
-    if (e >= 0) {
-      const int32_t row = a.off[e] + a.hist[(int64_t)b * a.E + e] + run[e] + rank;
-      if (row >= 0 && row < a.R) {
-        const int t = t0 + n / a.k;
-        a.pos[slot] = row;
-        a.perm[row] = t;
-        a.roww[row] = a.w[slot];
-      } else {
-        set_status(a.status, MOE_ERR_SHAPE);
-      }
-    }
-    __syncwarp();
-    if (e >= 0 && rank == 0) run[e] += __popc(peers);
-    __syncwarp();
-  }
+  scatter_chunk(a, t0, (min(a.T, t0 + kChunkTokens) - t0) * a.k, a.off, a.hist + (int64_t)b * a.E, run);
 }
 
 // xg[r] = x[perm[r]] (times roww[r] for weigh-inputs), 16-byte vectors: one warp
@@ -196,6 +240,10 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
 
 cudaError_t launch_sort(const SortArgs& a, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
+  if (a.nchunks == 1) {  // small batches: one launch instead of three
+    sort_one_chunk_kernel<<<1, 1024, 0, st>>>(a);
+    return cudaGetLastError();
+  }
   hist_kernel<<<a.nchunks, 256, a.E * sizeof(int32_t), st>>>(a);
   scan_kernel<<<1, 1024, 0, st>>>(a);
   const int blocks = (a.nchunks + kScatterWarps - 1) / kScatterWarps;
