@@ -10,8 +10,9 @@
 // One persistent CTA per SM walks the device-computed tile list (segment-major,
 // then N block, then M block, so CTAs working at the same time share a weight
 // tile through L2).  Warp roles:
-//   warp 0     TMA producer: A tile 128 x 64 and B tile 256 x 64 (bf16, 128-byte
-//              swizzle) per stage into a 4-stage shared-memory ring;
+//   warp 0     TMA producer: A tile 128 x 64 (32 or 64 rows for batches of at most
+//              that many tokens) and B tile 256 x 64 (bf16, 128-byte swizzle) per
+//              stage into a 4-stage (5, 6 with the smaller A tiles) shared-memory ring;
 //   warp 1     TMEM allocator and MMA issuer: tcgen05.mma M=128 N=256 K=16,
 //              fp32 accumulators in TMEM, two accumulator buffers of 256 columns;
 //   warps 2-5  epilogue: tcgen05.ld the accumulator rows, bias + activation (or
@@ -29,20 +30,22 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = kTcBM;            // 128
-#ifndef MOE_TC_BK
-#define MOE_TC_BK 64
-#endif
-constexpr int BK = MOE_TC_BK;        // K per stage: 64 (128-byte rows, 4 stages); 32 (64-byte rows, 8 stages) measured slower
+constexpr int BM = kTcBM;            // 128 rows per tile (the MMA's M)
+constexpr int BK = 64;               // K per stage: 128-byte swizzled rows
 constexpr int BNB = 256;             // B rows per tile
-constexpr int STAGES = BK == 32 ? 8 : 4;
-constexpr CUtensorMapSwizzle kSwizzle = BK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
-  return BK == 32 ? sdesc_k_sw64(saddr) : sdesc_k_sw128(saddr);
-}
-constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BNB * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+// Stage layout for ABOX loaded activation rows (128, or 64 / 32 when no segment
+// can have more rows, i.e. small batches): [ABOX x 64 bf16][256 x 64 bf16].  The
+// MMA always reads 128 A rows; rows past ABOX alias the stage's B tile and only
+// feed accumulator rows that are never stored (row i of D depends on row i of
+// A alone).  Smaller A tiles leave room for more stages of weights in flight.
+template <int ABOX>
+struct Stage {
+  static constexpr int A_BYTES = ABOX * BK * 2;
+  static constexpr int BYTES = A_BYTES + B_BYTES;  // 48, 40 or 36 KiB (1024-aligned)
+  static constexpr int COUNT = ABOX == 128 ? 4 : ABOX == 64 ? 5 : 6;
+  static constexpr int SMEM = COUNT * BYTES + 1024 /*align*/ + 256 /*barriers*/;
+};
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
 #ifndef MOE_TC_EPI_WARPS
@@ -51,7 +54,6 @@ constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int kEpiWarps = MOE_TC_EPI_WARPS;  // 4, or 8 = two per TMEM lane quadrant splitting the chunks
 constexpr int kEpiGroups = kEpiWarps / 4;
 constexpr int kThreads = 64 + kEpiWarps * 32;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BNB);
 
 struct TcParams {
@@ -67,11 +69,12 @@ __device__ __forceinline__ int k_extent(const GemmCommon& c, bool shared) {
   return MODE == 0 ? c.d : (shared ? c.Fs : c.F);
 }
 
-template <int MODE>
+template <int MODE, int ABOX>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBs,
                    const TcParams p) {
+  constexpr int STAGES = Stage<ABOX>::COUNT, STAGE_BYTES = Stage<ABOX>::BYTES, A_BYTES = Stage<ABOX>::A_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
@@ -182,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
-          const uint64_t ad = sdesc(sa), bd = sdesc(sa + A_BYTES);
+          const uint64_t ad = sdesc_k_sw128(sa), bd = sdesc_k_sw128(sa + A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; kk++)
             mma_bf16(dt, ad + 2 * kk, bd + 2 * kk, IDESC, (kb > kb0 || kk > 0) ? 1u : 0u);
@@ -280,7 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // bf16 tensor map with the swizzle the UMMA descriptors expect.
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
               const uint32_t* box) {
-  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides, box, kSwizzle);
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // rows x K matrix with row pitch `pitch` elements; box 64 x box_rows.
@@ -313,16 +317,27 @@ bool map_down(CUtensorMap* m, const void* base, uint64_t F, uint64_t d, uint64_t
   return make_map(m, base, 3, dims, strides, box);
 }
 
-template <int MODE>
-cudaError_t launch(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMap& b, const CUtensorMap& bs,
-                   const TcParams& p, int num_sms, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       SMEM_BYTES);
+template <int MODE, int ABOX>
+cudaError_t launch_box(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMap& b, const CUtensorMap& bs,
+                       const TcParams& p, int num_sms, cudaStream_t st) {
+  constexpr int smem = Stage<ABOX>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE, ABOX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int units = p.c.max_tiles * p.c.splits;
   const int grid = units < num_sms ? units : num_sms;
-  tc_gemm_kernel<MODE><<<grid, kThreads, SMEM_BYTES, st>>>(a, as, b, bs, p);
+  tc_gemm_kernel<MODE, ABOX><<<grid, kThreads, smem, st>>>(a, as, b, bs, p);
   return cudaGetLastError();
+}
+
+// Activation rows each stage loads: no segment has more rows than there are tokens.
+int a_box_rows(const GemmCommon& c) { return c.T <= 32 ? 32 : c.T <= 64 ? 64 : BM; }
+
+template <int MODE>
+cudaError_t launch(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMap& b, const CUtensorMap& bs,
+                   const TcParams& p, int abox, int num_sms, cudaStream_t st) {
+  if (abox == 32) return launch_box<MODE, 32>(a, as, b, bs, p, num_sms, st);
+  if (abox == 64) return launch_box<MODE, 64>(a, as, b, bs, p, num_sms, st);
+  return launch_box<MODE, BM>(a, as, b, bs, p, num_sms, st);
 }
 
 }  // namespace
@@ -331,10 +346,11 @@ cudaError_t launch_tc_gate_up(const TcArgs& a, cudaStream_t st) {
   const GemmCommon& c = a.c;
   if (c.max_tiles == 0) return cudaSuccess;
   CUtensorMap mA, mAs, mB, mBs;
-  bool ok = map_rows(&mA, a.xg, c.d, c.R, c.d, BM);
+  const int abox = a_box_rows(c);
+  bool ok = map_rows(&mA, a.xg, c.d, c.R, c.d, abox);
   ok = ok && map_gate_up(&mB, a.gate_up, c.d, c.F, c.E, c.gu_layout);
   if (c.Fs > 0) {
-    ok = ok && map_rows(&mAs, a.x, c.d, c.T, c.d, BM);
+    ok = ok && map_rows(&mAs, a.x, c.d, c.T, c.d, abox);
     ok = ok && map_gate_up(&mBs, a.sh_gate_up, c.d, c.Fs, 1, c.gu_layout);
   } else {
     mAs = mA;
@@ -342,17 +358,18 @@ cudaError_t launch_tc_gate_up(const TcArgs& a, cudaStream_t st) {
   }
   if (!ok) return cudaErrorInvalidValue;
   TcParams p{c, (const uint16_t*)a.gate_up_bias, nullptr, a.roww, (uint16_t*)a.h};
-  return launch<0>(mA, mAs, mB, mBs, p, a.num_sms, st);
+  return launch<0>(mA, mAs, mB, mBs, p, abox, a.num_sms, st);
 }
 
 cudaError_t launch_tc_down(const TcArgs& a, cudaStream_t st) {
   const GemmCommon& c = a.c;
   if (c.max_tiles == 0) return cudaSuccess;
   CUtensorMap mA, mAs, mB, mBs;
-  bool ok = map_rows(&mA, a.h, c.F, c.R, c.Fmax, BM);
+  const int abox = a_box_rows(c);
+  bool ok = map_rows(&mA, a.h, c.F, c.R, c.Fmax, abox);
   ok = ok && map_down(&mB, a.down, c.F, c.d, c.E);
   if (c.Fs > 0) {
-    ok = ok && map_rows(&mAs, (const uint16_t*)a.h + (int64_t)c.R * c.Fmax, c.Fs, c.T, c.Fmax, BM);
+    ok = ok && map_rows(&mAs, (const uint16_t*)a.h + (int64_t)c.R * c.Fmax, c.Fs, c.T, c.Fmax, abox);
     ok = ok && map_down(&mBs, a.sh_down, c.Fs, c.d, 1);
   } else {
     mAs = mA;
@@ -360,7 +377,7 @@ cudaError_t launch_tc_down(const TcArgs& a, cudaStream_t st) {
   }
   if (!ok) return cudaErrorInvalidValue;
   TcParams p{c, nullptr, (const uint16_t*)a.down_bias, a.roww, (uint16_t*)a.Y};
-  return launch<1>(mA, mAs, mB, mBs, p, a.num_sms, st);
+  return launch<1>(mA, mAs, mB, mBs, p, abox, a.num_sms, st);
 }
 
 }  // namespace moe
