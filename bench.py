@@ -41,8 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu dram bytes (read + write) per launch of the dominant kernel, per workload, from the
 # profile summaries under profiles/ (None until captured for the current kernel version).
 NCU_TRAFFIC = {  # profiles/tc2_gemm_mixtral_shape_E2.md, profiles/tc_fp4_gptoss.md
-    ("mixtral_bf16", "gate_up"): 2710000000 + 245120000,
-    ("mixtral_bf16", "down"): 1550000000 + 70600000,
+    ("mixtral_bf16", "gate_up"): 2730000000 + 245070000,
+    ("mixtral_bf16", "down"): 1490000000 + 70610000,
     ("gptoss_mxfp4", "gate_up"): 329673728 + 38580992,
     ("gptoss_mxfp4", "down"): 188522240 + 30254336,
 }
