@@ -51,6 +51,23 @@ __device__ __forceinline__ Cand warp_best(Cand c) {
   return c;
 }
 
+// Order-preserving 64-bit image of a key for the top-k: larger keys map to larger
+// integers, NaN to 0 (below every number), -0 to the image of +0 (so equal keys,
+// +-0 included, fall to the index tie-break as in outranks()).
+__device__ __forceinline__ uint64_t ord_key(double k) {
+  if (isnan(k)) return 0ull;
+  if (k == 0.0) k = 0.0;
+  const uint64_t b = (uint64_t)__double_as_longlong(k);
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+// (key image, expert) candidates: larger image first, then the lower index; the
+// empty candidate (0, kNone) ranks below every expert, NaN keys included.
+constexpr int kNone = 0x7fffffff;
+__device__ __forceinline__ bool ahead(uint64_t ka, int ia, uint64_t kb, int ib) {
+  return ka > kb || (ka == kb && ia < ib);
+}
+
 __device__ __forceinline__ float load_logit(const void* p, int bf16, int64_t i) {
   return bf16 ? bf16_to_f32(((const uint16_t*)p)[i]) : ((const float*)p)[i];
 }
@@ -157,29 +174,54 @@ __global__ void __launch_bounds__(kWarps * 32) route_kernel(RouteArgs a) {
     }
   }
 
-  // ---- top-k: k rounds of a warp arg-best over the eligible, untaken experts
-  bool taken[EPL];
+  // ---- top-k: k rounds of a warp arg-best over the eligible, untaken experts,
+  // on the keys' order-preserving integer images (same order as outranks())
+  uint64_t okey[EPL];
+  bool avail[EPL];  // eligible and not yet taken
 #pragma unroll
-  for (int i = 0; i < EPL; i++) taken[i] = false;
+  for (int i = 0; i < EPL; i++) {
+    const int e = lane + 32 * i;
+    avail[i] = e < E && ((kept_groups >> (e / per)) & 1u);
+    okey[i] = ord_key(key[i]);
+  }
   double my_s = 0.0;
   int my_idx = -1;
   for (int j = 0; j < a.k; j++) {
-    Cand c{0.0, -1, 0.0};
+    uint64_t bk = 0ull;
+    int bi = kNone;
 #pragma unroll
     for (int i = 0; i < EPL; i++) {
       const int e = lane + 32 * i;
-      const bool elig = e < E && !taken[i] && ((kept_groups >> (e / per)) & 1u);
-      if (elig && outranks(key[i], e, c.key, c.idx)) c = Cand{key[i], e, s[i]};
+      if (avail[i] && ahead(okey[i], e, bk, bi)) {
+        bk = okey[i];
+        bi = e;
+      }
     }
-    c = warp_best(c);
-    if ((c.idx & 31) == lane) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+      const uint64_t ok = __shfl_xor_sync(0xffffffffu, bk, m);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, m);
+      if (ahead(ok, oi, bk, bi)) {
+        bk = ok;
+        bi = oi;
+      }
+    }
+    // the winner's owner lane marks it taken and hands its score to lane j
+    double sv = 0.0;
+    const int slot = bi >> 5;
+#pragma unroll
+    for (int i = 0; i < EPL; i++) {
+      if (i == slot) sv = s[i];
+    }
+    const double got = __shfl_sync(0xffffffffu, sv, bi & 31);
+    if ((bi & 31) == lane) {
 #pragma unroll
       for (int i = 0; i < EPL; i++)
-        if (lane + 32 * i == c.idx) taken[i] = true;
+        if (i == slot) avail[i] = false;
     }
     if (lane == j) {
-      my_s = c.s;
-      my_idx = c.idx;
+      my_s = got;
+      my_idx = bi == kNone ? -1 : bi;
     }
   }
 
