@@ -229,7 +229,7 @@ int choose_splits(int64_t tiles, int nkb, int sms);
 // MXFP4 expert stacks (gate_up / down are e2m1 codes); no shared expert.
 cudaError_t launch_fp4_gate_up(const TcArgs& a, cudaStream_t st);
 cudaError_t launch_fp4_down(const TcArgs& a, cudaStream_t st);
-constexpr int kFp4BM = 256;       // rows per MXFP4 tile (two M=128 halves share each decoded stage)
+constexpr int kFp4BM = 256;       // activation rows per MXFP4 tile (the MMA's N, trimmed to the live rows)
 constexpr int kFp4GuBN = 64;      // h features per MXFP4 gate_up tile (64 gate + 64 up rows)
 constexpr int kFp4DnBN = 128;     // output features per MXFP4 down tile
 

@@ -37,7 +37,7 @@ namespace {
 using namespace sm100;
 using namespace mxfp4;
 
-constexpr int BM = kFp4BM;              // 256 = 2 x 128
+constexpr int BM = kFp4BM;              // 256 activation rows per tile (MMA N)
 constexpr int BK = 64;                  // K elements per stage
 constexpr int BNB = 128;                // weight rows per tile
 // Three rings, so that decoding never holds an activation slot:
