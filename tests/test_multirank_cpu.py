@@ -66,3 +66,28 @@ def test_single_process_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(3.0) == 3.0
     assert bench.whole_job_throughput(1, 64, 5, 1.0) == pytest.approx(64 * 5 / 1e-3)
+
+
+def test_reference_arm_prints_one_contract_line_on_rank_zero(monkeypatch, capsys):
+    """The reference arm (the oracle on the host cores) runs without a GPU: one JSON
+    line with the contract's keys, its own cpu_baseline and a zero-copy e2e."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.delenv("RANK", raising=False)
+
+    class Args:
+        gpus, steps, warmup = 1, 1, 3
+    from workloads import CONFIGS
+    assert bench.run_reference(Args, CONFIGS["tiny_fp32"]) == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"].startswith("tiny_fp32")
