@@ -1,0 +1,259 @@
+// route.cuh -- routing of one token by one warp: picks k of E experts and their weights.
+//
+// Definitions ("Struct MoeSpec" field docs; graph-op page attributes k and
+// normalize_routing_weights; "Struct Moe" groups):
+//   l'_e = fp32(l_e) + fp32(router_bias_e)                      (router_bias)
+//   s_e  = softmax_e(l') over every expert, or sigmoid(l'_e)     (score)
+//   key_e = l'_e for an unbiased softmax (monotone in s_e), else s_e + B_e,
+//           formed in double                                     (selection_bias)
+//   groups: E/n_group contiguous experts per group, group score = the sum of
+//           its two best keys; only the best topk_group groups are eligible
+//   top-k by key, larger first, ties to the lower index, NaN keys last
+//   w_j = s_{e_j}; renormalize: w_j / max(sum_j w_j, 2^-14); then w_j * S
+// Scores and weights are computed in double, then rounded once to fp32.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+namespace routing {
+
+struct Cand {
+  double key;
+  int idx;  // -1 = none
+  double s;
+};
+
+// a outranks b: larger key, NaN below every number, then the lower index; -1 = none.
+__device__ __forceinline__ bool outranks(double ka, int ia, double kb, int ib) {
+  if (ib < 0) return ia >= 0;
+  if (ia < 0) return false;
+  const bool na = isnan(ka), nb = isnan(kb);
+  if (na || nb) return (na && nb) ? ia < ib : nb;
+  if (ka != kb) return ka > kb;
+  return ia < ib;
+}
+
+__device__ __forceinline__ Cand shfl_cand(const Cand& c, int src_lane_xor) {
+  Cand o;
+  o.key = __shfl_xor_sync(0xffffffffu, c.key, src_lane_xor);
+  o.idx = __shfl_xor_sync(0xffffffffu, c.idx, src_lane_xor);
+  o.s = __shfl_xor_sync(0xffffffffu, c.s, src_lane_xor);
+  return o;
+}
+
+__device__ __forceinline__ Cand warp_best(Cand c) {
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) {
+    Cand o = shfl_cand(c, m);
+    if (outranks(o.key, o.idx, c.key, c.idx)) c = o;
+  }
+  return c;
+}
+
+// Order-preserving 64-bit image of a key for the top-k: larger keys map to larger
+// integers, NaN to 0 (below every number), -0 to the image of +0 (so equal keys,
+// +-0 included, fall to the index tie-break as in outranks()).
+__device__ __forceinline__ uint64_t ord_key(double k) {
+  if (isnan(k)) return 0ull;
+  if (k == 0.0) k = 0.0;
+  const uint64_t b = (uint64_t)__double_as_longlong(k);
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+// (key image, expert) candidates: larger image first, then the lower index; the
+// empty candidate (0, kNone) ranks below every expert, NaN keys included.
+constexpr int kNone = 0x7fffffff;
+__device__ __forceinline__ bool ahead(uint64_t ka, int ia, uint64_t kb, int ib) {
+  return ka > kb || (ka == kb && ia < ib);
+}
+
+__device__ __forceinline__ float load_logit(const void* p, int bf16, int64_t i) {
+  return bf16 ? bf16_to_f32(((const uint16_t*)p)[i]) : ((const float*)p)[i];
+}
+
+// Routes token t with the calling warp (lane = this thread's lane).
+template <int EPL>  // experts per lane: E <= 32 * EPL, expert e = lane + 32 * i
+__device__ __forceinline__ void route_token(const RouteArgs& a, int t, int lane) {
+  const int E = a.E;
+
+  float lp[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; i++) {
+    const int e = lane + 32 * i;
+    float l = 0.f;
+    if (e < E) {
+      l = load_logit(a.logits, a.logit_bf16, (int64_t)t * E + e);
+      if (a.router_bias) l = l + load_logit(a.router_bias, a.logit_bf16, e);
+    }
+    lp[i] = l;
+  }
+
+  // ---- scores (double)
+  double s[EPL];
+  if (a.score == MOE_SCORE_SOFTMAX) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < EPL; i++)
+      if (lane + 32 * i < E && lp[i] > m) m = lp[i];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const float v = __shfl_xor_sync(0xffffffffu, m, o);
+      m = v > m ? v : m;
+    }
+    double den = 0.0;
+#pragma unroll
+    for (int i = 0; i < EPL; i++) {
+      s[i] = (lane + 32 * i < E) ? exp((double)lp[i] - (double)m) : 0.0;
+      den += s[i];
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+#pragma unroll
+    for (int i = 0; i < EPL; i++) s[i] = s[i] / den;
+  } else {
+#pragma unroll
+    for (int i = 0; i < EPL; i++) s[i] = 1.0 / (1.0 + exp(-(double)lp[i]));
+  }
+
+  // ---- keys
+  double key[EPL];
+  const bool plain_softmax = a.score == MOE_SCORE_SOFTMAX && a.sel_bias == nullptr;
+#pragma unroll
+  for (int i = 0; i < EPL; i++) {
+    const int e = lane + 32 * i;
+    if (plain_softmax)
+      key[i] = (double)lp[i];
+    else
+      key[i] = s[i] + ((a.sel_bias && e < E) ? (double)a.sel_bias[e] : 0.0);
+  }
+
+  // ---- group limit -> eligibility mask over groups
+  uint32_t kept_groups = 0xffffffffu;
+  int per = E;
+  if (a.n_group > 0) {
+    per = E / a.n_group;
+    double my_gscore = 0.0;
+    for (int g = 0; g < a.n_group; g++) {
+      // lane-local best two of group g, then a warp merge of the pairs
+      Cand b1{0.0, -1, 0.0}, b2{0.0, -1, 0.0};
+#pragma unroll
+      for (int i = 0; i < EPL; i++) {
+        const int e = lane + 32 * i;
+        if (e < E && e / per == g) {
+          if (outranks(key[i], e, b1.key, b1.idx)) {
+            b2 = b1;
+            b1 = Cand{key[i], e, 0.0};
+          } else if (outranks(key[i], e, b2.key, b2.idx)) {
+            b2 = Cand{key[i], e, 0.0};
+          }
+        }
+      }
+#pragma unroll
+      for (int m = 16; m >= 1; m >>= 1) {
+        const Cand o1 = shfl_cand(b1, m), o2 = shfl_cand(b2, m);
+        if (outranks(b1.key, b1.idx, o1.key, o1.idx)) {
+          if (outranks(o1.key, o1.idx, b2.key, b2.idx)) b2 = o1;
+        } else {
+          b2 = outranks(b1.key, b1.idx, o2.key, o2.idx) ? b1 : o2;
+          b1 = o1;
+        }
+      }
+      const double gs = per >= 2 ? b1.key + b2.key : b1.key;
+      if (lane == g) my_gscore = gs;
+    }
+    kept_groups = 0;
+    bool gtaken = false;
+    for (int r = 0; r < a.topk_group; r++) {
+      Cand c{my_gscore, (lane < a.n_group && !gtaken) ? lane : -1, 0.0};
+      c = warp_best(c);
+      kept_groups |= 1u << c.idx;
+      if (lane == c.idx) gtaken = true;
+    }
+  }
+
+  // ---- top-k: k rounds of a warp arg-best over the eligible, untaken experts,
+  // on the keys' order-preserving integer images (same order as outranks())
+  uint64_t okey[EPL];
+  bool avail[EPL];  // eligible and not yet taken
+#pragma unroll
+  for (int i = 0; i < EPL; i++) {
+    const int e = lane + 32 * i;
+    avail[i] = e < E && ((kept_groups >> (e / per)) & 1u);
+    okey[i] = ord_key(key[i]);
+  }
+  double my_s = 0.0;
+  int my_idx = -1;
+  for (int j = 0; j < a.k; j++) {
+    uint64_t bk = 0ull;
+    int bi = kNone;
+#pragma unroll
+    for (int i = 0; i < EPL; i++) {
+      const int e = lane + 32 * i;
+      if (avail[i] && ahead(okey[i], e, bk, bi)) {
+        bk = okey[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+      const uint64_t ok = __shfl_xor_sync(0xffffffffu, bk, m);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, m);
+      if (ahead(ok, oi, bk, bi)) {
+        bk = ok;
+        bi = oi;
+      }
+    }
+    // the winner's owner lane marks it taken and hands its score to lane j
+    double sv = 0.0;
+    const int slot = bi >> 5;
+#pragma unroll
+    for (int i = 0; i < EPL; i++) {
+      if (i == slot) sv = s[i];
+    }
+    const double got = __shfl_sync(0xffffffffu, sv, bi & 31);
+    if ((bi & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i < EPL; i++)
+        if (i == slot) avail[i] = false;
+    }
+    if (lane == j) {
+      my_s = got;
+      my_idx = bi == kNone ? -1 : bi;
+    }
+  }
+
+  // ---- weights: renormalize (sum in slot order) with the 2^-14 clamp, then the scale
+  double sum = 0.0;
+  for (int j = 0; j < a.k; j++) sum += __shfl_sync(0xffffffffu, my_s, j);
+  if (lane < a.k) {
+    double w = my_s;
+    if (a.renorm) {
+      const double den = sum > 0x1p-14 ? sum : 0x1p-14;
+      w = w / den;
+    }
+    w = w * (double)a.scale;
+    const int64_t o = (int64_t)t * a.k + lane;
+    a.idx[o] = my_idx;
+    a.w[o] = (float)w;
+    if (a.idx_user) a.idx_user[o] = my_idx;
+    if (a.w_user) a.w_user[o] = (float)w;
+  }
+
+  // ---- shared expert gate sigma(x_t . g)
+  if (a.sgate) {
+    float acc = 0.f;
+    for (int i = lane; i < a.d; i += 32) {
+      const int64_t xi = (int64_t)t * a.d + i;
+      const float xv = a.act_bf16 ? bf16_to_f32(((const uint16_t*)a.x)[xi]) : ((const float*)a.x)[xi];
+      const float gv = a.act_bf16 ? bf16_to_f32(((const uint16_t*)a.gvec)[i]) : ((const float*)a.gvec)[i];
+      acc = fmaf(xv, gv, acc);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) a.sgate[t] = 1.f / (1.f + expf(-acc));
+  }
+}
+
+}  // namespace routing
+}  // namespace moe

@@ -6,10 +6,12 @@
 // expert (when present) is segment E with one row per token at R + t.  The same
 // pass computes, per GEMM, the prefix of tiles per segment that the grouped
 // GEMMs walk on the device (no host round trip).
-#include "common.cuh"
+#include "sort.cuh"
 
 namespace moe {
 namespace {
+
+using namespace sorting;
 
 // Per-chunk expert histogram: hist[b][e] = #(t in chunk b, j) with idx[t][j] == e.
 __global__ void __launch_bounds__(256) hist_kernel(SortArgs a) {
@@ -26,79 +28,6 @@ __global__ void __launch_bounds__(256) hist_kernel(SortArgs a) {
   }
   __syncthreads();
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) a.hist[(int64_t)b * a.E + e] = sh[e];
-}
-
-// Block-wide exclusive scan of up to 1024 * kItems values held in shared memory.
-template <int kItems>
-__device__ void block_exclusive_scan(int32_t* v, int n, int32_t* total, int32_t* warp_tot) {
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  int32_t loc[kItems];
-  int32_t run = 0;
-#pragma unroll
-  for (int i = 0; i < kItems; i++) {
-    const int idx = tid * kItems + i;
-    loc[i] = idx < n ? v[idx] : 0;
-    run += loc[i];
-  }
-  int32_t incl = run;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int32_t u = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += u;
-  }
-  if (lane == 31) warp_tot[wid] = incl;
-  __syncthreads();
-  if (wid == 0) {
-    const int nw = blockDim.x >> 5;
-    int32_t wv = lane < nw ? warp_tot[lane] : 0, wi = wv;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int32_t u = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += u;
-    }
-    if (lane < nw) warp_tot[lane] = wi - wv;
-    if (lane == nw - 1) *total = wi;
-  }
-  __syncthreads();
-  int32_t base = warp_tot[wid] + incl - run;
-#pragma unroll
-  for (int i = 0; i < kItems; i++) {
-    const int idx = tid * kItems + i;
-    if (idx < n) v[idx] = base;
-    base += loc[i];
-  }
-  __syncthreads();
-}
-
-// Segment offsets and per-GEMM tile prefixes from the per-expert row counts in
-// cnt[0..E) (shared memory; a block of 1024 threads).  Leaves the segments'
-// first rows (exclusive prefix) in cnt.
-__device__ void segment_scan(const SortArgs& a, int32_t* cnt, int32_t* tg, int32_t* td, int32_t* warp_tot,
-                             int32_t* tot) {
-  if (threadIdx.x == 0 && a.NS > a.E) cnt[a.E] = a.shared_rows;
-  __syncthreads();
-  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) {
-    const bool sh = s >= a.E;
-    const int32_t mt = (cnt[s] + a.bm - 1) / a.bm;
-    a.cnt[s] = cnt[s];
-    tg[s] = mt * (sh ? a.nt_gu_shared : a.nt_gu_routed);
-    td[s] = mt * (sh ? a.nt_dn_shared : a.nt_dn_routed);
-  }
-  __syncthreads();
-  block_exclusive_scan<2>(cnt, a.NS, tot, warp_tot);
-  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.off[s] = cnt[s];
-  if (threadIdx.x == 0) {
-    a.off[a.NS] = *tot;
-    if (*tot != a.R + a.shared_rows) set_status(a.status, MOE_ERR_SHAPE);
-  }
-  __syncthreads();
-  block_exclusive_scan<2>(tg, a.NS, tot, warp_tot);
-  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.tile_gu[s] = tg[s];
-  if (threadIdx.x == 0) a.tile_gu[a.NS] = *tot;
-  __syncthreads();
-  block_exclusive_scan<2>(td, a.NS, tot, warp_tot);
-  for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.tile_dn[s] = td[s];
-  if (threadIdx.x == 0) a.tile_dn[a.NS] = *tot;
 }
 
 // One block of 1024 threads: per-expert chunk prefixes, segment offsets, tile prefixes.
@@ -118,39 +47,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(SortArgs a) {
     }
     cnt[e] = run;
   }
-  segment_scan(a, cnt, tg, td, warp_tot, &tot);
-}
-
-// Stable in-order placement of the (t, j) entries n0 .. n0 + n_ent - 1 of one chunk by
-// one warp: row = first row of the expert + `before` (rows of earlier chunks, or null)
-// + run (earlier entries of this chunk; run[] zeroed, in shared memory).
-__device__ void scatter_chunk(const SortArgs& a, int t0, int n_ent, const int32_t* first_row,
-                              const int32_t* before, int32_t* run) {
-  const int lane = threadIdx.x & 31;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = 0; base < n_ent; base += 32) {
-    const int n = base + lane;
-    const bool valid = n < n_ent;
-    const int64_t slot = (int64_t)t0 * a.k + n;
-    int e = valid ? a.idx[slot] : -1;
-    if (e < 0 || e >= a.E) e = -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & lt_mask);
-    if (e >= 0) {
-      const int32_t row = first_row[e] + (before ? before[e] : 0) + run[e] + rank;
-      if (row >= 0 && row < a.R) {
-        const int t = t0 + n / a.k;
-        a.pos[slot] = row;
-        a.perm[row] = t;
-        a.roww[row] = a.w[slot];
-      } else {
-        set_status(a.status, MOE_ERR_SHAPE);
-      }
-    }
-    __syncwarp();
-    if (e >= 0 && rank == 0) run[e] += __popc(peers);
-    __syncwarp();
-  }
+  segment_scan<2>(a, cnt, tg, td, warp_tot, &tot);
 }
 
 // The whole sort for a single chunk of tokens (T <= kChunkTokens) in one block:
@@ -174,7 +71,7 @@ __global__ void __launch_bounds__(1024) sort_one_chunk_kernel(SortArgs a) {
     else set_status(a.status, MOE_ERR_SHAPE);
   }
   __syncthreads();
-  segment_scan(a, cnt, tg, td, warp_tot, &tot);
+  segment_scan<2>(a, cnt, tg, td, warp_tot, &tot);
   __syncthreads();
   if (threadIdx.x < 32) scatter_chunk(a, 0, n_ent, cnt, nullptr, run);
 }
