@@ -110,26 +110,33 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
   const int v0 = blockIdx.y * per, v1 = min(nv, v0 + per);
   const uint4* src = reinterpret_cast<const uint4*>((const T*)a.x + (int64_t)t * a.d);
   uint4* dst = reinterpret_cast<uint4*>((T*)a.xg + r * a.d);
-  if (!a.weigh_inputs) {
-    for (int v = v0 + lane; v < v1; v += 32) dst[v] = __ldg(src + v);
-    return;
-  }
-  const float w = a.roww[r];
-  for (int v = v0 + lane; v < v1; v += 32) {
-    uint4 q = __ldg(src + v);
-    if constexpr (sizeof(T) == 2) {
-      uint32_t* u = reinterpret_cast<uint32_t*>(&q);
+  const float w = a.weigh_inputs ? a.roww[r] : 1.f;
+  // four vectors per lane in flight: loads first, then the (scaled) stores
+  constexpr int kBatch = 4;
+  for (int v = v0 + lane; v < v1; v += 32 * kBatch) {
+    uint4 q[kBatch];
 #pragma unroll
-      for (int i = 0; i < 4; i++) {
-        const float lo = bf16_to_f32(u[i] & 0xffff) * w, hi = bf16_to_f32(u[i] >> 16) * w;
-        u[i] = pack_bf16x2(lo, hi);
+    for (int b = 0; b < kBatch; b++)
+      if (v + 32 * b < v1) q[b] = __ldg(src + v + 32 * b);
+#pragma unroll
+    for (int b = 0; b < kBatch; b++) {
+      if (v + 32 * b >= v1) break;
+      if (a.weigh_inputs) {
+        if constexpr (sizeof(T) == 2) {
+          uint32_t* u = reinterpret_cast<uint32_t*>(&q[b]);
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            const float lo = bf16_to_f32(u[i] & 0xffff) * w, hi = bf16_to_f32(u[i] >> 16) * w;
+            u[i] = pack_bf16x2(lo, hi);
+          }
+        } else {
+          float* f = reinterpret_cast<float*>(&q[b]);
+#pragma unroll
+          for (int i = 0; i < 4; i++) f[i] *= w;
+        }
       }
-    } else {
-      float* f = reinterpret_cast<float*>(&q);
-#pragma unroll
-      for (int i = 0; i < 4; i++) f[i] *= w;
+      dst[v + 32 * b] = q[b];
     }
-    dst[v] = q;
   }
 }
 
