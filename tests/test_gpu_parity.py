@@ -59,6 +59,8 @@ CASES = {
     "mxfp4_concat": small(FP4, name="mxfp4_concat", gu_layout="concat", limit=0.0, alpha=1.0),
     "mxfp4_T1_many_experts": small(FP4, name="mxfp4_T1_many_experts", T=1, E=32, k=4),
     "mxfp4_big_rows": small(FP4, name="mxfp4_big_rows", T=700, E=4, k=2, d=256, F=256),
+    # 450 rows per expert: a full 256-row tile and a 194-row one
+    "mxfp4_three_row_tiles": small(FP4, name="mxfp4_three_row_tiles", T=450, E=2, k=2, d=256, F=256),
     # small batch over many experts with a long K (32-row activation tiles)
     "small_batch_long_k": small(CONFIGS["decode_T8"], name="small_batch_long_k", T=16, d=2048, F=384),
 }
