@@ -173,6 +173,10 @@ MOE_API size_t moe_workspace_size(const moe_shape *shape, const moe_options *opt
  * SMs); the environment variable MOE_B200_PAIR_GEMM=0 or =1, read at every
  * call, forces the single-CTA or the pair kernels.  Set it before
  * moe_workspace_size: the two choices may need different workspace sizes.
+ * Launches: every kernel after the first may be scheduled while its
+ * predecessor in the stream still runs (programmatic dependent launch) and
+ * waits on the device for the predecessor's results; MOE_B200_PDL=0, read
+ * once per process, turns this off.
  */
 MOE_API int moe_forward(const moe_shape *shape, const moe_options *opts, const moe_tensors *t,
                 void *workspace, size_t workspace_bytes, void *stream);

@@ -317,6 +317,14 @@ int set_error(int code, const char* msg) { return fail(code, "%s", msg); }
 // CTA-pair GEMMs for large batches with bf16 weights: every expert then has
 // several 256-row tiles on average, and the pair kernel needs a third less TMA
 // traffic per SM.  MOE_B200_PAIR_GEMM=0 or 1 overrides the choice.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* env = std::getenv("MOE_B200_PDL");
+    return !(env && env[0] == '0');
+  }();
+  return on;
+}
+
 bool use_pair_gemm(int64_t R, int64_t E) {
   const char* env = std::getenv("MOE_B200_PAIR_GEMM");
   if (env && env[0] == '0') return false;

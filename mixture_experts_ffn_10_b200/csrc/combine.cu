@@ -35,6 +35,7 @@ __device__ __forceinline__ void load8(const T* p, float* f) {
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
+  pdl_enter();
   const int t = blockIdx.x;
   const int c = (blockIdx.y * kThreads + threadIdx.x) * 8;
   if (c >= a.d) return;
@@ -95,9 +96,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   const dim3 grid(a.T, (a.d / 8 + kThreads - 1) / kThreads);
-  if (a.bf16) combine_kernel<uint16_t><<<grid, kThreads, 0, st>>>(a);
-  else combine_kernel<float><<<grid, kThreads, 0, st>>>(a);
-  return cudaGetLastError();
+  if (a.bf16) return launch_pdl(combine_kernel<uint16_t>, grid, kThreads, 0, st, a);
+  return launch_pdl(combine_kernel<float>, grid, kThreads, 0, st, a);
 }
 
 }  // namespace moe

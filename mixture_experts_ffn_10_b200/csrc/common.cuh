@@ -233,4 +233,34 @@ constexpr int kFp4BM = 256;       // activation rows per MXFP4 tile (the MMA's N
 constexpr int kFp4GuBN = 64;      // h features per MXFP4 gate_up tile (64 gate + 64 up rows)
 constexpr int kFp4DnBN = 128;     // output features per MXFP4 down tile
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Every kernel of the forward is launched with programmatic stream serialization:
+// it may be scheduled, and run a prologue that touches only shared memory, TMEM
+// and its parameters, while the kernel before it in the stream still runs.
+// pdl_enter() must come before the kernel's first global-memory access: it
+// returns once the preceding kernel has completed with its writes visible, then
+// lets the next kernel be scheduled.  Without the launch attribute (or with
+// MOE_B200_PDL=0) the wait returns at once and launches serialize as usual.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+bool pdl_enabled();  // false when the environment sets MOE_B200_PDL=0
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace moe

@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_enter();
   const uint32_t tmem_base = *tmem_slot;
   const int total = c.tiles[c.NS];
   const int K = k_extent<MODE>(c);
@@ -403,8 +404,7 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& q, const Fp4Params& 
                                        SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = p.c.max_tiles < num_sms ? p.c.max_tiles : num_sms;
-  fp4_gemm_kernel<MODE><<<grid, kThreads, SMEM_BYTES, st>>>(a, q, p);
-  return cudaGetLastError();
+  return launch_pdl(fp4_gemm_kernel<MODE>, (unsigned)grid, kThreads, SMEM_BYTES, st, a, q, p);
 }
 
 }  // namespace

@@ -41,6 +41,7 @@ __device__ __forceinline__ bool find_tile(const GemmCommon& c, int tile, TileInf
 }
 
 __global__ void __launch_bounds__(256) simt_gate_up_kernel(SimtArgs a) {
+  pdl_enter();
   const GemmCommon& c = a.c;
   TileInfo ti;
   if (!find_tile(c, blockIdx.x, &ti)) return;
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(256) simt_gate_up_kernel(SimtArgs a) {
 }
 
 __global__ void __launch_bounds__(256) simt_down_kernel(SimtArgs a) {
+  pdl_enter();
   const GemmCommon& c = a.c;
   TileInfo ti;
   if (!find_tile(c, blockIdx.x, &ti)) return;
@@ -186,14 +188,12 @@ __global__ void __launch_bounds__(256) simt_down_kernel(SimtArgs a) {
 
 cudaError_t launch_simt_gate_up(const SimtArgs& a, cudaStream_t st) {
   if (a.c.max_tiles == 0) return cudaSuccess;
-  simt_gate_up_kernel<<<a.c.max_tiles, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(simt_gate_up_kernel, (unsigned)a.c.max_tiles, 256, 0, st, a);
 }
 
 cudaError_t launch_simt_down(const SimtArgs& a, cudaStream_t st) {
   if (a.c.max_tiles == 0) return cudaSuccess;
-  simt_down_kernel<<<a.c.max_tiles, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(simt_down_kernel, (unsigned)a.c.max_tiles, 256, 0, st, a);
 }
 
 }  // namespace moe

@@ -112,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_enter();
   const uint32_t tmem_base = *tmem_slot;
   // Work units: (tile, split).  Split sp of a tile covers k-blocks
   // [sp * nkb / S, (sp + 1) * nkb / S) of the tile's K range.
@@ -325,8 +326,7 @@ cudaError_t launch_box(const CUtensorMap& a, const CUtensorMap& as, const CUtens
   if (e != cudaSuccess) return e;
   const int units = p.c.max_tiles * p.c.splits;
   const int grid = units < num_sms ? units : num_sms;
-  tc_gemm_kernel<MODE, ABOX><<<grid, kThreads, smem, st>>>(a, as, b, bs, p);
-  return cudaGetLastError();
+  return launch_pdl(tc_gemm_kernel<MODE, ABOX>, (unsigned)grid, kThreads, smem, st, a, as, b, bs, p);
 }
 
 // Activation rows each stage loads: no segment has more rows than there are tokens.

@@ -113,6 +113,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_before();
   cluster_sync();  // barrier init and the TMEM address visible to both CTAs
   tc_fence_after();
+  pdl_enter();
   const uint32_t tmem_base = *tmem_slot;
   const int S = 1;  // the plan never splits K for pair tiles (launch rejects it)
   const int total = c.tiles[c.NS];
@@ -334,8 +335,7 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMa
   const int units = p.c.max_tiles;
   const int mc = max_clusters<MODE>(num_sms);
   const int clusters = units < mc ? units : mc;
-  tc2_gemm_kernel<MODE><<<2 * clusters, kThreads, SMEM_BYTES, st>>>(a, as, b, bs, p);
-  return cudaGetLastError();
+  return launch_pdl(tc2_gemm_kernel<MODE>, (unsigned)(2 * clusters), kThreads, SMEM_BYTES, st, a, as, b, bs, p);
 }
 
 }  // namespace

@@ -9,6 +9,7 @@ constexpr int kWarps = 8;
 
 template <int EPL>
 __global__ void __launch_bounds__(kWarps * 32) route_kernel(RouteArgs a) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (t >= a.T) return;
@@ -21,13 +22,12 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   const dim3 grid((a.T + kWarps - 1) / kWarps), block(kWarps * 32);
   const int epl = (a.E + 31) / 32;
-  if (epl <= 1) route_kernel<1><<<grid, block, 0, st>>>(a);
-  else if (epl <= 2) route_kernel<2><<<grid, block, 0, st>>>(a);
-  else if (epl <= 4) route_kernel<4><<<grid, block, 0, st>>>(a);
-  else if (epl <= 8) route_kernel<8><<<grid, block, 0, st>>>(a);
-  else if (epl <= 16) route_kernel<16><<<grid, block, 0, st>>>(a);
-  else route_kernel<32><<<grid, block, 0, st>>>(a);
-  return cudaGetLastError();
+  if (epl <= 1) return launch_pdl(route_kernel<1>, grid, block, 0, st, a);
+  if (epl <= 2) return launch_pdl(route_kernel<2>, grid, block, 0, st, a);
+  if (epl <= 4) return launch_pdl(route_kernel<4>, grid, block, 0, st, a);
+  if (epl <= 8) return launch_pdl(route_kernel<8>, grid, block, 0, st, a);
+  if (epl <= 16) return launch_pdl(route_kernel<16>, grid, block, 0, st, a);
+  return launch_pdl(route_kernel<32>, grid, block, 0, st, a);
 }
 
 }  // namespace moe

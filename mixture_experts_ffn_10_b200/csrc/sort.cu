@@ -15,6 +15,7 @@ using namespace sorting;
 
 // Per-chunk expert histogram: hist[b][e] = #(t in chunk b, j) with idx[t][j] == e.
 __global__ void __launch_bounds__(256) hist_kernel(SortArgs a) {
+  pdl_enter();
   extern __shared__ int32_t sh[];
   const int b = blockIdx.x;
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) sh[e] = 0;
@@ -37,6 +38,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(SortArgs a) {
   __shared__ int32_t td[kMaxE + 1];
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t tot;
+  pdl_enter();
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
     int32_t run = 0;
     for (int b = 0; b < a.nchunks; b++) {
@@ -59,6 +61,7 @@ __global__ void __launch_bounds__(1024) sort_one_chunk_kernel(SortArgs a) {
   __shared__ int32_t run[kMaxE];
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t tot;
+  pdl_enter();
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
     cnt[e] = 0;
     run[e] = 0;
@@ -81,6 +84,7 @@ __global__ void __launch_bounds__(1024) sort_one_chunk_kernel(SortArgs a) {
 constexpr int kScatterWarps = 4;
 __global__ void __launch_bounds__(kScatterWarps * 32) scatter_kernel(SortArgs a) {
   extern __shared__ int32_t run_all[];  // [kScatterWarps][E]
+  pdl_enter();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int b = blockIdx.x * kScatterWarps + wid;
   int32_t* run = run_all + wid * a.E;
@@ -96,6 +100,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) scatter_kernel(SortArgs a)
 // when there are too few rows to fill the GPU).
 template <typename T>
 __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (r >= a.R) return;
@@ -145,14 +150,14 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
 cudaError_t launch_sort(const SortArgs& a, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   if (a.nchunks == 1) {  // small batches: one launch instead of three
-    sort_one_chunk_kernel<<<1, 1024, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(sort_one_chunk_kernel, 1, 1024, 0, st, a);
   }
-  hist_kernel<<<a.nchunks, 256, a.E * sizeof(int32_t), st>>>(a);
-  scan_kernel<<<1, 1024, 0, st>>>(a);
+  cudaError_t e = launch_pdl(hist_kernel, (unsigned)a.nchunks, 256, a.E * sizeof(int32_t), st, a);
+  if (e == cudaSuccess) e = launch_pdl(scan_kernel, 1, 1024, 0, st, a);
   const int blocks = (a.nchunks + kScatterWarps - 1) / kScatterWarps;
-  scatter_kernel<<<blocks, kScatterWarps * 32, kScatterWarps * a.E * sizeof(int32_t), st>>>(a);
-  return cudaGetLastError();
+  if (e == cudaSuccess)
+    e = launch_pdl(scatter_kernel, (unsigned)blocks, kScatterWarps * 32, kScatterWarps * a.E * sizeof(int32_t), st, a);
+  return e;
 }
 
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t st) {
@@ -163,9 +168,8 @@ cudaError_t launch_gather(const GatherArgs& a, cudaStream_t st) {
   int slices = 1;
   while (blocks * slices * 2 <= 512 && nv / (slices * 2) >= 32) slices *= 2;
   const dim3 grid(blocks, slices);
-  if (a.bf16) gather_kernel<uint16_t><<<grid, 256, 0, st>>>(a);
-  else gather_kernel<float><<<grid, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  if (a.bf16) return launch_pdl(gather_kernel<uint16_t>, grid, 256, 0, st, a);
+  return launch_pdl(gather_kernel<float>, grid, 256, 0, st, a);
 }
 
 }  // namespace moe

@@ -22,6 +22,7 @@ __device__ __forceinline__ int segment_of(const GemmCommon& c, int row) {
 
 // One block per (row, 128 features); thread = feature.
 __global__ void __launch_bounds__(128) reduce_gate_up_kernel(TcArgs a) {
+  pdl_enter();
   const GemmCommon& c = a.c;
   const int row = blockIdx.x;
   const int f = blockIdx.y * 128 + threadIdx.x;
@@ -48,6 +49,7 @@ __global__ void __launch_bounds__(128) reduce_gate_up_kernel(TcArgs a) {
 
 // One block per (row, 256 outputs); thread = output feature.
 __global__ void __launch_bounds__(256) reduce_down_kernel(TcArgs a) {
+  pdl_enter();
   const GemmCommon& c = a.c;
   const int row = blockIdx.x;
   const int o = blockIdx.y * 256 + threadIdx.x;
@@ -90,8 +92,7 @@ cudaError_t launch_splitk_gate_up_reduce(const TcArgs& a, cudaStream_t st) {
   const int rows = c.R + (c.Fs > 0 ? c.T : 0);
   if (rows == 0) return cudaSuccess;
   const dim3 grid(rows, (c.Fmax + 127) / 128);
-  reduce_gate_up_kernel<<<grid, 128, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(reduce_gate_up_kernel, grid, 128, 0, st, a);
 }
 
 cudaError_t launch_splitk_down_reduce(const TcArgs& a, cudaStream_t st) {
@@ -99,8 +100,7 @@ cudaError_t launch_splitk_down_reduce(const TcArgs& a, cudaStream_t st) {
   const int rows = c.R + (c.Fs > 0 ? c.T : 0);
   if (rows == 0) return cudaSuccess;
   const dim3 grid(rows, (c.d + 255) / 256);
-  reduce_down_kernel<<<grid, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(reduce_down_kernel, grid, 256, 0, st, a);
 }
 
 }  // namespace moe
