@@ -42,14 +42,15 @@ METRIC = "MoE layer tokens/s; achieved TFLOP/s or HBM GB/s as % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu dram bytes (read + write) per launch of the dominant kernel, per workload, from the
 # profile summaries under profiles/ (None until captured for the current kernel version).
-NCU_TRAFFIC = {  # profiles/tc2_gemm_mixtral_shape_E2.md, tc_fp4_gptoss.md, tc_gemm_decode_deepseek.md
-    ("mixtral_bf16", "gate_up"): 2730000000 + 245070000,
-    ("mixtral_bf16", "down"): 1490000000 + 70610000,
-    ("deepseek_bf16", "gate_up"): 16340000000 + 470610000,
-    ("deepseek_bf16", "down"): 6630000000 + 1050000000,
-    ("decode_T1", "gate_up"): 207700000,  # read + write, from throughput x duration of one capture
-    ("gptoss_mxfp4", "gate_up"): 329673728 + 38580992,
-    ("gptoss_mxfp4", "down"): 188522240 + 30254336,
+NCU_TRAFFIC = {  # median dram__bytes_read.sum + dram__bytes_write.sum per launch: profiles/launches_<workload>.md
+    ("mixtral_bf16", "gate_up"): 2925367552 + 242864000,
+    ("mixtral_bf16", "down"): 1662191232 + 71625088,
+    ("deepseek_bf16", "gate_up"): 15873404672 + 468926208,
+    ("deepseek_bf16", "down"): 6651168128 + 1050486016,
+    ("decode_T1", "gate_up"): 203038592 + 206080,
+    ("decode_T1", "down"): 100721536 + 144000,
+    ("gptoss_mxfp4", "gate_up"): 329679232 + 35157760,
+    ("gptoss_mxfp4", "down"): 188540544 + 26514816,
 }
 
 
