@@ -2,8 +2,9 @@
 
 Argument marshalling only: every step of the forward runs in the CUDA library
 (``libmoe_b200.so``, built in-tree by ``build.py``).  PyTorch supplies device
-memory and streams.  There is no fallback: if the library is missing the
-import fails.
+memory and streams.  There is no fallback: while the library is missing,
+every entry point raises ImportError (the package itself stays importable so
+that ``build.py`` can run).
 
 Entry points mirror ``include/moe.h``: ``moe_options_init``,
 ``moe_workspace_size``, ``moe_forward``, ``moe_route``, ``moe_last_error``,
@@ -55,35 +56,54 @@ class moe_tensors(C.Structure):
         "shared_gate_vec", "shared_output", "y", "topk_idx", "topk_w")]
 
 
-if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m "
-                      "mixture_experts_ffn_10_b200.build` (nvcc, sm_100a)")
-_lib = C.CDLL(LIB_PATH)
 _P = C.POINTER
-_lib.moe_options_init.argtypes = [_P(moe_options)]
-_lib.moe_options_init.restype = None
-_lib.moe_workspace_size.argtypes = [_P(moe_shape), _P(moe_options)]
-_lib.moe_workspace_size.restype = C.c_size_t
-for _fn in (_lib.moe_forward, _lib.moe_route):
-    _fn.argtypes = [_P(moe_shape), _P(moe_options), _P(moe_tensors), C.c_void_p, C.c_size_t,
-                    C.c_void_p]
-    _fn.restype = C.c_int
-_lib.moe_forward_events.argtypes = [_P(moe_shape), _P(moe_options), _P(moe_tensors), C.c_void_p,
-                                   C.c_size_t, C.c_void_p, _P(C.c_void_p), C.c_int]
-_lib.moe_forward_events.restype = C.c_int
 MOE_STAGE_EVENTS = 7
-_lib.moe_forward_noalloc.argtypes = [_P(moe_shape), _P(moe_options), _P(moe_tensors), C.c_void_p]
-_lib.moe_forward_noalloc.restype = C.c_int
 MOE_NOALLOC_WORKSPACE_BYTES = 64 << 20
-_lib.moe_forward_kernel_count.argtypes = [_P(moe_shape), _P(moe_options)]
-_lib.moe_forward_kernel_count.restype = C.c_int
 STAGES = ("route", "sort", "gather", "gate_up", "down", "combine")
-_lib.moe_last_error.argtypes = []
-_lib.moe_last_error.restype = C.c_char_p
-_lib.moe_debug_status.argtypes = [C.c_void_p, C.c_void_p]
-_lib.moe_debug_status.restype = C.c_int
-_lib.moe_version.argtypes = []
-_lib.moe_version.restype = C.c_char_p
+
+
+def _bind(lib: C.CDLL) -> C.CDLL:
+    """Declares the argument and result types of every entry point of include/moe.h."""
+    lib.moe_options_init.argtypes = [_P(moe_options)]
+    lib.moe_options_init.restype = None
+    lib.moe_workspace_size.argtypes = [_P(moe_shape), _P(moe_options)]
+    lib.moe_workspace_size.restype = C.c_size_t
+    for fn in (lib.moe_forward, lib.moe_route):
+        fn.argtypes = [_P(moe_shape), _P(moe_options), _P(moe_tensors), C.c_void_p, C.c_size_t,
+                       C.c_void_p]
+        fn.restype = C.c_int
+    lib.moe_forward_events.argtypes = [_P(moe_shape), _P(moe_options), _P(moe_tensors), C.c_void_p,
+                                       C.c_size_t, C.c_void_p, _P(C.c_void_p), C.c_int]
+    lib.moe_forward_events.restype = C.c_int
+    lib.moe_forward_noalloc.argtypes = [_P(moe_shape), _P(moe_options), _P(moe_tensors), C.c_void_p]
+    lib.moe_forward_noalloc.restype = C.c_int
+    lib.moe_forward_kernel_count.argtypes = [_P(moe_shape), _P(moe_options)]
+    lib.moe_forward_kernel_count.restype = C.c_int
+    lib.moe_last_error.argtypes = []
+    lib.moe_last_error.restype = C.c_char_p
+    lib.moe_debug_status.argtypes = [C.c_void_p, C.c_void_p]
+    lib.moe_debug_status.restype = C.c_int
+    lib.moe_version.argtypes = []
+    lib.moe_version.restype = C.c_char_p
+    return lib
+
+
+class _UnbuiltLibrary:
+    """Stands in for the CUDA library until it exists.  The package stays importable
+    without it, so that its build step can run; every entry point then loads the
+    library on first use and raises ImportError while it has not been built.  There
+    is no fallback: nothing here computes without the CUDA library."""
+
+    def __getattr__(self, name):
+        global _lib
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python "
+                              f"{os.path.join(_HERE, 'build.py')}` (nvcc, sm_100a)")
+        _lib = _bind(C.CDLL(LIB_PATH))
+        return getattr(_lib, name)
+
+
+_lib = _bind(C.CDLL(LIB_PATH)) if os.path.exists(LIB_PATH) else _UnbuiltLibrary()
 
 EXPORTED = ("moe_options_init", "moe_workspace_size", "moe_forward", "moe_route",
             "moe_forward_events", "moe_forward_noalloc", "moe_forward_kernel_count",

@@ -133,3 +133,28 @@ def test_route_needs_outputs(moe):
     t = moe.moe_tensors()
     t.router_logits = FAKE
     assert moe.moe_route(s, o, t, FAKE, 1 << 40, None) == moe.MOE_ERR_NULL
+
+
+def test_binding_without_its_library_imports_but_every_entry_point_raises(tmp_path):
+    """A fresh checkout has no libmoe_b200.so: the package must import (its build
+    step lives inside it) and each entry point must fail loudly, never compute."""
+    import shutil
+    import subprocess
+    import sys
+
+    pkg = tmp_path / "mixture_experts_ffn_10_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "mixture_experts_ffn_10_b200", "__init__.py"), pkg / "__init__.py")
+    code = (
+        "import mixture_experts_ffn_10_b200 as m\n"
+        "for call in (m.moe_version, m.moe_options_init, lambda: m.moe_last_error()):\n"
+        "    try:\n"
+        "        call()\n"
+        "    except ImportError as e:\n"
+        "        assert 'is missing' in str(e)\n"
+        "    else:\n"
+        "        raise SystemExit('entry point ran without the library')\n"
+        "print('ok')\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True,
+                       env={**os.environ, "PYTHONPATH": str(tmp_path)})
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
