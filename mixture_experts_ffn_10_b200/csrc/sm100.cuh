@@ -148,18 +148,6 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
   return d;
 }
 
-// Same for the 64-byte swizzle (rows of 64 bytes, 8-row atoms 512 bytes apart,
-// swizzle mode 4).
-__device__ __forceinline__ uint64_t sdesc_k_sw64(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
-  d |= (uint64_t)1 << 16;
-  d |= (uint64_t)(512 >> 4) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)4 << 61;
-  return d;
-}
-
 // Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1), A and B
 // bf16 (bits 7-9 and 10-12 = 1), both K-major, N >> 3 in bits 17-22, M >> 4 in 24-28.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
