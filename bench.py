@@ -446,6 +446,7 @@ def run_own(args, cfg):
 
     # ------------------------------------------------------------ roofline of the dominant kernel
     distinct = int(torch.unique(idx).numel())
+    rows_per_expert = torch.bincount(idx.flatten().long(), minlength=cfg.E)
     pk, pk_src = peaks()
     model = stage_model(cfg, distinct)
     t_dom = dom_ms / 1e3
@@ -472,7 +473,9 @@ def run_own(args, cfg):
              "hbm_gbs": layer_bytes / t_step / 1e9, "hbm_frac": layer_bytes / t_step / 1e9 / pk["hbm_gbs"],
              "tensor_frac_vendor_2250": layer_flops / t_step / 1e12 / 2250.0,
              "hbm_frac_vendor_8000": layer_bytes / t_step / 1e9 / 8000.0,
-             "distinct_experts": distinct, "flops": layer_flops, "bytes": layer_bytes}
+             "distinct_experts": distinct, "flops": layer_flops, "bytes": layer_bytes,
+             "rows_per_expert": {"max": int(rows_per_expert.max()), "mean_touched": cfg.T * cfg.k / distinct,
+                                 "empty_experts": int((rows_per_expert == 0).sum())}}
 
     if graph is not None:
         del graph
