@@ -158,3 +158,31 @@ def test_binding_without_its_library_imports_but_every_entry_point_raises(tmp_pa
     r = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True,
                        env={**os.environ, "PYTHONPATH": str(tmp_path)})
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
+
+
+@pytest.mark.parametrize("name,count", [
+    ("tiny_fp32", 6), ("decode_T1", 7), ("decode_T8", 6), ("decode_T64", 6), ("decode_T256", 8),
+    ("mixtral_bf16", 8), ("gptoss_mxfp4", 8), ("deepseek_bf16", 8)])
+def test_kernel_count_of_each_workload(moe, name, count):
+    """The launch plan on a 148-SM part (what the host assumes without a GPU): route,
+    sort (one kernel for a single 64-token chunk, else histogram + scan + scatter),
+    gather, gate_up, down, combine, plus a reduction per GEMM whose K is split.  Decode
+    T=1 splits gate_up only (96 tiles of 64 k-blocks would leave 52 SMs idle); the
+    counts agree with the ncu launch lists of these workloads."""
+    from workloads import CONFIGS
+    cfg = CONFIGS[name]
+    assert moe.moe_forward_kernel_count(moe.shape_of(cfg), moe.options_of(cfg)) == count
+
+
+def test_split_k_choice_follows_the_cost_model(moe):
+    """choose_splits: cost = waves * (k-blocks per unit + 2) + 4 for the reduction.
+    T=1, E=8, k=1, d=4096, F=1024: gate_up has 8 tiles x 64 k-blocks -> 8 splits (one
+    wave of 64 units of 8 k-blocks: cost 14 against 66); down has 16 tiles x 16 k-blocks
+    -> 8 splits (cost 8 against 18).  T=65 (two sort chunks): gate_up 64 tiles -> 2
+    splits (cost 38; 4 splits cost 40), down 128 tiles -> no split (18 against 24)."""
+    o = moe.make_options()
+    assert moe.moe_forward_kernel_count(moe.make_shape(T=1, d=4096, F=1024, E=8, k=1), o) == 6 + 2
+    assert moe.moe_forward_kernel_count(moe.make_shape(T=65, d=4096, F=1024, E=8, k=1), o) == 8 + 1
+    # fp32 problems run the SIMT GEMMs, which never split K
+    f32 = moe.make_shape(T=1, d=4096, F=1024, E=8, k=1, act_dtype="f32", w_dtype="f32", logit_dtype="f32")
+    assert moe.moe_forward_kernel_count(f32, o) == 6
