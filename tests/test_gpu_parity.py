@@ -246,3 +246,25 @@ def test_stage_events_inside_a_cuda_graph_time_every_replay():
         stages = [evs[i].elapsed_time(evs[i + 1]) for i in range(len(evs) - 1)]
         assert all(t >= 0.0 for t in stages) and sum(stages) > 0.0
     del g
+
+
+# The library's limits: E = 1024 experts (32 per routing lane), k = 32, 32 groups.
+MAX_CASES = {
+    "max_experts": small(MIX, name="max_experts", E=1024, k=8, T=64, d=128, F=64),
+    "max_k": small(MIX, name="max_k", E=64, k=32, T=40, d=128, F=64, renormalize=True),
+}
+
+
+@pytest.mark.parametrize("name", list(MAX_CASES))
+def test_maximum_sizes_match_oracle(name):
+    parity(MAX_CASES[name])
+
+
+def test_routing_with_the_maximum_group_count():
+    cfg = small(DSK, name="max_groups", E=1024, k=8, n_group=32, topk_group=4, T=97, score="sigmoid",
+                selection_bias_std=0.1)
+    import mixture_experts_ffn_10_b200 as m
+    inputs = make_inputs(cfg, "cuda", with_weights=False)
+    idx, w = m.route(cfg, inputs)
+    torch.cuda.synchronize()
+    check_routing(oracle.Problem(cfg, host(inputs)), idx, w)
