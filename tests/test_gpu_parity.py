@@ -268,3 +268,27 @@ def test_routing_with_the_maximum_group_count():
     idx, w = m.route(cfg, inputs)
     torch.cuda.synchronize()
     check_routing(oracle.Problem(cfg, host(inputs)), idx, w)
+
+
+def test_routing_with_nan_and_infinite_logits():
+    """NaN keys rank below every number (ties to the lower index); sigmoid(+inf) = 1 and
+    sigmoid(-inf) = 0 are ordinary keys.  Token 0 has only NaN logits (its weights are
+    NaN on both sides), token 1 only -inf and one NaN (weights 0 after the clamp)."""
+    cfg = small(MIX, name="route_nonfinite", E=32, k=4, T=65, score="sigmoid", renormalize=True)
+    g = torch.Generator().manual_seed(7)
+    logits = torch.randn(cfg.T, cfg.E, generator=g)
+    logits[torch.rand(cfg.T, cfg.E, generator=g) < 0.10] = float("nan")
+    logits[torch.rand(cfg.T, cfg.E, generator=g) < 0.05] = float("inf")
+    logits[torch.rand(cfg.T, cfg.E, generator=g) < 0.05] = float("-inf")
+    logits[0] = float("nan")
+    logits[1, :] = float("-inf")
+    logits[1, 5] = float("nan")
+    logits = logits.to(torch.bfloat16)
+    import mixture_experts_ffn_10_b200 as m
+    inputs = {"logits": logits.cuda()}
+    idx, w = m.route(cfg, inputs)
+    torch.cuda.synchronize()
+    p = oracle.Problem(cfg, host(inputs))
+    ri, rw, _, _ = p.route(0)
+    assert np.array_equal(idx[0].cpu().numpy(), ri) and np.isnan(rw).all() and torch.isnan(w[0]).all()
+    check_routing(p, idx, w, tokens=range(1, cfg.T))
