@@ -292,3 +292,14 @@ def test_routing_with_nan_and_infinite_logits():
     ri, rw, _, _ = p.route(0)
     assert np.array_equal(idx[0].cpu().numpy(), ri) and np.isnan(rw).all() and torch.isnan(w[0]).all()
     check_routing(p, idx, w, tokens=range(1, cfg.T))
+
+
+def test_every_token_on_the_same_two_experts():
+    """Extreme skew: experts 3 and 5 take all 600 tokens (five 128-row tiles each, a
+    ragged last one), the other six experts are empty."""
+    cfg = small(MIX, name="two_hot_experts", T=600, E=8, k=2)
+    g = torch.Generator().manual_seed(11)
+    logits = torch.randn(cfg.T, cfg.E, generator=g) * 0.1
+    logits[:, 3] += 4.0
+    logits[:, 5] += 3.0
+    parity(cfg, override={"logits": logits.to(torch.bfloat16)})
