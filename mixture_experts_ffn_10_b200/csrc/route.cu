@@ -1,5 +1,6 @@
-// route.cu -- routing kernel: one warp per token (the per-token work is route_token
-// in route.cuh, shared with the small-batch front kernel).
+// route.cu -- routing kernel: one warp per token picks k of E experts and their
+// weights ("Struct MoeSpec" score, selection_bias, groups, renormalize, scale; the
+// per-token steps and their definitions are in route.cuh).
 #include "route.cuh"
 
 namespace moe {

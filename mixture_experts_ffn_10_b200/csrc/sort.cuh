@@ -1,7 +1,6 @@
-// sort.cuh -- block-level pieces of the expert sort shared by the sort kernels and
-// the small-batch front kernel: a block-wide exclusive scan, the segment scan
-// (offsets and per-GEMM tile prefixes), and the stable in-order scatter of one
-// chunk of (token, slot) entries.
+// sort.cuh -- block-level pieces of the expert sort used by the sort kernels: a
+// block-wide exclusive scan, the segment scan (offsets and per-GEMM tile
+// prefixes), and the stable in-order scatter of one chunk of (token, slot) entries.
 #pragma once
 
 #include "common.cuh"
