@@ -8,6 +8,7 @@
 // or a bias without its slot; a dtype it cannot serve is Unsupported), mapped
 // to status codes.
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdarg>
@@ -113,15 +114,16 @@ int check_tensors(const moe_shape* s, const moe_options* o, const moe_tensors* t
 }
 
 int num_sms_of_current_device() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64] = {};  // callers may race: each writes the same value
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = n > 0 ? n : 148;
+    if (n <= 0) n = 148;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 template <typename P>

@@ -28,6 +28,8 @@
 //   warps 2-5  epilogue of this CTA's 128 accumulator rows; each warp signals the
 //              even CTA's `tempty` barrier when it has read an accumulator buffer.
 // Every wait is bounded (2 s) and reports MOE_ERR_TIMEOUT through the status word.
+#include <atomic>
+
 #include "epilogue.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
@@ -308,10 +310,11 @@ bool map_down(CUtensorMap* m, const void* base, uint64_t F, uint64_t d, uint64_t
 // Co-resident clusters of the kernel on the current device (cached per device and mode).
 template <int MODE>
 int max_clusters(int num_sms) {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64] = {};  // callers may race: each writes the same value
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms / 2;
-  if (cache[dev] > 0) return cache[dev];
+  const int cached = cache[dev].load(std::memory_order_relaxed);
+  if (cached > 0) return cached;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * (unsigned)(num_sms / 2), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -321,7 +324,7 @@ int max_clusters(int num_sms) {
     (void)cudaGetLastError();
     n = num_sms / 2;
   }
-  cache[dev] = n;
+  cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
