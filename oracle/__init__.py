@@ -66,27 +66,31 @@ class _Problem(C.Structure):
 _lib = None
 
 
+def _bind(lib):
+    """Declares the argument and result types of the oracle's C functions on ``lib``."""
+    P = C.POINTER(_Problem)
+    lib.orc_route.argtypes = [P, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
+    lib.orc_route.restype = C.c_int
+    lib.orc_expert.argtypes = [P, C.c_int64, C.c_void_p, C.c_void_p]
+    lib.orc_expert.restype = C.c_int
+    lib.orc_token.argtypes = [P, C.c_int64, C.c_void_p]
+    lib.orc_token.restype = C.c_int
+    lib.orc_forward.argtypes = [P, C.c_void_p, C.c_int64, C.c_void_p, C.c_int]
+    lib.orc_forward.restype = C.c_int
+    lib.orc_bf16.argtypes = [C.c_uint16]
+    lib.orc_bf16.restype = C.c_double
+    lib.orc_e2m1.argtypes = [C.c_int]
+    lib.orc_e2m1.restype = C.c_double
+    lib.orc_e8m0.argtypes = [C.c_int]
+    lib.orc_e8m0.restype = C.c_double
+    lib.orc_max_threads.restype = C.c_int
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = C.CDLL(build())
-        P = C.POINTER(_Problem)
-        lib.orc_route.argtypes = [P, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
-        lib.orc_route.restype = C.c_int
-        lib.orc_expert.argtypes = [P, C.c_int64, C.c_void_p, C.c_void_p]
-        lib.orc_expert.restype = C.c_int
-        lib.orc_token.argtypes = [P, C.c_int64, C.c_void_p]
-        lib.orc_token.restype = C.c_int
-        lib.orc_forward.argtypes = [P, C.c_void_p, C.c_int64, C.c_void_p, C.c_int]
-        lib.orc_forward.restype = C.c_int
-        lib.orc_bf16.argtypes = [C.c_uint16]
-        lib.orc_bf16.restype = C.c_double
-        lib.orc_e2m1.argtypes = [C.c_int]
-        lib.orc_e2m1.restype = C.c_double
-        lib.orc_e8m0.argtypes = [C.c_int]
-        lib.orc_e8m0.restype = C.c_double
-        lib.orc_max_threads.restype = C.c_int
-        _lib = lib
+        _lib = _bind(C.CDLL(build()))
     return _lib
 
 

@@ -85,10 +85,14 @@ def test_routing_with_ties_and_groups(E, k, G, TG):
     check_routing(oracle.Problem(cfg, host(inputs)), idx, w)
 
 
-@pytest.mark.parametrize("score,sel", [("softmax", 0.0), ("softmax", 0.05), ("sigmoid", 0.1)])
-def test_routing_scores(score, sel):
+@pytest.mark.parametrize("score,sel,groups", [("softmax", 0.0, 0), ("softmax", 0.05, 0), ("sigmoid", 0.1, 0),
+                                              ("softmax", 0.05, 8), ("softmax", 0.1, 12)])
+def test_routing_scores(score, sel, groups):
+    # softmax with a selection bias ranks by softmax(l') + B ("Struct MoeSpec" selection_bias),
+    # with and without a group limit
     cfg = small(MIX, name="route_scores", E=96, k=6, T=513, score=score, selection_bias_std=sel,
-                router_bias=True, renormalize=score == "sigmoid", routed_scale=2.5)
+                router_bias=True, renormalize=score == "sigmoid", routed_scale=2.5,
+                n_group=groups, topk_group=groups // 2)
     import mixture_experts_ffn_10_b200 as m
     inputs = make_inputs(cfg, "cuda", with_weights=False)
     idx, w = m.route(cfg, inputs)

@@ -227,6 +227,73 @@ def test_selection_bias_changes_choice_not_weight(oracle_lib):
         assert ib.tolist() == _best_subset(kb, range(E), k)
 
 
+def test_softmax_selection_bias_worked_example(oracle_lib):
+    """"Struct MoeSpec" selection_bias on a softmax score: chosen by s + B, weighed by s.
+    The fixture's numbers are chosen so that biasing the logit instead (l + B, or
+    softmax(l + B), which ranks the same way) or ignoring B picks (3, 2), not (3, 0)."""
+    logits = torch.log(torch.arange(1, 5, dtype=torch.float32)).reshape(1, 4)
+    bias = torch.tensor([0.25, 0.125, 0.0, 0.0])
+    for case, renorm, scale, i0, i1, w0, w1 in _rows("routing_selection_bias_example.txt"):
+        cfg = _cfg(T=1, E=4, k=2, renormalize=bool(int(renorm)), routed_scale=float(scale))
+        p, _ = _problem(cfg, logits=logits, selection_bias=bias)
+        idx, w, keys, s = p.route(0)
+        assert idx.tolist() == [int(i0), int(i1)], case
+        assert np.allclose(w, [float(w0), float(w1)], rtol=1e-6, atol=0), case
+        assert np.allclose(keys, [0.35, 0.325, 0.3, 0.4], rtol=1e-6, atol=0), case
+
+
+def _independent_keys(lp, score, bias):
+    """Selection keys computed here, outside the oracle: score(l') + B (scipy)."""
+    s = sp.softmax(lp) if score == "softmax" else sp.expit(lp)
+    return s, s + (bias if bias is not None else 0.0)
+
+
+@pytest.mark.parametrize("score,E,k,renorm,S", [
+    ("softmax", 6, 2, True, 1.0), ("softmax", 9, 3, False, 1.0), ("softmax", 12, 4, True, 2.5),
+    ("sigmoid", 8, 3, True, 2.5), ("sigmoid", 11, 2, False, 1.0)])
+def test_biased_selection_matches_brute_force_on_independent_keys(oracle_lib, score, E, k, renorm, S):
+    """Random l' and B ~ N(0, 0.1): the chosen set is the best k-subset by
+    (score(l') + B descending, index ascending) with the scores computed by scipy,
+    and the weights are the unbiased scores of that set (renormalized, times S)."""
+    T = 40
+    cfg = _cfg(T=T, E=E, k=k, score=score, renormalize=renorm, routed_scale=S,
+               selection_bias_std=0.1, router_bias=True)
+    p, t = _problem(cfg)
+    lp = (t["logits"].float() + t["router_bias"].float()).double().numpy()  # fp32 add
+    bias = t["selection_bias"].double().numpy()
+    for tok in range(T):
+        s, key = _independent_keys(lp[tok], score, bias)
+        want = _best_subset(key, range(E), k)
+        idx, w, _, _ = p.route(tok)
+        assert idx.tolist() == want, tok
+        ws = s[want]
+        if renorm:
+            ws = ws / max(ws.sum(), 2.0 ** -14)
+        assert np.allclose(w, ws * _f32(S), rtol=1e-12, atol=0), tok
+
+
+@pytest.mark.parametrize("score", ["softmax", "sigmoid"])
+def test_biased_group_selection_matches_exhaustive_search_on_independent_keys(oracle_lib, score):
+    """Groups on keys score(l') + B computed outside the oracle: a group scores the
+    sum of its best two keys (any pair), the best topk_group groups are kept, then the
+    best k experts among them."""
+    E, G, TG, k = 12, 4, 2, 3
+    per = E // G
+    cfg = _cfg(T=40, E=E, k=k, score=score, n_group=G, topk_group=TG, selection_bias_std=0.1)
+    p, t = _problem(cfg)
+    lp = t["logits"].double().numpy()
+    bias = t["selection_bias"].double().numpy()
+    for tok in range(40):
+        _, key = _independent_keys(lp[tok], score, bias)
+        gs = [max(key[a] + key[b] for a, b in itertools.combinations(range(q * per, (q + 1) * per), 2))
+              for q in range(G)]
+        best_groups = min(itertools.combinations(range(G), TG),
+                          key=lambda sub: sorted((-gs[q], q) for q in sub))
+        cand = [e for q in sorted(best_groups) for e in range(q * per, (q + 1) * per)]
+        idx, _, _, _ = p.route(tok)
+        assert idx.tolist() == _best_subset(key, cand, k), tok
+
+
 @pytest.mark.parametrize("sel_std", [0.0, 0.1])
 def test_group_limited_selection_matches_exhaustive_search(oracle_lib, sel_std):
     E, G, TG, k = 16, 4, 2, 3
