@@ -214,18 +214,32 @@ MOE_API int moe_forward_events(const moe_shape *shape, const moe_options *opts, 
  * the same as moe_forward, run on a static scratch array of
  * MOE_NOALLOC_WORKSPACE_BYTES inside the library, held by every GPU that
  * loads the library until the process exits.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *   - The first call in each CUDA context (the device's primary context, or a
+ *     caller's own context current on the calling thread) looks up the array's
+ *     device address there (cudaGetSymbolAddress, with that device current) and
+ *     caches it for that context; make that first call before any stream
+ *     capture.
  *   - Problems whose moe_workspace_size() exceeds the array are rejected with
  *     MOE_ERR_WORKSPACE (nothing is launched); use moe_forward for them.
- *   - All calls share the array: calls that overlap on the GPU (other streams
- *     or threads) race and give wrong results; serialise them.
- *   - It calls no cudaMalloc or cudaFree.  Other errors as moe_forward.
+ *   - All calls share the array and it keeps the last call's contents: calls
+ *     that overlap on the GPU (other streams or threads) race and give wrong
+ *     results; serialise them.
+ *   - It calls no cudaMalloc or cudaFree.  Other errors as moe_forward; the
+ *     device status word lives in the array, read it with
+ *     moe_noalloc_debug_status.
  */
 #define MOE_NOALLOC_WORKSPACE_BYTES (64u << 20)
 MOE_API int moe_forward_noalloc(const moe_shape *shape, const moe_options *opts, const moe_tensors *t,
                                 void *stream);
+
+/* moe_debug_status for moe_forward_noalloc: synchronises `stream` and reads the
+ * device status word the last call on the current context left in the static
+ * array (no counterpart on the pages). */
+MOE_API int moe_noalloc_debug_status(void *stream);
+
+/* Size in bytes of the static scratch array (MOE_NOALLOC_WORKSPACE_BYTES of the
+ * library as built). */
+MOE_API size_t moe_noalloc_workspace_bytes(void);
 
 /* Number of CUDA kernels one moe_forward of this problem launches (-1 if the
  * arguments are invalid; 0 for T == 0).  For launch accounting. */

@@ -58,7 +58,6 @@ class moe_tensors(C.Structure):
 
 _P = C.POINTER
 MOE_STAGE_EVENTS = 7
-MOE_NOALLOC_WORKSPACE_BYTES = 64 << 20
 STAGES = ("route", "sort", "gather", "gate_up", "down", "combine")
 
 
@@ -77,6 +76,10 @@ def _bind(lib: C.CDLL) -> C.CDLL:
     lib.moe_forward_events.restype = C.c_int
     lib.moe_forward_noalloc.argtypes = [_P(moe_shape), _P(moe_options), _P(moe_tensors), C.c_void_p]
     lib.moe_forward_noalloc.restype = C.c_int
+    lib.moe_noalloc_debug_status.argtypes = [C.c_void_p]
+    lib.moe_noalloc_debug_status.restype = C.c_int
+    lib.moe_noalloc_workspace_bytes.argtypes = []
+    lib.moe_noalloc_workspace_bytes.restype = C.c_size_t
     lib.moe_forward_kernel_count.argtypes = [_P(moe_shape), _P(moe_options)]
     lib.moe_forward_kernel_count.restype = C.c_int
     lib.moe_last_error.argtypes = []
@@ -106,7 +109,8 @@ class _UnbuiltLibrary:
 _lib = _bind(C.CDLL(LIB_PATH)) if os.path.exists(LIB_PATH) else _UnbuiltLibrary()
 
 EXPORTED = ("moe_options_init", "moe_workspace_size", "moe_forward", "moe_route",
-            "moe_forward_events", "moe_forward_noalloc", "moe_forward_kernel_count",
+            "moe_forward_events", "moe_forward_noalloc", "moe_noalloc_debug_status",
+            "moe_noalloc_workspace_bytes", "moe_forward_kernel_count",
             "moe_last_error", "moe_debug_status", "moe_version")
 
 
@@ -148,6 +152,16 @@ def moe_forward_events(shape, opts, tensors, workspace: int, workspace_bytes: in
 def moe_forward_noalloc(shape, opts, tensors, stream: int) -> int:
     """moe_forward on the library's static scratch array (no workspace argument)."""
     return _lib.moe_forward_noalloc(C.byref(shape), C.byref(opts), C.byref(tensors), stream)
+
+
+def moe_noalloc_debug_status(stream: int) -> int:
+    """Device status word of the last moe_forward_noalloc on the current context."""
+    return _lib.moe_noalloc_debug_status(stream)
+
+
+def moe_noalloc_workspace_bytes() -> int:
+    """Size of the library's static scratch array (read from the library)."""
+    return _lib.moe_noalloc_workspace_bytes()
 
 
 def moe_forward_kernel_count(shape, opts) -> int:

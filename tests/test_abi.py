@@ -26,8 +26,16 @@ def _declared():
 def test_header_declares_the_entry_points():
     assert _declared() == sorted(["moe_options_init", "moe_workspace_size", "moe_forward",
                                   "moe_route", "moe_forward_events", "moe_forward_noalloc",
+                                  "moe_noalloc_debug_status", "moe_noalloc_workspace_bytes",
                                   "moe_forward_kernel_count", "moe_last_error", "moe_debug_status",
                                   "moe_version"])
+
+
+def test_static_scratch_size_matches_the_header(moe):
+    with open(os.path.join(ROOT, "include", "moe.h")) as f:
+        m = re.search(r"#define MOE_NOALLOC_WORKSPACE_BYTES \((\d+)u << (\d+)\)", f.read())
+    assert m, "MOE_NOALLOC_WORKSPACE_BYTES not found in the header"
+    assert moe.moe_noalloc_workspace_bytes() == int(m.group(1)) << int(m.group(2))
 
 
 def test_library_exports_every_declared_symbol(moe):

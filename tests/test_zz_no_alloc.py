@@ -5,7 +5,6 @@ owns all device memory, a request path that must not call cudaMalloc) use this
 entry point instead of passing a workspace.  This file is collected last so
 that a run stopping at its first failure has already run every other test.
 """
-import numpy as np
 import pytest
 import torch
 
@@ -13,37 +12,37 @@ from workloads import CONFIGS, make_inputs, small
 
 pytestmark = pytest.mark.gpu
 
-TOL = 2e-2  # bf16 output tolerance of the parity tests (of max|y|)
-
 
 def _cfg(seed):
     return small(CONFIGS["decode_T64"], name="noalloc", T=96, d=512, F=384, E=32, k=4, seed=seed)
 
 
 def test_noalloc_entry_matches_moe_forward_on_two_calls_in_a_row():
+    """Both entry points run the same bitwise-reproducible forward, one on a caller
+    workspace and one on the static array, so their outputs must be identical; two
+    calls in a row with different inputs also show that nothing stale from the
+    previous call's scratch contents leaks into the next."""
     import mixture_experts_ffn_10_b200 as m
     stream = torch.cuda.current_stream().cuda_stream
-    for seed in (2101, 2102):  # two calls in a row, different inputs each time
+    for seed in (2101, 2102):
         cfg = _cfg(seed)
         inputs = make_inputs(cfg, "cuda")
         ref = m.forward(cfg, inputs)          # the existing entry point, caller workspace
         y = torch.full_like(inputs["x"], float("nan"))
         shape, opts = m.shape_of(cfg), m.options_of(cfg)
-        assert m.moe_workspace_size(shape, opts) <= m.MOE_NOALLOC_WORKSPACE_BYTES
+        assert m.moe_workspace_size(shape, opts) <= m.moe_noalloc_workspace_bytes()
         rc = m.moe_forward_noalloc(shape, opts, m.tensors_of(inputs, y), stream)
         assert rc == m.MOE_OK, m.moe_last_error()
+        assert m.moe_noalloc_debug_status(stream) == m.MOE_OK
         torch.cuda.synchronize()
-        a = y.float().cpu().numpy()
-        b = ref.float().cpu().numpy()
-        assert np.isfinite(a).all()
-        assert np.abs(a - b).max() <= TOL * np.abs(b).max()
+        assert torch.equal(y, ref)
 
 
 def test_noalloc_entry_rejects_problems_beyond_its_scratch():
     import mixture_experts_ffn_10_b200 as m
     cfg = small(CONFIGS["mixtral_bf16"], T=4096)
     shape, opts = m.shape_of(cfg), m.options_of(cfg)
-    assert m.moe_workspace_size(shape, opts) > m.MOE_NOALLOC_WORKSPACE_BYTES
+    assert m.moe_workspace_size(shape, opts) > m.moe_noalloc_workspace_bytes()
     t = m.moe_tensors()
     fake = 1 << 20
     for n in ("x", "router_logits", "gate_up", "down"):
