@@ -1,11 +1,14 @@
 """Parity at the full workload sizes the benchmark times (same entry point and launch).
 
-Every token's routing is compared bit-exactly with the oracle; outputs are
-compared element by element on a sample of tokens (first, last and seeded
-random ones), which the oracle computes one by one; and the forward is run
-twice to check bitwise determinism at full size.  Weights of experts the
-sampled tokens do not use are never copied to the host (the host arrays are
-lazily zero-filled).
+Every token's routing is compared bit-exactly with the oracle.  Outputs are
+compared element by element on a sample of tokens that the oracle computes one
+by one: for every expert that receives rows, the tokens of its first and last
+row and of the rows on both sides of every 128-row boundary inside its segment
+(the GEMM tile edges of both the 128- and the 256-row tiles), up to a budget,
+plus the first and last token of the batch; batches of at most 256 tokens are
+compared on every token.  The forward is run twice to check bitwise
+determinism at full size.  Weights of experts the sampled tokens do not use are
+never copied to the host (the host arrays are lazily zero-filled).
 """
 import numpy as np
 import pytest
@@ -20,7 +23,8 @@ pytestmark = pytest.mark.gpu
 
 FULL = ["tiny_fp32", "mixtral_bf16", "gptoss_mxfp4", "deepseek_bf16", "decode_T1", "decode_T8",
         "decode_T64", "decode_T256"]
-N_SAMPLE = 6
+MAX_SAMPLE = 160   # tokens the oracle recomputes per workload (about 10-15 s on 16 host cores)
+ALL_TOKENS_UP_TO = 256
 
 
 def _np(t):
@@ -28,6 +32,41 @@ def _np(t):
     if t.dtype == torch.bfloat16:
         t = t.view(torch.int16)
     return t
+
+
+def boundary_sample(idx, E, seed, budget=MAX_SAMPLE, tile=128):
+    """Tokens whose rows sit at the edges of each expert's segment and of its
+    row tiles (rows are token-ascending inside an expert's segment)."""
+    T = idx.shape[0]
+    if T <= ALL_TOKENS_UP_TO:
+        return list(range(T))
+    per_expert = [[] for _ in range(E)]
+    for t, row in enumerate(idx.tolist()):
+        for e in row:
+            per_expert[e].append(t)
+    # one list of edge tokens per expert, nearest edges first
+    edges = []
+    for toks in per_expert:
+        n = len(toks)
+        if n == 0:
+            continue
+        pos = [0, n - 1]
+        for b in range(tile, n, tile):
+            pos += [b - 1, b]
+        edges.append([toks[i] for i in dict.fromkeys(pos)])
+    rng = np.random.default_rng(seed)
+    rng.shuffle(edges)
+    chosen = {0, T - 1}
+    depth = 0
+    # round robin over the experts: every expert's first edge, then every second, ...
+    while len(chosen) < budget and any(depth < len(e) for e in edges):
+        for e in edges:
+            if depth < len(e):
+                chosen.add(e[depth])
+                if len(chosen) >= budget:
+                    break
+        depth += 1
+    return sorted(chosen)
 
 
 def _host_sparse(inputs, experts):
@@ -75,8 +114,7 @@ def _full_size(name):
     idx_h, w_h = idx.cpu().numpy(), w.cpu().numpy()
     routing_only = {k: inputs[k] for k in ("logits", "router_bias", "selection_bias")}
     pr = oracle.Problem(cfg, {k: (None if v is None else v.cpu()) for k, v in routing_only.items()})
-    rng = np.random.default_rng(cfg.seed)
-    sample = sorted({0, cfg.T - 1, *rng.integers(0, cfg.T, N_SAMPLE - 2).tolist()})
+    sample = boundary_sample(idx.cpu().numpy(), cfg.E, cfg.seed)
     for t in range(cfg.T):
         ri, rw, _, _ = pr.route(t)
         assert np.array_equal(idx_h[t], ri), f"token {t}: {idx_h[t]} vs {ri}"
