@@ -40,18 +40,33 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer tokens/s; achieved TFLOP/s or HBM GB/s as % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# ncu dram bytes (read + write) per launch of the dominant kernel, per workload, from the
-# profile summaries under profiles/ (None until captured for the current kernel version).
-NCU_TRAFFIC = {  # median dram__bytes_read.sum + dram__bytes_write.sum per launch: profiles/launches_<workload>.md
-    ("mixtral_bf16", "gate_up"): 2925367552 + 242864000,
-    ("mixtral_bf16", "down"): 1662191232 + 71625088,
-    ("deepseek_bf16", "gate_up"): 15873404672 + 468926208,
-    ("deepseek_bf16", "down"): 6651168128 + 1050486016,
-    ("decode_T1", "gate_up"): 203038592 + 206080,
-    ("decode_T1", "down"): 100721536 + 144000,
-    ("gptoss_mxfp4", "gate_up"): 329679232 + 35157760,
-    ("gptoss_mxfp4", "down"): 188540544 + 26514816,
-}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a workload's
+# dominant GEMM, each from one ncu capture of that kernel, keyed with the hash of the CUDA
+# sources the captured library was built from (kernel_sources_hash).  A figure whose hash
+# is not the current sources' belongs to an older kernel and is reported as null.
+NCU_TRAFFIC = {}
+
+
+def kernel_sources_hash() -> str:
+    """Short hash of the library's CUDA sources (csrc/*.cu, *.cuh) and its header."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mixture_experts_ffn_10_b200", "csrc")
+    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    for f in files + [os.path.join(ROOT, "include", "moe.h")]:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def ncu_traffic(workload: str, stage: str):
+    """ncu DRAM bytes per launch for this workload and stage, or None if not captured
+    for the current sources."""
+    rec = NCU_TRAFFIC.get((workload, stage))
+    if rec is None or rec[1] != kernel_sources_hash():
+        return None
+    return rec[0]
 
 
 def peaks():
@@ -224,6 +239,97 @@ def stage_model(cfg, distinct):
         "down": {"flops": 2.0 * (R * cfg.d * cfg.F + cfg.T * cfg.d * cfg.Fs),
                  "bytes": dn_w + (R + (cfg.T if cfg.Fs else 0)) * (cfg.F + cfg.d) * ab},
     }
+
+
+def measure_workload(cfg, steps, warmup, flush, stream):
+    """Device-timed summary of one more workload (rank-local): CUDA-graph replays of
+    moe_forward with the L2 flushed before each, then each GEMM stage alone between
+    two library events (one graph per stage), and the roofline of the dominant one."""
+    import torch
+
+    import mixture_experts_ffn_10_b200 as moe
+    from workloads import algorithmic_bytes, flops, make_inputs
+
+    inputs = make_inputs(cfg, "cuda")
+    shape, opts = moe.shape_of(cfg), moe.options_of(cfg)
+    ws = moe.Workspace(moe.moe_workspace_size(shape, opts))
+    y = torch.empty_like(inputs["x"])
+    idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    tens = moe.tensors_of(inputs, y, idx, None)
+    sptr = stream.cuda_stream
+    names = list(moe.STAGES)
+
+    def call(handles=None):
+        rc = (moe.moe_forward(shape, opts, tens, ws.ptr, ws.nbytes, sptr) if handles is None else
+              moe.moe_forward_events(shape, opts, tens, ws.ptr, ws.nbytes, sptr, handles))
+        if rc != 0:
+            raise moe.MoeError(rc, moe.moe_last_error())
+
+    def capture(handles=None):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            call(handles)
+        torch.cuda.synchronize()
+        return g
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush.zero_()
+            call()
+    torch.cuda.synchronize()
+    graphs = [capture()]
+    stage_ev = {}
+    for st in ("gate_up", "down"):
+        s_i = names.index(st)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        for ev in evs:
+            ev.record(stream)
+        h = [None] * moe.MOE_STAGE_EVENTS
+        h[s_i], h[s_i + 1] = evs[0].cuda_event, evs[1].cuda_event
+        stage_ev[st] = evs
+        graphs.append(capture(h))
+    t0s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    t1s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    stage_ms = {"gate_up": 0.0, "down": 0.0}
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            flush.zero_()
+            t0s[i].record(stream)
+            graphs[0].replay()
+            t1s[i].record(stream)
+        for gi, st in ((1, "gate_up"), (2, "down")):
+            for _ in range(steps):
+                flush.zero_()
+                graphs[gi].replay()
+                torch.cuda.synchronize()
+                stage_ms[st] += stage_ev[st][0].elapsed_time(stage_ev[st][1]) / steps
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in zip(t0s, t1s)) / steps
+    status = moe.moe_debug_status(ws.ptr, sptr)
+    if status != 0:
+        raise RuntimeError(f"{cfg.name}: device status {moe.STATUS_NAMES.get(status, status)}")
+    distinct = int(torch.unique(idx).numel())
+    rows = torch.bincount(idx.flatten().long(), minlength=cfg.E)
+    pk, pk_src = peaks()
+    model = stage_model(cfg, distinct)
+    dom = max(stage_ms, key=stage_ms.get)
+    m, t_dom = model[dom], stage_ms[dom] / 1e3
+    tensor = m["flops"] / pk["bf16_tflops"] / 1e12 >= m["bytes"] / pk["hbm_gbs"] / 1e9
+    achieved = m["flops"] / t_dom / 1e12 if tensor else m["bytes"] / t_dom / 1e9
+    peak = pk["bf16_tflops"] if tensor else pk["hbm_gbs"]
+    lf, lb = flops(cfg), algorithmic_bytes(cfg, distinct)
+    del graphs
+    return {"workload": workload_name(cfg), "ms_per_step": ms, "tokens_per_s": cfg.T / (ms / 1e3),
+            "stage_ms": stage_ms,
+            "roofline": {"kernel": f"{dom} grouped GEMM", "bound": "tensor" if tensor else "hbm",
+                         "achieved": achieved, "unit": "TFLOP/s" if tensor else "GB/s", "peak": peak,
+                         "frac": achieved / peak, "peak_source": f"{pk_src} (burst)",
+                         "traffic": ncu_traffic(cfg.name, dom)},
+            "layer": {"tensor_frac": lf / (ms / 1e3) / 1e12 / pk["bf16_tflops"],
+                      "hbm_frac": lb / (ms / 1e3) / 1e9 / pk["hbm_gbs"], "distinct_experts": distinct,
+                      "rows_per_expert_max": int(rows.max()), "empty_experts": int((rows == 0).sum())},
+            "gpu_launches_per_step": moe.moe_forward_kernel_count(shape, opts),
+            "timed": f"{steps} CUDA-graph replays after {warmup} warm-up calls, L2 flushed before each"}
 
 
 def run_own(args, cfg):
@@ -461,7 +567,8 @@ def run_own(args, cfg):
                 "unit": unit, "frac": achieved / peak, "peak_source": f"{pk_src} (burst)",
                 "frac_vs_sustained_peak": (achieved / sustained) if sustained else None,
                 # the figures belong to the kernels the library picks by itself
-                "traffic": None if os.environ.get("MOE_B200_PAIR_GEMM") else NCU_TRAFFIC.get((cfg.name, dom)),
+                "traffic": None if os.environ.get("MOE_B200_PAIR_GEMM") else ncu_traffic(cfg.name, dom),
+                "kernel_sources": kernel_sources_hash(),
                 "algorithmic_per_launch": m["flops"] if bound == "tensor" else m["bytes"],
                 "kernel_ms": dom_ms,
                 "timed": "CUDA events around this stage only (GEMM + split-K reduction), "
@@ -509,6 +616,24 @@ def run_own(args, cfg):
         v, n, dt, threads = oracle_sample(cfg, hin, budget_s=args.cpu_budget)
         out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                "sample": f"{n} of {cfg.T} tokens (whole layer per token), {dt:.1f} s"}
+    # ------------------------------------------------------------ the other workloads (N=1)
+    # Device-timed summaries of every other workload of the benchmark suite in the same
+    # run, so that one default invocation measures them all (the fields above stay the
+    # default workload's).
+    if world == 1 and args.workloads == "all":
+        from workloads import CONFIGS
+        del tens, ws, inputs, y, slots, xb, lb, yb
+        torch.cuda.empty_cache()
+        others = {}
+        sampler2 = ClockSampler(physical_gpu_index(local))
+        for name, ocfg in CONFIGS.items():
+            if name == cfg.name:
+                continue
+            others[name] = measure_workload(ocfg, args.other_steps, 3, flush, stream)
+            torch.cuda.empty_cache()
+        out["other_workloads"] = others
+        out["other_workloads_clocks"] = sampler2.stop()
+
     if rank == 0:
         print(json.dumps(out), flush=True)
     if dist is not None:
@@ -524,6 +649,10 @@ def main():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--config", default="mixtral_bf16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workloads", default=None, choices=["all", "none"],
+                    help="also time every other workload briefly (default: all for the default "
+                         "workload at N=1, none otherwise)")
+    ap.add_argument("--other-steps", type=int, default=10, help="timed steps per other workload")
     ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of a CUDA graph replay")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle wall time")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
@@ -532,6 +661,8 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     from workloads import CONFIGS, small
+    if args.workloads is None:
+        args.workloads = "all" if args.config == "mixtral_bf16" and not args.set else "none"
     cfg = CONFIGS[args.config]
     for kv in args.set:
         k, v = kv.split("=", 1)
