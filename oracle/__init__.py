@@ -24,13 +24,15 @@ _LIB = os.path.join(_HERE, "libmoe_oracle.so")
 F32, BF16, MXFP4 = 0, 1, 2
 SOFTMAX, SIGMOID = 0, 1
 SILU, GELU_ERF, GELU_TANH, RELU, IDENTITY = 0, 1, 2, 3, 4
-CONCAT, INTERLEAVED = 0, 1
+CONCAT, INTERLEAVED, UNFUSED = 0, 1, 2
+GATED, PLAIN = 0, 1
 
 _DTYPE_CODE = {"f32": F32, "bf16": BF16, "mxfp4": MXFP4}
 _SCORE_CODE = {"softmax": SOFTMAX, "sigmoid": SIGMOID}
 _ACT_CODE = {"silu": SILU, "gelu_erf": GELU_ERF, "gelu_tanh": GELU_TANH, "relu": RELU,
              "identity": IDENTITY}
-_LAYOUT_CODE = {"concat": CONCAT, "interleaved": INTERLEAVED}
+_LAYOUT_CODE = {"concat": CONCAT, "interleaved": INTERLEAVED, "unfused": UNFUSED}
+_FFN_CODE = {"gated": GATED, "plain": PLAIN}
 
 
 def build(force: bool = False) -> str:
@@ -53,13 +55,15 @@ class _Problem(C.Structure):
         ("n_group", C.c_int32), ("topk_group", C.c_int32), ("weigh_inputs", C.c_int32),
         ("act", C.c_int32),
         ("alpha", C.c_double), ("beta", C.c_double), ("limit", C.c_double),
-        ("gu_layout", C.c_int32), ("shared_gate", C.c_int32),
+        ("gu_layout", C.c_int32), ("shared_gate", C.c_int32), ("ffn", C.c_int32),
         ("x", C.c_void_p), ("logits", C.c_void_p), ("router_bias", C.c_void_p),
         ("selection_bias", C.c_void_p),
         ("gate_up", C.c_void_p), ("gate_up_scales", C.c_void_p), ("gate_up_bias", C.c_void_p),
         ("down", C.c_void_p), ("down_scales", C.c_void_p), ("down_bias", C.c_void_p),
         ("shared_gate_up", C.c_void_p), ("shared_down", C.c_void_p),
         ("shared_gate_vec", C.c_void_p), ("shared_output", C.c_void_p),
+        ("gate", C.c_void_p), ("gate_scales", C.c_void_p), ("gate_bias", C.c_void_p),
+        ("router_weight", C.c_void_p),
     ]
 
 
@@ -112,7 +116,7 @@ def _arr(a):
 
 _TENSORS = ("x", "logits", "router_bias", "selection_bias", "gate_up", "gate_up_scales",
             "gate_up_bias", "down", "down_scales", "down_bias", "shared_gate_up", "shared_down",
-            "shared_gate_vec", "shared_output")
+            "shared_gate_vec", "shared_output", "gate", "gate_scales", "gate_bias", "router_weight")
 
 
 @dataclass
@@ -147,6 +151,7 @@ class Problem:
         p.limit = float(np.float32(c.limit))
         p.gu_layout = _LAYOUT_CODE[c.gu_layout]
         p.shared_gate = int(c.shared_gate)
+        p.ffn = _FFN_CODE[getattr(c, "ffn", "gated")]
         for n in _TENSORS:
             a = self._keep[n]
             setattr(p, n, None if a is None else a.ctypes.data)

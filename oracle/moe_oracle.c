@@ -54,7 +54,8 @@
 enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_MXFP4 = 2 };
 enum { ORC_SOFTMAX = 0, ORC_SIGMOID = 1 };
 enum { ORC_SILU = 0, ORC_GELU_ERF = 1, ORC_GELU_TANH = 2, ORC_RELU = 3, ORC_IDENTITY = 4 };
-enum { ORC_CONCAT = 0, ORC_INTERLEAVED = 1 };
+enum { ORC_CONCAT = 0, ORC_INTERLEAVED = 1, ORC_UNFUSED = 2 };
+enum { ORC_GATED = 0, ORC_PLAIN = 1 };
 
 typedef struct {
   int64_t T, d, F, E, k, Fs;
@@ -66,12 +67,18 @@ typedef struct {
   int32_t n_group, topk_group, weigh_inputs, act;
   double alpha, beta, limit;
   int32_t gu_layout, shared_gate;
+  int32_t ffn;          /* ORC_GATED: act(gate) * (up + beta); ORC_PLAIN: act(fc1) alone */
   /* host pointers; NULL = absent */
   const void *x, *logits, *router_bias;
   const float *selection_bias;
   const void *gate_up, *gate_up_scales, *gate_up_bias;
   const void *down, *down_scales, *down_bias;
   const void *shared_gate_up, *shared_down, *shared_gate_vec, *shared_output;
+  /* unfused layout: the gate stack [E, F, d] (w_dtype; MXFP4 scales [E, F, d/32])
+     and its bias [E, F]; gate_up then holds the up rows [E, F, d] and their bias */
+  const void *gate, *gate_scales, *gate_bias;
+  /* router weight Wr [d, E] (act dtype): logits = x Wr when logits is NULL */
+  const void *router_weight;
 } orc_problem;
 
 /* ---------------- decoders ---------------- */
@@ -153,9 +160,19 @@ int orc_route(const orc_problem *p, int64_t t, int32_t *idx, double *w, double *
   char *eligible = (char *)malloc(E);
   char *taken = (char *)malloc(E);
 
-  /* l' = l + Br, an fp32 add ([MoeSpec] router_bias: added to each logit before scoring) */
+  /* l' = l + Br, an fp32 add ([MoeSpec] router_bias: added to each logit before scoring).
+     Without caller logits, l = x_t Wr ([MoeSpec] wr, indexed wr[(i-1)E + e]: Wr is [d, E]),
+     summed in double over i and rounded once to fp32. */
   for (int64_t e = 0; e < E; e++) {
-    float l = load_f32(p->logits, p->logit_dtype, t * E + e);
+    float l;
+    if (p->logits) {
+      l = load_f32(p->logits, p->logit_dtype, t * E + e);
+    } else {
+      double acc = 0.0;
+      for (int64_t i = 0; i < p->d; i++)
+        acc += load(p->x, p->act_dtype, t * p->d + i) * load(p->router_weight, p->act_dtype, i * E + e);
+      l = (float)acc;
+    }
     if (p->router_bias) l = l + load_f32(p->router_bias, p->logit_dtype, e);
     lp[e] = l;
   }
@@ -267,10 +284,29 @@ static double gated(const orc_problem *p, double g, double u) {
   return a * (u + p->beta);
 }
 
+/* The non-gated expert's activation of fc1's output ([Op] activation_type relu, gelu,
+   silu or identity with fusion_size 1): the same functions without an up value,
+   alpha for SiLU only, no limit and no beta. */
+static double plain(const orc_problem *p, double g) {
+  switch (p->act) {
+  case ORC_SILU: return g * sigmoid(p->alpha * g);
+  case ORC_GELU_ERF: return 0.5 * g * (1.0 + erf(g / sqrt(2.0)));
+  case ORC_GELU_TANH: return 0.5 * g * (1.0 + tanh(sqrt(2.0 / acos(-1.0)) * (g + 0.044715 * g * g * g)));
+  case ORC_RELU: return g > 0.0 ? g : 0.0;
+  default: return g; /* identity */
+  }
+}
+
 /*
  * One expert on input z[d]: out[d] = W_down[e] h + b_down[e], with
- * h_f = gated(W_gate[e] z + b_gate[e], W_up[e] z + b_up[e]).
- * e == E selects the shared expert (act dtype weights, dff = Fs, no biases).
+ *   gated: h_f = gated(W_gate[e] z + b_gate[e], W_up[e] z + b_up[e]);
+ *   plain: h_f = plain(W_1[e] z + b_1[e])  ([Op] fc1 with fusion_size 1).
+ * Gate and up rows come from the fused stack (concat or interleaved) or, unfused,
+ * from the separate gate stack and the up stack ([MoE] set_weights gate_experts,
+ * gate_bias; [Op] fc3_experts_weights).
+ * e == E selects the shared expert (act dtype weights, dff = Fs, no biases; its
+ * stack is [2Fs, d] gate rows first when the routed experts are unfused, [Fs, d]
+ * for a plain FFN).
  */
 int orc_expert(const orc_problem *p, int64_t e, const double *z, double *out) {
   const int64_t d = p->d;
@@ -286,17 +322,35 @@ int orc_expert(const orc_problem *p, int64_t e, const double *z, double *out) {
   const void *bgu = shared ? NULL : p->gate_up_bias;
   const void *bd = shared ? NULL : p->down_bias;
   double *h = (double *)malloc(sizeof(double) * F);
-  for (int64_t f = 0; f < F; f++) {
-    int64_t rg = p->gu_layout == ORC_INTERLEAVED ? 2 * f : f;
-    int64_t ru = p->gu_layout == ORC_INTERLEAVED ? 2 * f + 1 : F + f;
-    double g = 0.0, u = 0.0;
-    for (int64_t i = 0; i < d; i++) g += weight(gu, gus, wdt, ee, 2 * F, d, rg, i) * z[i];
-    for (int64_t i = 0; i < d; i++) u += weight(gu, gus, wdt, ee, 2 * F, d, ru, i) * z[i];
-    if (bgu) {
-      g += load(bgu, p->act_dtype, ee * 2 * F + rg);
-      u += load(bgu, p->act_dtype, ee * 2 * F + ru);
+  if (p->ffn == ORC_PLAIN) {
+    for (int64_t f = 0; f < F; f++) {
+      double g = 0.0;
+      for (int64_t i = 0; i < d; i++) g += weight(gu, gus, wdt, ee, F, d, f, i) * z[i];
+      if (bgu) g += load(bgu, p->act_dtype, ee * F + f);
+      h[f] = plain(p, g);
     }
-    h[f] = gated(p, g, u);
+  } else if (p->gu_layout == ORC_UNFUSED && !shared) {
+    for (int64_t f = 0; f < F; f++) {
+      double g = 0.0, u = 0.0;
+      for (int64_t i = 0; i < d; i++) g += weight(p->gate, p->gate_scales, wdt, ee, F, d, f, i) * z[i];
+      for (int64_t i = 0; i < d; i++) u += weight(gu, gus, wdt, ee, F, d, f, i) * z[i];
+      if (p->gate_bias) g += load(p->gate_bias, p->act_dtype, ee * F + f);
+      if (bgu) u += load(bgu, p->act_dtype, ee * F + f);
+      h[f] = gated(p, g, u);
+    }
+  } else {
+    for (int64_t f = 0; f < F; f++) {
+      int64_t rg = p->gu_layout == ORC_INTERLEAVED ? 2 * f : f;
+      int64_t ru = p->gu_layout == ORC_INTERLEAVED ? 2 * f + 1 : F + f;
+      double g = 0.0, u = 0.0;
+      for (int64_t i = 0; i < d; i++) g += weight(gu, gus, wdt, ee, 2 * F, d, rg, i) * z[i];
+      for (int64_t i = 0; i < d; i++) u += weight(gu, gus, wdt, ee, 2 * F, d, ru, i) * z[i];
+      if (bgu) {
+        g += load(bgu, p->act_dtype, ee * 2 * F + rg);
+        u += load(bgu, p->act_dtype, ee * 2 * F + ru);
+      }
+      h[f] = gated(p, g, u);
+    }
   }
   for (int64_t o = 0; o < d; o++) {
     double acc = 0.0;

@@ -66,9 +66,9 @@ MUTATIONS = [
      [("test_softmax_and_sigmoid_scores_match_scipy", {})]),
     ("gate and up halves swapped",
      "int64_t rg = p->gu_layout == ORC_INTERLEAVED ? 2 * f : f;\n"
-     "    int64_t ru = p->gu_layout == ORC_INTERLEAVED ? 2 * f + 1 : F + f;",
+     "      int64_t ru = p->gu_layout == ORC_INTERLEAVED ? 2 * f + 1 : F + f;",
      "int64_t ru = p->gu_layout == ORC_INTERLEAVED ? 2 * f : f;\n"
-     "    int64_t rg = p->gu_layout == ORC_INTERLEAVED ? 2 * f + 1 : F + f;",
+     "      int64_t rg = p->gu_layout == ORC_INTERLEAVED ? 2 * f + 1 : F + f;",
      [("test_single_expert_equals_textbook_ffn",
        dict(act="silu", alpha=1.0, beta=0.0, limit=0.0)),
       ("test_expert_worked_example", {})]),
@@ -94,6 +94,18 @@ MUTATIONS = [
      "gate = sigmoid(dot);",
      "gate = 1.0 + 0.0 * dot;",
      [("test_shared_expert_with_sigmoid_gate", {})]),
+    ("plain FFN multiplies by beta as the gated form does",
+     "  case ORC_SILU: return g * sigmoid(p->alpha * g);",
+     "  case ORC_SILU: return g * sigmoid(p->alpha * g) * (1.0 + p->beta);",
+     [("test_plain_expert_equals_textbook_ffn", dict(act="silu", alpha=1.702))]),
+    ("unfused gate read from the up stack",
+     "g += weight(p->gate, p->gate_scales, wdt, ee, F, d, f, i) * z[i];",
+     "g += weight(gu, gus, wdt, ee, F, d, f, i) * z[i];",
+     [("test_unfused_gate_stack_equals_concat", {})]),
+    ("router weight read expert-major ([E, d])",
+     "load(p->router_weight, p->act_dtype, i * E + e);",
+     "load(p->router_weight, p->act_dtype, e * p->d + i);",
+     [("test_router_weight_worked_example", {}), ("test_router_weight_matches_numpy_matmul", {})]),
     ("SiLU limit not applied to the up value",
      "u = u < p->limit ? (u > -p->limit ? u : -p->limit) : p->limit;",
      ";",

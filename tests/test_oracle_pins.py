@@ -452,3 +452,98 @@ def test_thread_count_does_not_change_results(oracle_lib):
     cfg = _cfg(T=12, E=8, k=2)
     p, _ = _problem(cfg)
     assert np.array_equal(p.forward(nthreads=1), p.forward(nthreads=4))
+
+
+# ------------------------------------------------------------------ layouts, plain FFN, router weight
+
+
+def test_unfused_gate_stack_equals_concat(oracle_lib):
+    """Unfused ("MoE" set_weights gate_experts + gate_bias; graph-op fc3): the gate
+    rows come from their own stack and gate_up holds the up rows.  Stacking gate on
+    top of up gives the concatenated layout, which must give the same y."""
+    cfg = _cfg(T=10, d=32, F=24, E=4, k=2, expert_bias=True, gu_layout="unfused", Fs=16)
+    p, t = _problem(cfg)
+    cat = torch.cat([t["gate"], t["gate_up"]], 1)
+    cat_bias = torch.cat([t["gate_bias"], t["gate_up_bias"]], 1)
+    pc, _ = _problem(small(cfg, gu_layout="concat"), gate_up=cat, gate_up_bias=cat_bias, gate=None,
+                     gate_bias=None, shared_gate_up=t["shared_gate_up"], x=t["x"])
+    assert np.array_equal(p.forward(), pc.forward())
+
+
+def test_unfused_mxfp4_gate_stack_equals_concat(oracle_lib):
+    cfg = _cfg(T=5, d=64, F=32, E=3, k=2, w_dtype="mxfp4", act_dtype="bf16", logit_dtype="bf16",
+               gu_layout="unfused")
+    p, t = _problem(cfg)
+    pc, _ = _problem(small(cfg, gu_layout="concat"), gate_up=torch.cat([t["gate"], t["gate_up"]], 1),
+                     gate_up_scales=torch.cat([t["gate_scales"], t["gate_up_scales"]], 1), gate=None,
+                     gate_scales=None)
+    assert np.array_equal(p.forward(), pc.forward())
+
+
+def _plain_ffn(x, w1, wd, act, alpha, b1=None, bd=None):
+    """Textbook non-gated FFN with torch fp64 library activations."""
+    g = x @ w1.T + (b1 if b1 is not None else 0)
+    if act == "silu":
+        a = g * torch.sigmoid(alpha * g)
+    elif act == "gelu_erf":
+        a = Fn.gelu(g, approximate="none")
+    elif act == "gelu_tanh":
+        a = Fn.gelu(g, approximate="tanh")
+    elif act == "relu":
+        a = Fn.relu(g)
+    else:
+        a = g
+    return a @ wd.T + (bd if bd is not None else 0)
+
+
+@pytest.mark.parametrize("act,alpha", [("silu", 1.0), ("silu", 1.702), ("gelu_erf", 1.0),
+                                       ("gelu_tanh", 1.0), ("relu", 1.0), ("identity", 1.0)])
+def test_plain_expert_equals_textbook_ffn(oracle_lib, act, alpha):
+    """Graph-op page "MoE": fc1 [E, fusion_size * inter, hidden] with fusion_size 1 and
+    activation_type relu / gelu / silu / identity: h = act(fc1 x + b1), y = fc2 h + b2
+    (beta and the SwiGLU limit do not apply: there is no up value)."""
+    cfg = _cfg(T=6, d=24, F=40, E=1, k=1, ffn="plain", act=act, alpha=alpha, beta=0.75, limit=0.5,
+               expert_bias=True)
+    p, t = _problem(cfg)
+    ref = _plain_ffn(t["x"].double(), t["gate_up"][0].double(), t["down"][0].double(), act, _f32(alpha),
+                     t["gate_up_bias"][0].double(), t["down_bias"][0].double())
+    assert np.allclose(p.forward(), ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_plain_shared_expert(oracle_lib):
+    cfg = _cfg(T=6, d=16, F=8, E=4, k=2, Fs=12, ffn="plain", act="relu")
+    p, t = _problem(cfg)
+    base = _problem(small(cfg, Fs=0))[0].forward()
+    ffn = _plain_ffn(t["x"].double(), t["shared_gate_up"].double(), t["shared_down"].double(), "relu", 1.0)
+    assert np.allclose(p.forward() - base, ffn.numpy(), rtol=1e-10, atol=1e-13)
+
+
+def test_router_weight_worked_example(oracle_lib):
+    x = torch.tensor([[1.0, 2.0, 3.0], [-1.0, 0.0, 2.0]])
+    wr = torch.tensor([[1.0, 0.0], [0.0, 1.0], [1.0, -1.0]])
+    cfg = _cfg(T=2, d=3, F=8, E=2, k=1, router="weight")
+    p, _ = _problem(cfg, x=x, router_weight=wr)
+    for tok, l0, l1 in _rows("router_worked_example.txt"):
+        _, _, keys, _ = p.route(int(tok))
+        assert keys.tolist() == [float(l0), float(l1)]   # unbiased softmax ranks by the logit
+
+
+def test_router_weight_matches_numpy_matmul(oracle_lib):
+    """Logits from Wr [d, E] equal numpy's fp64 x @ Wr rounded once to fp32 (to one fp32
+    ulp: the two sums may round differently in the last double bit), and the routing
+    on them equals the routing on those logits passed in."""
+    cfg = _cfg(T=12, d=64, F=8, E=16, k=4, router="weight", act_dtype="bf16", w_dtype="bf16",
+               router_bias=True, logit_dtype="f32")
+    p, t = _problem(cfg)
+    x = t["x"].double().numpy()
+    wr = t["router_weight"].double().numpy()
+    ref = (x @ wr).astype(np.float32)
+    br = t["router_bias"].numpy()
+    cfg_l = small(cfg, router="logits")
+    pl, _ = _problem(cfg_l, logits=torch.from_numpy(ref), router_bias=t["router_bias"])
+    for tok in range(cfg.T):
+        _, _, keys, _ = p.route(tok)
+        want = (ref[tok] + br).astype(np.float64)
+        assert np.all(np.abs(keys - want) <= np.spacing(np.abs(want).astype(np.float32)).astype(np.float64))
+        if np.array_equal(keys, want):
+            assert np.array_equal(p.route(tok)[0], pl.route(tok)[0])

@@ -44,7 +44,9 @@ class MoeConfig:
     alpha: float = 1.0
     beta: float = 0.0
     limit: float = 0.0
-    gu_layout: str = "concat"       # concat (gate rows first) | interleaved (even rows gate)
+    gu_layout: str = "concat"       # concat (gate rows first) | interleaved (even rows gate) | unfused
+    ffn: str = "gated"              # gated: act(gate) * (up + beta) | plain: act(fc1) alone
+    router: str = "logits"          # logits: caller's router logits | weight: logits = x Wr in the layer
     shared_gate: bool = False
     router_bias: bool = False
     expert_bias: bool = False
@@ -145,33 +147,48 @@ def make_inputs(cfg: MoeConfig, device="cpu", with_weights: bool = True) -> dict
     gate_up_scales [E,2F,d/32]), gate_up_bias [E,2F], down [E,d,F] (or codes
     [E,d,F/2] with down_scales [E,d,F/32]), down_bias [E,d], shared_gate_up
     [2Fs,d], shared_down [d,Fs], shared_gate_vec [d], shared_output [T,d].
+    Unfused layout: gate [E,F,d] (+ gate_scales, gate_bias [E,F]) and gate_up holds
+    the up rows [E,F,d] (bias [E,F]).  Plain FFN: gate_up is fc1 [E,F,d] (bias
+    [E,F]) and the shared stack [Fs,d].  Router weight: router_weight [d,E] (act
+    dtype) and logits None.
     """
     T, d, F, E = cfg.T, cfg.d, cfg.F, cfg.E
     adt = _TORCH_DTYPE[cfg.act_dtype]
     ldt = _TORCH_DTYPE[cfg.logit_dtype]
     out = dict.fromkeys(["x", "logits", "router_bias", "selection_bias", "gate_up",
                          "gate_up_scales", "gate_up_bias", "down", "down_scales", "down_bias",
-                         "shared_gate_up", "shared_down", "shared_gate_vec", "shared_output"])
+                         "shared_gate_up", "shared_down", "shared_gate_vec", "shared_output",
+                         "gate", "gate_scales", "gate_bias", "router_weight"])
     out["x"] = _normal((T, d), 1.0, adt, _gen(cfg, 0, device), device)
-    logits = torch.randn((T, E), generator=_gen(cfg, 1, device), device=device)
-    if cfg.logits == "zipf":
-        g = _gen(cfg, 2, device)
-        rank = torch.randperm(E, generator=g, device=device).to(torch.float32) + 1.0
-        logits = logits - cfg.zipf_s * torch.log(rank)
-    out["logits"] = logits.to(ldt)
+    if cfg.router == "weight":
+        out["router_weight"] = _normal((d, E), 0.02, adt, _gen(cfg, 13, device), device)
+    else:
+        logits = torch.randn((T, E), generator=_gen(cfg, 1, device), device=device)
+        if cfg.logits == "zipf":
+            g = _gen(cfg, 2, device)
+            rank = torch.randperm(E, generator=g, device=device).to(torch.float32) + 1.0
+            logits = logits - cfg.zipf_s * torch.log(rank)
+        out["logits"] = logits.to(ldt)
     if cfg.router_bias:
         out["router_bias"] = _normal((E,), 0.02, ldt, _gen(cfg, 3, device), device)
     if cfg.selection_bias_std > 0:
         out["selection_bias"] = _normal((E,), cfg.selection_bias_std, torch.float32,
                                         _gen(cfg, 4, device), device)
+    separate = cfg.gu_layout == "unfused" or cfg.ffn == "plain"  # gate_up holds F rows per expert
+    fc1_rows = F if separate else 2 * F
     if with_weights:
-        out["gate_up"], out["gate_up_scales"] = _weights(cfg, 5, E, 2 * F, d, device)
+        out["gate_up"], out["gate_up_scales"] = _weights(cfg, 5, E, fc1_rows, d, device)
         out["down"], out["down_scales"] = _weights(cfg, 6, E, d, F, device)
+        if cfg.gu_layout == "unfused" and cfg.ffn == "gated":
+            out["gate"], out["gate_scales"] = _weights(cfg, 14, E, F, d, device)
     if cfg.expert_bias:
-        out["gate_up_bias"] = _normal((E, 2 * F), 0.02, adt, _gen(cfg, 7, device), device)
+        out["gate_up_bias"] = _normal((E, fc1_rows), 0.02, adt, _gen(cfg, 7, device), device)
         out["down_bias"] = _normal((E, d), 0.02, adt, _gen(cfg, 8, device), device)
+        if cfg.gu_layout == "unfused" and cfg.ffn == "gated":
+            out["gate_bias"] = _normal((E, F), 0.02, adt, _gen(cfg, 15, device), device)
     if cfg.Fs > 0 and with_weights:
-        out["shared_gate_up"] = _normal((2 * cfg.Fs, d), 0.02, adt, _gen(cfg, 9, device), device)
+        sh_rows = cfg.Fs if cfg.ffn == "plain" else 2 * cfg.Fs
+        out["shared_gate_up"] = _normal((sh_rows, d), 0.02, adt, _gen(cfg, 9, device), device)
         out["shared_down"] = _normal((d, cfg.Fs), 0.02, adt, _gen(cfg, 10, device), device)
     if cfg.shared_gate:
         out["shared_gate_vec"] = _normal((d,), 0.02, adt, _gen(cfg, 11, device), device)
@@ -180,30 +197,41 @@ def make_inputs(cfg: MoeConfig, device="cpu", with_weights: bool = True) -> dict
     return out
 
 
+def _mats(cfg: MoeConfig) -> int:
+    """Weight matrices per expert: gate, up and down (gated) or fc1 and down (plain)."""
+    return 2 if cfg.ffn == "plain" else 3
+
+
 def flops(cfg: MoeConfig) -> float:
-    """Algorithmic FLOPs of one forward: 2*R*3*d*F routed + 2*T*3*d*Fs shared."""
-    return 2.0 * cfg.T * cfg.k * 3 * cfg.d * cfg.F + 2.0 * cfg.T * 3 * cfg.d * cfg.Fs
+    """Algorithmic FLOPs of one forward: 2*R*m*d*F routed + 2*T*m*d*Fs shared (m = 3
+    matrices per gated expert, 2 per plain one), + 2*T*d*E for a router weight."""
+    m = _mats(cfg)
+    f = 2.0 * cfg.T * cfg.k * m * cfg.d * cfg.F + 2.0 * cfg.T * m * cfg.d * cfg.Fs
+    if cfg.router == "weight":
+        f += 2.0 * cfg.T * cfg.d * cfg.E
+    return f
 
 
 def weight_bytes_per_expert(cfg: MoeConfig) -> float:
-    n = 3 * cfg.d * cfg.F
+    n = _mats(cfg) * cfg.d * cfg.F
     if cfg.w_dtype == "mxfp4":
         b = n / 2 + n / 32
     else:
         b = n * (4 if cfg.w_dtype == "f32" else 2)
     if cfg.expert_bias:
-        b += (2 * cfg.F + cfg.d) * (4 if cfg.act_dtype == "f32" else 2)
+        b += ((_mats(cfg) - 1) * cfg.F + cfg.d) * (4 if cfg.act_dtype == "f32" else 2)
     return b
 
 
 def algorithmic_bytes(cfg: MoeConfig, distinct_experts: int) -> float:
     """Bytes a forward must move: touched experts' weights (+biases, scales), shared
-    weights, x, logits and y."""
+    weights, x, the router logits (or the router weight) and y."""
     ab = 4 if cfg.act_dtype == "f32" else 2
     lb = 4 if cfg.logit_dtype == "f32" else 2
     b = distinct_experts * weight_bytes_per_expert(cfg)
-    b += 3 * cfg.d * cfg.Fs * ab
-    b += cfg.T * cfg.d * ab * 2 + cfg.T * cfg.E * lb
+    b += _mats(cfg) * cfg.d * cfg.Fs * ab
+    b += cfg.T * cfg.d * ab * 2
+    b += cfg.d * cfg.E * ab if cfg.router == "weight" else cfg.T * cfg.E * lb
     if cfg.shared_output:
         b += cfg.T * cfg.d * ab
     return b
