@@ -76,8 +76,11 @@ enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };
 /* ---- gated activation ("Struct MoeSpec" act; graph-op activation_type) ---- */
 enum { MOE_ACT_SILU = 0, MOE_ACT_GELU_ERF = 1, MOE_ACT_GELU_TANH = 2, MOE_ACT_RELU = 3,
        MOE_ACT_IDENTITY = 4 };
-/* ---- fused gate||up layout (graph-op swiglu_fusion: 2 = concat, 1 = interleaved) ---- */
-enum { MOE_GU_CONCAT = 0, MOE_GU_INTERLEAVED = 1 };
+/* ---- gate/up layout (graph-op swiglu_fusion: 2 = fused concat, 1 = fused interleaved,
+ *      0 = not fused: the gate rows in their own stack, "MoE" set_weights gate_experts) ---- */
+enum { MOE_GU_CONCAT = 0, MOE_GU_INTERLEAVED = 1, MOE_GU_UNFUSED = 2 };
+/* ---- expert FFN form (graph-op fc1 fusion_size: 2 = gated, 1 = plain) ---- */
+enum { MOE_FFN_GATED = 0, MOE_FFN_PLAIN = 1 };
 
 /*
  * Problem sizes.  T tokens (a 3-D x [B, S, d] is passed as T = B*S), d hidden,
@@ -108,6 +111,10 @@ typedef struct {
   float limit;         /* SiLU clamp; 0 = none                           default 0       */
   int32_t gu_layout;   /* MOE_GU_*                                       default CONCAT  */
   int32_t shared_gate; /* 0/1: shared expert output times sigmoid(x . g) default 0       */
+  int32_t ffn;         /* MOE_FFN_GATED: h = act(g) * (u + beta);        default GATED   */
+                       /* MOE_FFN_PLAIN: h = act(fc1 x + b1), one matrix (graph-op       */
+                       /* activation_type relu/gelu/silu/identity with fusion_size 1;    */
+                       /* alpha for SiLU, no beta, no limit)                             */
 } moe_options;
 
 /*
@@ -130,6 +137,18 @@ typedef struct {
  *   y               [T, d] act_dtype, output (must not alias any input)
  *   topk_idx        [T, k] int32, optional output: chosen experts, best first
  *   topk_w          [T, k] fp32, optional output: their weights
+ *   gate            MOE_GU_UNFUSED only: the gate rows [E, F, d] w_dtype (MXFP4: codes
+ *                   [E, F, d/2] with gate_scales [E, F, d/32]); gate_up then holds the
+ *                   up rows [E, F, d] and gate_up_bias their bias [E, F]
+ *   gate_bias       [E, F] act_dtype, optional (MOE_GU_UNFUSED)
+ *   router_weight   [d, E] act_dtype ("Struct MoeSpec" wr, wr[(i-1)E + e]): with
+ *                   router_logits NULL the layer computes the logits x Wr itself
+ *                   (fp32 accumulation) and routes on them without storing them
+ *   logits_out      [T, E] fp32, optional output (router_weight only): the logits
+ *                   the layer computed, before router_bias
+ * With MOE_FFN_PLAIN, gate_up is fc1 [E, F, d] (bias [E, F]) and shared_gate_up
+ * [Fs, d].  The shared expert of an unfused layer keeps one stack [2Fs, d], gate
+ * rows first.
  */
 typedef struct {
   const void *x, *router_logits, *router_bias;
@@ -144,6 +163,11 @@ typedef struct {
   void *y;
   int32_t *topk_idx;
   float *topk_w;
+  const void *gate;
+  const uint8_t *gate_scales;
+  const void *gate_bias;
+  const void *router_weight;
+  float *logits_out;
 } moe_tensors;
 
 /* Fill `opts` with the defaults listed in moe_options (the graph-op page's
@@ -184,8 +208,8 @@ MOE_API int moe_forward(const moe_shape *shape, const moe_options *opts, const m
 /*
  * Routing only ("Struct MoeSpec" score, selection_bias, groups, renormalize,
  * scale): writes t->topk_idx [T, k] and t->topk_w [T, k] (both required here).
- * Only x (when shared_gate), router_logits, router_bias and selection_bias
- * are read.  Same workspace rules as moe_forward.
+ * Only x (when shared_gate or router_weight), router_logits or router_weight,
+ * router_bias and selection_bias are read.  Same workspace rules as moe_forward.
  */
 MOE_API int moe_route(const moe_shape *shape, const moe_options *opts, const moe_tensors *t,
               void *workspace, size_t workspace_bytes, void *stream);

@@ -24,7 +24,8 @@ MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_A
 MOE_F32, MOE_BF16, MOE_MXFP4 = 0, 1, 2
 MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
 MOE_ACT_SILU, MOE_ACT_GELU_ERF, MOE_ACT_GELU_TANH, MOE_ACT_RELU, MOE_ACT_IDENTITY = 0, 1, 2, 3, 4
-MOE_GU_CONCAT, MOE_GU_INTERLEAVED = 0, 1
+MOE_GU_CONCAT, MOE_GU_INTERLEAVED, MOE_GU_UNFUSED = 0, 1, 2
+MOE_FFN_GATED, MOE_FFN_PLAIN = 0, 1
 
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_NULL", 2: "MOE_ERR_SHAPE", 3: "MOE_ERR_DTYPE",
                 4: "MOE_ERR_ALIGN", 5: "MOE_ERR_UNSUPPORTED", 6: "MOE_ERR_WORKSPACE",
@@ -33,7 +34,8 @@ DTYPE_CODES = {"f32": MOE_F32, "bf16": MOE_BF16, "mxfp4": MOE_MXFP4}
 SCORE_CODES = {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID}
 ACT_CODES = {"silu": MOE_ACT_SILU, "gelu_erf": MOE_ACT_GELU_ERF, "gelu_tanh": MOE_ACT_GELU_TANH,
              "relu": MOE_ACT_RELU, "identity": MOE_ACT_IDENTITY}
-LAYOUT_CODES = {"concat": MOE_GU_CONCAT, "interleaved": MOE_GU_INTERLEAVED}
+LAYOUT_CODES = {"concat": MOE_GU_CONCAT, "interleaved": MOE_GU_INTERLEAVED, "unfused": MOE_GU_UNFUSED}
+FFN_CODES = {"gated": MOE_FFN_GATED, "plain": MOE_FFN_PLAIN}
 
 
 class moe_shape(C.Structure):
@@ -46,14 +48,16 @@ class moe_options(C.Structure):
     _fields_ = [("score", C.c_int32), ("renormalize", C.c_int32), ("routed_scale", C.c_float),
                 ("n_group", C.c_int32), ("topk_group", C.c_int32), ("weigh_inputs", C.c_int32),
                 ("act", C.c_int32), ("alpha", C.c_float), ("beta", C.c_float),
-                ("limit", C.c_float), ("gu_layout", C.c_int32), ("shared_gate", C.c_int32)]
+                ("limit", C.c_float), ("gu_layout", C.c_int32), ("shared_gate", C.c_int32),
+                ("ffn", C.c_int32)]
 
 
 class moe_tensors(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in (
         "x", "router_logits", "router_bias", "selection_bias", "gate_up", "gate_up_scales",
         "gate_up_bias", "down", "down_scales", "down_bias", "shared_gate_up", "shared_down",
-        "shared_gate_vec", "shared_output", "y", "topk_idx", "topk_w")]
+        "shared_gate_vec", "shared_output", "y", "topk_idx", "topk_w", "gate", "gate_scales",
+        "gate_bias", "router_weight", "logits_out")]
 
 
 _P = C.POINTER
@@ -188,7 +192,7 @@ def make_shape(T, d, F, E, k, Fs=0, act_dtype="bf16", w_dtype="bf16", logit_dtyp
 
 def make_options(score="softmax", renormalize=False, routed_scale=1.0, n_group=0, topk_group=0,
                  weigh_inputs=False, act="silu", alpha=1.0, beta=0.0, limit=0.0,
-                 gu_layout="concat", shared_gate=False) -> moe_options:
+                 gu_layout="concat", shared_gate=False, ffn="gated") -> moe_options:
     o = moe_options_init()
     o.score = SCORE_CODES[score]
     o.renormalize = int(renormalize)
@@ -199,6 +203,7 @@ def make_options(score="softmax", renormalize=False, routed_scale=1.0, n_group=0
     o.alpha, o.beta, o.limit = alpha, beta, limit
     o.gu_layout = LAYOUT_CODES[gu_layout]
     o.shared_gate = int(shared_gate)
+    o.ffn = FFN_CODES[ffn]
     return o
 
 
@@ -211,22 +216,24 @@ def shape_of(cfg) -> moe_shape:
 def options_of(cfg) -> moe_options:
     return make_options(cfg.score, cfg.renormalize, cfg.routed_scale, cfg.n_group,
                         cfg.topk_group, cfg.weigh_inputs, cfg.act, cfg.alpha, cfg.beta,
-                        cfg.limit, cfg.gu_layout, cfg.shared_gate)
+                        cfg.limit, cfg.gu_layout, cfg.shared_gate, getattr(cfg, "ffn", "gated"))
 
 
 def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
-def tensors_of(inputs: dict, y=None, topk_idx=None, topk_w=None) -> moe_tensors:
+def tensors_of(inputs: dict, y=None, topk_idx=None, topk_w=None, logits_out=None) -> moe_tensors:
     """moe_tensors from a dict of device tensors (keys as in moe.h)."""
     t = moe_tensors()
     for name in ("x", "router_bias", "selection_bias", "gate_up", "gate_up_scales",
                  "gate_up_bias", "down", "down_scales", "down_bias", "shared_gate_up",
-                 "shared_down", "shared_gate_vec", "shared_output"):
+                 "shared_down", "shared_gate_vec", "shared_output", "gate", "gate_scales",
+                 "gate_bias", "router_weight"):
         setattr(t, name, _ptr(inputs.get(name)))
     t.router_logits = _ptr(inputs.get("logits", inputs.get("router_logits")))
     t.y, t.topk_idx, t.topk_w = _ptr(y), _ptr(topk_idx), _ptr(topk_w)
+    t.logits_out = _ptr(logits_out)
     return t
 
 
@@ -249,7 +256,7 @@ class Workspace:
 
 
 def forward(cfg, inputs: dict, y=None, workspace: Workspace | None = None, stream=None,
-            topk_idx=None, topk_w=None):
+            topk_idx=None, topk_w=None, logits_out=None):
     """Run moe_forward on device tensors; returns y [T, d] (allocated by torch if None)."""
     import torch
     x = inputs["x"]
@@ -259,7 +266,7 @@ def forward(cfg, inputs: dict, y=None, workspace: Workspace | None = None, strea
     if workspace is None:
         workspace = Workspace(moe_workspace_size(shape, opts), x.device)
     st = (stream if stream is not None else torch.cuda.current_stream(x.device)).cuda_stream
-    tens = tensors_of(inputs, y, topk_idx, topk_w)
+    tens = tensors_of(inputs, y, topk_idx, topk_w, logits_out)
     _check(moe_forward(shape, opts, tens, workspace.ptr, workspace.nbytes, st))
     return y
 
@@ -267,7 +274,7 @@ def forward(cfg, inputs: dict, y=None, workspace: Workspace | None = None, strea
 def route(cfg, inputs: dict, workspace: Workspace | None = None, stream=None):
     """Run moe_route; returns (topk_idx [T, k] int32, topk_w [T, k] fp32)."""
     import torch
-    logits = inputs["logits"]
+    logits = inputs["logits"] if inputs.get("logits") is not None else inputs["x"]
     shape, opts = shape_of(cfg), options_of(cfg)
     idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=logits.device)
     w = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=logits.device)

@@ -62,16 +62,17 @@ int check_shape_opts(const moe_shape* s, const moe_options* o) {
     return fail(MOE_ERR_SHAPE, "d, F and Fs must be multiples of 8 (16-byte rows)");
   if (s->w_dtype == MOE_MXFP4 && (s->d % 32 || s->F % 32))
     return fail(MOE_ERR_SHAPE, "MXFP4 experts need d and F multiples of 32 (block size)");
-  if (s->w_dtype == MOE_MXFP4 && s->Fs > 0)
-    return fail(MOE_ERR_UNSUPPORTED, "a shared expert next to MXFP4 routed experts is not built");
   const int64_t rows = s->T * s->k + (s->Fs > 0 ? s->T : 0);
   if (s->T > (1ll << 26) || rows >= (1ll << 31))
     return fail(MOE_ERR_SHAPE, "T*k + T must stay below 2^31 rows (T=%lld)", (long long)s->T);
 
   if (o->score != MOE_SCORE_SOFTMAX && o->score != MOE_SCORE_SIGMOID) return fail(MOE_ERR_ARG, "score %d", o->score);
   if (o->act < MOE_ACT_SILU || o->act > MOE_ACT_IDENTITY) return fail(MOE_ERR_ARG, "act %d", o->act);
-  if (o->gu_layout != MOE_GU_CONCAT && o->gu_layout != MOE_GU_INTERLEAVED)
+  if (o->gu_layout != MOE_GU_CONCAT && o->gu_layout != MOE_GU_INTERLEAVED && o->gu_layout != MOE_GU_UNFUSED)
     return fail(MOE_ERR_ARG, "gu_layout %d", o->gu_layout);
+  if (o->ffn != MOE_FFN_GATED && o->ffn != MOE_FFN_PLAIN) return fail(MOE_ERR_ARG, "ffn %d", o->ffn);
+  if (o->ffn == MOE_FFN_PLAIN && o->gu_layout == MOE_GU_UNFUSED)
+    return fail(MOE_ERR_ARG, "an unfused gate stack needs a gated FFN (ffn = MOE_FFN_GATED)");
   if ((o->renormalize & ~1) || (o->weigh_inputs & ~1) || (o->shared_gate & ~1))
     return fail(MOE_ERR_ARG, "renormalize, weigh_inputs and shared_gate are 0 or 1");
   if (!std::isfinite(o->routed_scale) || !std::isfinite(o->alpha) || !std::isfinite(o->beta) ||
@@ -93,7 +94,12 @@ int check_shape_opts(const moe_shape* s, const moe_options* o) {
 int check_tensors(const moe_shape* s, const moe_options* o, const moe_tensors* t, bool full) {
   if (!t) return fail(MOE_ERR_NULL, "tensors must not be NULL");
   if (s->T == 0) return MOE_OK;  // nothing is read or written (empty tensors may have NULL data)
-  if (!t->router_logits) return fail(MOE_ERR_NULL, "router_logits is required");
+  if (!t->router_logits && !t->router_weight)
+    return fail(MOE_ERR_NULL, "router_logits or router_weight is required");
+  if (t->router_logits && t->router_weight)
+    return fail(MOE_ERR_ARG, "give router_logits or router_weight, not both");
+  if (t->router_weight && !t->x) return fail(MOE_ERR_NULL, "router_weight needs x");
+  if (t->logits_out && !t->router_weight) return fail(MOE_ERR_ARG, "logits_out needs router_weight");
   if (o->shared_gate && !t->shared_gate_vec) return fail(MOE_ERR_NULL, "shared_gate needs shared_gate_vec");
   if (o->shared_gate && !t->x) return fail(MOE_ERR_NULL, "shared_gate needs x");
   if (!full) {
@@ -103,9 +109,15 @@ int check_tensors(const moe_shape* s, const moe_options* o, const moe_tensors* t
   if (!t->x || !t->gate_up || !t->down || !t->y) return fail(MOE_ERR_NULL, "x, gate_up, down and y are required");
   if (s->w_dtype == MOE_MXFP4 && (!t->gate_up_scales || !t->down_scales))
     return fail(MOE_ERR_NULL, "MXFP4 experts need gate_up_scales and down_scales");
+  if (o->gu_layout == MOE_GU_UNFUSED && !t->gate) return fail(MOE_ERR_NULL, "the unfused layout needs gate");
+  if (o->gu_layout == MOE_GU_UNFUSED && s->w_dtype == MOE_MXFP4 && !t->gate_scales)
+    return fail(MOE_ERR_NULL, "unfused MXFP4 experts need gate_scales");
+  if (o->gu_layout != MOE_GU_UNFUSED && (t->gate || t->gate_bias))
+    return fail(MOE_ERR_ARG, "gate and gate_bias belong to the unfused layout");
   if (s->Fs > 0 && (!t->shared_gate_up || !t->shared_down))
     return fail(MOE_ERR_NULL, "Fs > 0 needs shared_gate_up and shared_down");
-  const void* tma[] = {t->x, t->gate_up, t->down, t->y, t->shared_output, t->shared_gate_up, t->shared_down};
+  const void* tma[] = {t->x, t->gate_up, t->down, t->y, t->shared_output, t->shared_gate_up, t->shared_down,
+                       t->gate};
   for (const void* p : tma)
     if (p && !aligned16(p)) return fail(MOE_ERR_ALIGN, "x, weights, y and shared_output must be 16-byte aligned");
   if (t->y == t->x || (t->shared_output && t->y == t->shared_output))
@@ -186,7 +198,10 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
   ra.d = (int)p.d;
   ra.act_bf16 = s->act_dtype == MOE_BF16;
   ra.sgate = (full && o->shared_gate) ? at<float>(ws, p.o_sgate) : nullptr;
-  if ((e = launch_route(ra, st)) != cudaSuccess) return cuda_fail(e, "route kernel");
+  ra.router_weight = t->router_weight;
+  ra.logits_out = t->logits_out;
+  if ((e = t->router_weight ? launch_router(ra, st) : launch_route(ra, st)) != cudaSuccess)
+    return cuda_fail(e, "route kernel");
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   if (!full) return MOE_OK;
 
@@ -217,9 +232,13 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
   if ((e = launch_sort(sa, st)) != cudaSuccess) return cuda_fail(e, "sort kernels");
   if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
 
-  GatherArgs ga{t->x, sa.perm, sa.roww, at<void>(ws, p.o_x), (int)p.R, (int)p.d, (int)p.T,
-                s->act_dtype == MOE_BF16, o->weigh_inputs, status};
-  if ((e = launch_gather(ga, st)) != cudaSuccess) return cuda_fail(e, "gather kernel");
+  // The rows in expert order: gathered from x, except for small batches on the
+  // single-CTA bf16 GEMMs, whose gate_up reads x in place (direct_x).
+  if (!p.direct_x) {
+    GatherArgs ga{t->x, sa.pos, sa.roww, at<void>(ws, p.o_x), (int)p.R, (int)p.d, (int)p.T, (int)p.k,
+                  s->act_dtype == MOE_BF16, o->weigh_inputs, status};
+    if ((e = launch_gather(ga, st)) != cudaSuccess) return cuda_fail(e, "gather kernel");
+  }
   if ((e = mark(3)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
 
   GemmCommon gc{};
@@ -234,6 +253,11 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
   gc.Fs = (int)p.Fs;
   gc.Fmax = (int)p.Fmax;
   gc.gu_layout = o->gu_layout;
+  gc.ffn = o->ffn;
+  gc.direct_x = p.direct_x;
+  gc.k = (int)p.k;
+  gc.topk_idx = ra.idx;
+  gc.pos = sa.pos;
   gc.act = ActParams{o->act, o->alpha, o->beta, o->limit};
   gc.weigh_inputs = o->weigh_inputs;
   gc.status = status;
@@ -257,6 +281,9 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
     ta.xg = at<void>(ws, p.o_x);
     ta.gate_up = t->gate_up;
     ta.gate_up_bias = t->gate_up_bias;
+    ta.gate = t->gate;
+    ta.gate_bias = t->gate_bias;
+    ta.gate_scales = t->gate_scales;
     ta.down = t->down;
     ta.down_bias = t->down_bias;
     ta.sh_gate_up = t->shared_gate_up;
@@ -268,15 +295,42 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
     ta.gate_up_scales = t->gate_up_scales;
     ta.down_scales = t->down_scales;
     const bool fp4 = s->w_dtype == MOE_MXFP4;
-    ta.c = gu;
-    e = fp4 ? launch_fp4_gate_up(ta, st) : p.pair ? launch_tc2_gate_up(ta, st) : launch_tc_gate_up(ta, st);
+    // With MXFP4 experts the shared expert (bf16 weights) is a second launch: the
+    // CTA-pair bf16 kernel over the shared segment alone (its tiles are 256 rows,
+    // the MXFP4 tile height, so one tile list serves both).
+    GemmCommon gu_routed = gu, gu_shared = gu;
+    if (fp4 && p.Fs > 0) {
+      gu_routed.NS = (int)p.E;
+      gu_routed.max_tiles = (int)(mt_routed * p.nt_gu_routed);
+      gu_shared.seg_begin = (int)p.E;
+      gu_shared.max_tiles = (int)(mt_shared * p.nt_gu_shared);
+    }
+    ta.c = fp4 ? gu_routed : gu;
+    e = fp4 ? (p.pair_fp4 ? launch_fp4p_gate_up(ta, st) : launch_fp4_gate_up(ta, st))
+            : p.swap ? launch_tcs_gate_up(ta, st) : p.pair ? launch_tc2_gate_up(ta, st) : launch_tc_gate_up(ta, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core gate_up GEMM");
+    if (fp4 && p.Fs > 0) {
+      ta.c = gu_shared;
+      if ((e = launch_tc2_gate_up(ta, st)) != cudaSuccess) return cuda_fail(e, "shared expert gate_up GEMM");
+    }
     if (gu.splits > 1 && (e = launch_splitk_gate_up_reduce(ta, st)) != cudaSuccess)
       return cuda_fail(e, "split-K gate_up reduction");
     if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    ta.c = dn;
-    e = fp4 ? launch_fp4_down(ta, st) : p.pair ? launch_tc2_down(ta, st) : launch_tc_down(ta, st);
+    GemmCommon dn_routed = dn, dn_shared = dn;
+    if (fp4 && p.Fs > 0) {
+      dn_routed.NS = (int)p.E;
+      dn_routed.max_tiles = (int)(mt_routed * p.nt_dn_routed);
+      dn_shared.seg_begin = (int)p.E;
+      dn_shared.max_tiles = (int)(mt_shared * p.nt_dn_shared);
+    }
+    ta.c = fp4 ? dn_routed : dn;
+    e = fp4 ? (p.pair_fp4 ? launch_fp4p_down(ta, st) : launch_fp4_down(ta, st))
+            : p.swap ? launch_tcs_down(ta, st) : p.pair ? launch_tc2_down(ta, st) : launch_tc_down(ta, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core down GEMM");
+    if (fp4 && p.Fs > 0) {
+      ta.c = dn_shared;
+      if ((e = launch_tc2_down(ta, st)) != cudaSuccess) return cuda_fail(e, "shared expert down GEMM");
+    }
     if (dn.splits > 1 && (e = launch_splitk_down_reduce(ta, st)) != cudaSuccess)
       return cuda_fail(e, "split-K down reduction");
   } else {
@@ -285,6 +339,8 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
     sm.xg = at<float>(ws, p.o_x);
     sm.gate_up = (const float*)t->gate_up;
     sm.gate_up_bias = (const float*)t->gate_up_bias;
+    sm.gate = (const float*)t->gate;
+    sm.gate_bias = (const float*)t->gate_bias;
     sm.down = (const float*)t->down;
     sm.down_bias = (const float*)t->down_bias;
     sm.sh_gate_up = (const float*)t->shared_gate_up;
@@ -327,6 +383,28 @@ bool pdl_enabled() {
   return on;
 }
 
+// MXFP4 GEMMs on CTA pairs when every expert holds on average a tile's worth of rows
+// (128); MOE_B200_PAIR_FP4=0 or 1 overrides the choice.
+bool use_pair_fp4(int64_t R, int64_t E) {
+  const char* env = std::getenv("MOE_B200_PAIR_FP4");
+  if (env && env[0] == '0') return false;
+  if (env && env[0] == '1') return true;
+  return R >= (int64_t)kFp4PairMinRows * E;
+}
+
+// bf16 GEMMs with swapped operands on CTA pairs for large batches that the
+// CTA-pair kernel with token tiles of 256 rows does not take (fewer than 512 rows
+// per expert on average: token tiles would be mostly padding); not for the unfused
+// layout.  MOE_B200_SWAP_GEMM=0 or 1 overrides the choice (1 still needs a batch
+// without split-K and a fused or plain layout).
+bool use_swap_gemm(int64_t R, bool pair, int layout) {
+  if (layout == MOE_GU_UNFUSED || R <= kSplitMaxRows) return false;
+  const char* env = std::getenv("MOE_B200_SWAP_GEMM");
+  if (env && env[0] == '0') return false;
+  if (env && env[0] == '1') return true;
+  return !pair;
+}
+
 bool use_pair_gemm(int64_t R, int64_t E) {
   const char* env = std::getenv("MOE_B200_PAIR_GEMM");
   if (env && env[0] == '0') return false;
@@ -335,7 +413,6 @@ bool use_pair_gemm(int64_t R, int64_t E) {
 }
 
 size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
-  (void)o;
   p->T = s->T;
   p->d = s->d;
   p->F = s->F;
@@ -352,20 +429,36 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   p->logit_dtype = s->logit_dtype;
   p->tc = s->act_dtype == MOE_BF16;
   p->pair = p->tc && s->w_dtype == MOE_BF16 && use_pair_gemm(p->R, s->E);
+  p->direct_x = p->tc && s->w_dtype == MOE_BF16 && !p->pair && s->T <= kDirectMaxTokens;
+  p->pair_fp4 = s->w_dtype == MOE_MXFP4 && use_pair_fp4(p->R, s->E);
+  p->swap = p->tc && s->w_dtype == MOE_BF16 && use_swap_gemm(p->R, p->pair, o->gu_layout);
+  if (p->swap) p->pair = false;
+  // h features per gate_up tile: a gated tile holds each feature's gate and up
+  // rows, a plain one a single row per feature (twice the features)
+  const int plain = o->ffn == MOE_FFN_PLAIN ? 2 : 1;
   if (s->w_dtype == MOE_MXFP4) {
     p->bm = kFp4BM;
-    p->nt_gu_routed = (int)cdiv(s->F, kFp4GuBN);
-    p->nt_dn_routed = (int)cdiv(s->d, kFp4DnBN);
-    p->nt_gu_shared = p->nt_dn_shared = 0;
+    const int wide = p->pair_fp4 ? 2 : 1;  // a pair tile covers twice the weight rows
+    p->nt_gu_routed = (int)cdiv(s->F, kFp4GuBN * plain * wide);
+    p->nt_dn_routed = (int)cdiv(s->d, kFp4DnBN * wide);
+    // the shared expert (bf16) runs on the CTA-pair bf16 kernel: 256-row tiles of
+    // 128 gated (256 plain) features, or of 256 outputs
+    p->nt_gu_shared = (int)cdiv(s->Fs, kTcGuBN * plain);
+    p->nt_dn_shared = (int)cdiv(s->d, kTcDnBN);
+  } else if (p->swap) {  // pair tiles of 256 weight rows: 128 gated features or 256 plain ones
+    p->bm = kSwapBM;
+    p->nt_gu_routed = (int)cdiv(s->F, kTcGuBN * plain);
+    p->nt_gu_shared = (int)cdiv(s->Fs, kTcGuBN * plain);
+    p->nt_dn_routed = p->nt_dn_shared = (int)cdiv(s->d, kTcDnBN);
   } else if (p->tc) {
     p->bm = p->pair ? kPairBM : kTcBM;
-    p->nt_gu_routed = (int)cdiv(s->F, kTcGuBN);
-    p->nt_gu_shared = (int)cdiv(s->Fs, kTcGuBN);
+    p->nt_gu_routed = (int)cdiv(s->F, kTcGuBN * plain);
+    p->nt_gu_shared = (int)cdiv(s->Fs, kTcGuBN * plain);
     p->nt_dn_routed = p->nt_dn_shared = (int)cdiv(s->d, kTcDnBN);
   } else {
     p->bm = kSimtBM;
-    p->nt_gu_routed = (int)cdiv(s->F, 32);
-    p->nt_gu_shared = (int)cdiv(s->Fs, 32);
+    p->nt_gu_routed = (int)cdiv(s->F, 32 * plain);
+    p->nt_gu_shared = (int)cdiv(s->Fs, 32 * plain);
     p->nt_dn_routed = p->nt_dn_shared = (int)cdiv(s->d, 64);
   }
   // split-K for the bf16 tensor-core GEMMs when even the largest possible tile
@@ -401,7 +494,7 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   p->o_perm = take(p->R * 4);
   p->o_roww = take(p->R * 4);
   p->o_sgate = take(p->T * 4);
-  p->o_x = take(p->R * p->d * elt);
+  p->o_x = take(p->direct_x ? 0 : p->R * p->d * elt);  // rows in expert order (none for direct_x)
   p->o_h = take(p->rows * p->Fmax * elt);
   p->o_y = take(p->rows * p->d * elt);
   p->o_part = take((size_t)std::max(p->splits_gu, p->splits_dn) * p->rows * p->partial_pitch * 4 *
@@ -452,8 +545,10 @@ int moe_forward_kernel_count(const moe_shape* s, const moe_options* o) {
   if (s->T == 0) return 0;
   moe::Plan p;
   moe::make_plan(s, o, &p);
-  // route, histogram, scan, scatter, gather, gate_up, down, combine (+ split-K reductions)
-  return (p.nchunks == 1 ? 6 : 8) + (p.splits_gu > 1) + (p.splits_dn > 1);
+  // route, histogram, scan, scatter, gather (not for direct_x), gate_up, down, combine
+  // (+ split-K reductions); a single 64-token chunk sorts in one kernel
+  return (p.nchunks == 1 ? 4 : 6) + (p.direct_x ? 0 : 1) + 1 + (p.splits_gu > 1) + (p.splits_dn > 1) +
+         (s->w_dtype == MOE_MXFP4 && p.Fs > 0 ? 2 : 0);  // the shared expert beside MXFP4 experts
 }
 
 const char* moe_last_error(void) { return moe::g_err.c_str(); }

@@ -23,6 +23,7 @@ constexpr int kTcGuBN = 128;      // h features per gate_up tile (gate rows + up
 constexpr int kTcDnBN = 256;      // output features per down tile
 constexpr int kTcBK = 64;         // K elements per pipeline stage of the bf16 tensor-core GEMMs
 constexpr int kSplitMaxRows = 4096;  // split-K only for problems with at most this many routed rows
+constexpr int kDirectMaxTokens = 64; // batches whose gate_up reads x in place (one 64-row A tile)
 
 // ---------------------------------------------------------------- workspace plan
 // Segments: experts 0..E-1 (routed rows, sorted by expert, token-ascending
@@ -40,6 +41,9 @@ struct Plan {
   int act_dtype, w_dtype, logit_dtype;
   bool tc;            // tensor-core path (bf16 activations) vs SIMT fp32 path
   bool pair;          // bf16 GEMMs on CTA pairs (256 x 256 tiles over two SMs)
+  bool direct_x;      // gate_up reads x in place (small batches, single-CTA bf16 GEMMs)
+  bool pair_fp4;      // MXFP4 GEMMs on CTA pairs (256 weight rows over two SMs)
+  bool swap;          // bf16 GEMMs on CTA pairs with the weights as M (256 weight rows x <= 256 tokens)
   int bm;             // GEMM tile rows
   int nt_gu_routed, nt_gu_shared, nt_dn_routed, nt_dn_shared;  // N tiles per segment
   int splits_gu, splits_dn;  // split-K factors of the two GEMMs (1 = none)
@@ -102,6 +106,36 @@ __device__ __forceinline__ float gated_act(const ActParams& a, float g, float u)
   return v * (u + a.beta);
 }
 
+// Activation of a non-gated expert ("MoE" graph-op activation_type with fusion_size 1):
+// the gated forms without an up value; alpha for SiLU, no limit, no beta.
+__device__ __forceinline__ float plain_act(const ActParams& a, float g) {
+  switch (a.act) {
+    case MOE_ACT_SILU: return g / (1.f + __expf(-a.alpha * g));
+    case MOE_ACT_GELU_ERF: return 0.5f * g * (1.f + erff(g * 0.70710678118654752f));
+    case MOE_ACT_GELU_TANH: {
+      const float c = 0.79788456080286536f;  // sqrt(2/pi)
+      return 0.5f * g * (1.f + tanhf(c * (g + 0.044715f * g * g * g)));
+    }
+    case MOE_ACT_RELU: return fmaxf(g, 0.f);
+    default: return g;
+  }
+}
+
+// Where the gate and up values of feature f of a gated expert come from: weight /
+// bias rows gate_base + stride * f and up_base + stride * f of the expert's stacks.
+//   concat:      one stack [2F]: gate rows 0..F-1, up rows F..2F-1 (stride 1)
+//   interleaved: one stack [2F]: gate rows 2f, up rows 2f + 1 (stride 2)
+//   unfused:     gate stack [F] and up stack [F] (stride 1)
+struct GuRows {
+  int64_t gate0, up0;  // row of feature 0 (in its own stack for unfused)
+  int stride;
+};
+__host__ __device__ __forceinline__ GuRows gu_rows(int layout, int64_t F) {
+  if (layout == MOE_GU_INTERLEAVED) return GuRows{0, 1, 2};
+  if (layout == MOE_GU_UNFUSED) return GuRows{0, 0, 1};
+  return GuRows{0, F, 1};
+}
+
 // ---------------------------------------------------------------- launchers
 struct RouteArgs {
   const void* logits;
@@ -120,8 +154,13 @@ struct RouteArgs {
   const void* gvec;
   int d, act_bf16;
   float* sgate;     // [T] or null
+  // router weight Wr [d, E] (act dtype): with logits null the logits are x Wr,
+  // accumulated in double in index order and rounded once to fp32
+  const void* router_weight;
+  float* logits_out;  // [T, E] or null
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
+cudaError_t launch_router(const RouteArgs& a, cudaStream_t st);  // logits x Wr, then the routing
 
 struct SortArgs {
   const int32_t* idx;   // [T, k]
@@ -144,10 +183,10 @@ cudaError_t launch_sort(const SortArgs& a, cudaStream_t st);
 
 struct GatherArgs {
   const void* x;        // [T, d]
-  const int32_t* perm;  // [R]
+  const int32_t* pos;   // [T, k] token slot -> row
   const float* roww;    // [R]
   void* xg;             // [R, d]
-  int R, d, T, bf16, weigh_inputs;
+  int R, d, T, k, bf16, weigh_inputs;
   int* status;
 };
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t st);
@@ -169,11 +208,22 @@ struct GemmCommon {
   const int32_t* cnt;       // [NS]
   const int32_t* off;       // [NS + 1]
   const int32_t* tiles;     // [NS + 1] tile prefix for this GEMM
-  int max_tiles;            // host upper bound of tiles[NS]
+  int max_tiles;            // host upper bound of tiles[NS] - tiles[seg_begin]
+  int seg_begin;            // CTA-pair bf16 kernel: walk segments seg_begin .. NS-1 only (else 0)
   int d, F, Fs, Fmax;
-  int gu_layout;
+  int gu_layout;             // MOE_GU_* of the routed experts (the shared expert: concat if unfused)
+  int ffn;                   // MOE_FFN_GATED or MOE_FFN_PLAIN
   ActParams act;
   int weigh_inputs;
+  // Small batches (the single-CTA bf16 gate_up with T <= 64): the activation tile of
+  // every routed segment is x itself, rows 0 .. T-1, and accumulator row i belongs to
+  // token i; its output row is pos[i][j] for the slot j with topk_idx[i][j] == e (if
+  // any).  No copy of the rows in expert order is made.  Weigh-inputs then scales the
+  // accumulators (W (w x) = w (W x)) before the bias and the activation.
+  int direct_x;
+  int k;
+  const int32_t* topk_idx;  // [T, k]
+  const int32_t* pos;       // [T, k]
   int* status;
   // split-K: each tile's K range is cut into `splits` parts whose fp32 partial
   // accumulators go to partial[split][row][n_blk * 256 + col] (pitch floats per
@@ -187,8 +237,10 @@ struct SimtArgs {
   GemmCommon c;
   const float* x;           // [T, d] (shared rows read x directly)
   const float* xg;          // [R, d]
-  const float* gate_up;     // [E, 2F, d]
-  const float* gate_up_bias;// [E, 2F] or null
+  const float* gate_up;     // [E, 2F, d]; unfused: up rows [E, F, d]; plain: fc1 [E, F, d]
+  const float* gate_up_bias;// [E, 2F] ([E, F] unfused / plain) or null
+  const float* gate;        // unfused: gate rows [E, F, d]
+  const float* gate_bias;   // unfused: [E, F] or null
   const float* down;        // [E, d, F]
   const float* down_bias;   // [E, d] or null
   const float* sh_gate_up;  // [2Fs, d]
@@ -204,8 +256,11 @@ struct TcArgs {
   GemmCommon c;
   const void* x;            // [T, d] bf16
   const void* xg;           // [R, d] bf16
-  const void* gate_up;      // [E, 2F, d] bf16
-  const void* gate_up_bias; // [E, 2F] bf16 or null
+  const void* gate_up;      // [E, 2F, d] bf16; unfused: up rows [E, F, d]; plain: fc1 [E, F, d]
+  const void* gate_up_bias; // [E, 2F] ([E, F] unfused / plain) bf16 or null
+  const void* gate;         // unfused: gate rows [E, F, d] (MXFP4: codes [E, F, d/2])
+  const void* gate_bias;    // unfused: [E, F] bf16 or null
+  const uint8_t* gate_scales;  // unfused MXFP4: e8m0 [E, F, d/32]
   const void* down;         // [E, d, F] bf16
   const void* down_bias;    // [E, d] bf16 or null
   const void* sh_gate_up;   // [2Fs, d] bf16
@@ -219,6 +274,9 @@ struct TcArgs {
 };
 cudaError_t launch_tc_gate_up(const TcArgs& a, cudaStream_t st);
 cudaError_t launch_tc_down(const TcArgs& a, cudaStream_t st);
+cudaError_t launch_tcs_gate_up(const TcArgs& a, cudaStream_t st);  // CTA pairs, weights as M
+cudaError_t launch_tcs_down(const TcArgs& a, cudaStream_t st);
+constexpr int kSwapBM = 256;      // token rows per swapped-operand pair tile (the MMA's N, trimmed)
 cudaError_t launch_tc2_gate_up(const TcArgs& a, cudaStream_t st);  // CTA-pair variants
 cudaError_t launch_tc2_down(const TcArgs& a, cudaStream_t st);
 // Split-K reductions (partials -> epilogue) for the bf16 tensor-core GEMMs.
@@ -226,10 +284,15 @@ cudaError_t launch_splitk_gate_up_reduce(const TcArgs& a, cudaStream_t st);
 cudaError_t launch_splitk_down_reduce(const TcArgs& a, cudaStream_t st);
 // Split count for a GEMM of at most `tiles` tiles of `nkb` k-blocks on `sms` SMs.
 int choose_splits(int64_t tiles, int nkb, int sms);
-// MXFP4 expert stacks (gate_up / down are e2m1 codes); no shared expert.
+// MXFP4 expert stacks (gate_up / down are e2m1 codes), routed segments only (a shared
+// expert runs on the CTA-pair bf16 kernel, GemmCommon::seg_begin = E).
 cudaError_t launch_fp4_gate_up(const TcArgs& a, cudaStream_t st);
 cudaError_t launch_fp4_down(const TcArgs& a, cudaStream_t st);
+cudaError_t launch_fp4p_gate_up(const TcArgs& a, cudaStream_t st);  // CTA-pair variants
+cudaError_t launch_fp4p_down(const TcArgs& a, cudaStream_t st);
 constexpr int kFp4BM = 256;       // activation rows per MXFP4 tile (the MMA's N, trimmed to the live rows)
+constexpr int kFp4PairBN = 256;   // weight rows per CTA-pair MXFP4 tile (128 decoded by each CTA)
+constexpr int kFp4PairMinRows = 128;  // CTA pairs when routed rows per expert average at least this
 constexpr int kFp4GuBN = 64;      // h features per MXFP4 gate_up tile (64 gate + 64 up rows)
 constexpr int kFp4DnBN = 128;     // output features per MXFP4 down tile
 

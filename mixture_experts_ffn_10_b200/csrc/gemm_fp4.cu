@@ -62,8 +62,10 @@ static_assert(WST % kCvtGroups == 0, "a group's stages map to its own decoded-we
 
 struct Fp4Params {
   GemmCommon c;
-  const uint8_t* scales;        // e8m0 [E, rows, K/32]
-  const uint16_t* gate_up_bias; // [E, 2F] or null
+  const uint8_t* scales;        // e8m0 [E, rows, K/32] (unfused gate_up: the up rows' scales)
+  const uint8_t* gate_scales;   // unfused gate_up: the gate rows' scales [E, F, d/32]
+  const uint16_t* gate_up_bias; // [E, 2F] ([E, F] unfused / plain) or null
+  const uint16_t* gate_bias;    // unfused: [E, F] or null
   const uint16_t* down_bias;    // [E, d] or null
   const float* roww;            // [R]
   uint16_t* out;                // h [rows, Fmax] or Y [rows, d]
@@ -75,14 +77,25 @@ __device__ __forceinline__ int k_extent(const GemmCommon& c) {
 }
 
 // Row of the scale / code stack (inside expert e) that weight row r of the tile
-// (the MMA's M index) reads.  gate_up: rows 2j, 2j+1 = gate and up rows of
-// feature n_blk * 64 + j.
+// (the MMA's M index) reads.  Gated gate_up: rows 2j, 2j+1 = gate and up rows of
+// feature n_blk * 64 + j (for the unfused layout each in its own stack, *gate
+// set for the gate row); plain gate_up: feature n_blk * 128 + r of fc1.
 template <int MODE>
-__device__ __forceinline__ int weight_row(const GemmCommon& c, int n_blk, int r, bool* valid) {
+__device__ __forceinline__ int weight_row(const GemmCommon& c, int n_blk, int r, bool* valid, bool* gate) {
+  *gate = false;
+  if (MODE == 0 && c.ffn == MOE_FFN_PLAIN) {
+    const int f = n_blk * BNB + r;
+    *valid = f < c.F;
+    return f;
+  }
   if (MODE == 0) {
     const int half = r & 1;
     const int f = n_blk * (BNB / 2) + (r >> 1);
     *valid = f < c.F;
+    if (c.gu_layout == MOE_GU_UNFUSED) {
+      *gate = half == 0;
+      return f;
+    }
     if (c.gu_layout == MOE_GU_INTERLEAVED) return 2 * f + half;
     return half ? c.F + f : f;
   }
@@ -94,7 +107,7 @@ __device__ __forceinline__ int weight_row(const GemmCommon& c, int n_blk, int r,
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ,
-                    const Fp4Params p) {
+                    const __grid_constant__ CUtensorMap tmG, const Fp4Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ringA = smem;                                   // AST x 32 KiB (1024-aligned)
@@ -176,7 +189,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t* sq = ringQ + s * Q_BYTES;
             mbar_arrive_expect_tx(&full[s], Q_BYTES);
             const int kq = kb * (BK / 2);
-            if (MODE == 0) {
+            if (MODE == 0 && c.ffn == MOE_FFN_PLAIN) {
+              tma_load_3d(&tmQ, &full[s], sq, kq, t.n_blk * BNB, t.seg);  // 128 rows of fc1 codes
+            } else if (MODE == 0 && c.gu_layout == MOE_GU_UNFUSED) {
+              const int f0 = t.n_blk * (BNB / 2);  // 64 gate rows, then the 64 up rows
+              tma_load_3d(&tmG, &full[s], sq, kq, f0, t.seg);
+              tma_load_3d(&tmQ, &full[s], sq + Q_BYTES / 2, kq, f0, t.seg);
+            } else if (MODE == 0) {
               const int f0 = t.n_blk * (BNB / 2);
               const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
               for (int half = 0; half < 2; half++)
@@ -247,17 +266,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
       const int live = t.rows - t.m0;      // token rows of the tile (may exceed BM)
       const int64_t grow0 = (int64_t)c.off[t.seg] + t.m0;
-      if (MODE == 0) {
+      if (MODE == 0 && c.ffn == MOE_FFN_PLAIN) {
+        // lane r holds fc1 feature f for the tile's tokens
+        const int f = t.n_blk * BNB + r;
+        const float b = (p.gate_up_bias && f < c.F) ? bf16_to_f32(p.gate_up_bias[(int64_t)t.seg * c.F + f]) : 0.f;
+#pragma unroll 1
+        for (int ch = part; ch < BM / 16 && ch * 16 < live; ch += kEpiGroups) {
+          uint32_t v[16];
+          tmem_ld16(tb + ch * 16, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; i++) {
+            const int tok = ch * 16 + i;
+            if (tok < live && f < c.F)
+              p.out[(grow0 + tok) * c.Fmax + f] = f32_to_bf16_rn(plain_act_bf16(c.act, __uint_as_float(v[i]) + b));
+          }
+        }
+      } else if (MODE == 0) {
         // lanes 2j / 2j+1 hold the gate / up row of feature f; the even lane
         // finishes the chunk's first 8 tokens, the odd lane the last 8
         const int f = t.n_blk * (BNB / 2) + (r >> 1);
         const bool odd = lane & 1;
         float bg = 0.f, bu = 0.f;
-        if (p.gate_up_bias && f < c.F) {
-          const uint16_t* b = p.gate_up_bias + (int64_t)t.seg * 2 * c.F;
-          const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
-          bg = bf16_to_f32(b[il ? 2 * f : f]);
-          bu = bf16_to_f32(b[il ? 2 * f + 1 : c.F + f]);
+        if (f < c.F) {
+          const GuBias gb = gu_bias(c.gu_layout, c.F, t.seg, p.gate_up_bias, p.gate_bias);
+          if (gb.g) bg = bf16_to_f32(gb.g[(int64_t)gb.stride * f]);
+          if (gb.u) bu = bf16_to_f32(gb.u[(int64_t)gb.stride * f]);
         }
 #pragma unroll 1
         for (int ch = part; ch < BM / 16 && ch * 16 < live; ch += kEpiGroups) {
@@ -311,13 +345,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int group = cw / kCvtGroupWarps;       // 0 .. kCvtGroups-1
     const int r = (cw % kCvtGroupWarps) * 32 + lane;  // weight row inside the tile
     const int kblocks = K / 32;                  // scale bytes per weight row
-    const int rows_per_e = MODE == 0 ? 2 * c.F : c.d;
+    const int rows_per_e = MODE == 1 ? c.d : (c.ffn == MOE_FFN_PLAIN || c.gu_layout == MOE_GU_UNFUSED) ? c.F : 2 * c.F;
     uint32_t it = 0;  // stage index of the tile's first k-block
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, it += nkb) {
       const Tile t = decode_tile<BM>(c, tile);
       bool rvalid;
-      const int wr = weight_row<MODE>(c, t.n_blk, r, &rvalid);
-      const uint8_t* srow = p.scales + ((int64_t)t.seg * rows_per_e + wr) * kblocks;
+      bool gate_row;
+      const int wr = weight_row<MODE>(c, t.n_blk, r, &rvalid, &gate_row);
+      const uint8_t* srow = (gate_row ? p.gate_scales : p.scales) + ((int64_t)t.seg * rows_per_e + wr) * kblocks;
       auto load_scales = [&](int kb) -> uint32_t {  // the row's two block scales of k-block kb
         if (!rvalid || kb >= nkb) return 127u | (127u << 8);
         const int col = kb * 2;
@@ -337,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         // code rows in the slot: gate_up 64 gate rows then their 64 up rows; down in order
-        const int qr = MODE == 0 ? (r & 1) * (BNB / 2) + (r >> 1) : r;
+        const int qr = (MODE == 0 && c.ffn == MOE_FFN_GATED) ? (r & 1) * (BNB / 2) + (r >> 1) : r;
         const uint4* qrow = reinterpret_cast<const uint4*>(ringQ + sq * Q_BYTES + qr * (BK / 2));
         const uint4 q0 = qrow[0], q1 = qrow[1];
         __syncwarp();
@@ -398,13 +433,24 @@ bool map_codes_down(CUtensorMap* m, const void* base, uint64_t F, uint64_t d, ui
   return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// An [E][F][d/2] code stack (plain fc1, or an unfused gate or up stack) with
+// boxes of `rows` rows x 32 bytes.
+bool map_codes_rows(CUtensorMap* m, const void* base, uint64_t d, uint64_t F, uint64_t E, uint32_t rows) {
+  const uint64_t kb = d / 2;
+  const uint64_t dims[3] = {kb, F, E};
+  const uint64_t strides[2] = {kb, F * kb};
+  const uint32_t box[3] = {BK / 2, rows, 1};
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 template <int MODE>
-cudaError_t launch(const CUtensorMap& a, const CUtensorMap& q, const Fp4Params& p, int num_sms, cudaStream_t st) {
+cudaError_t launch(const CUtensorMap& a, const CUtensorMap& q, const CUtensorMap& g, const Fp4Params& p,
+                   int num_sms, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(fp4_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = p.c.max_tiles < num_sms ? p.c.max_tiles : num_sms;
-  return launch_pdl(fp4_gemm_kernel<MODE>, (unsigned)grid, kThreads, SMEM_BYTES, st, a, q, p);
+  return launch_pdl(fp4_gemm_kernel<MODE>, (unsigned)grid, kThreads, SMEM_BYTES, st, a, q, g, p);
 }
 
 }  // namespace
@@ -412,12 +458,22 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& q, const Fp4Params& 
 cudaError_t launch_fp4_gate_up(const TcArgs& a, cudaStream_t st) {
   const GemmCommon& c = a.c;
   if (c.max_tiles == 0) return cudaSuccess;
-  CUtensorMap mA, mQ;
+  CUtensorMap mA, mQ, mG;
   bool ok = map_act(&mA, a.xg, c.d, c.R, c.d);
-  ok = ok && map_codes_gate_up(&mQ, a.gate_up, c.d, c.F, c.E, c.gu_layout);
+  if (c.ffn == MOE_FFN_PLAIN) {
+    ok = ok && map_codes_rows(&mQ, a.gate_up, c.d, c.F, c.E, BNB);
+    mG = mQ;
+  } else if (c.gu_layout == MOE_GU_UNFUSED) {
+    ok = ok && map_codes_rows(&mQ, a.gate_up, c.d, c.F, c.E, BNB / 2);
+    ok = ok && map_codes_rows(&mG, a.gate, c.d, c.F, c.E, BNB / 2);
+  } else {
+    ok = ok && map_codes_gate_up(&mQ, a.gate_up, c.d, c.F, c.E, c.gu_layout);
+    mG = mQ;
+  }
   if (!ok) return cudaErrorInvalidValue;
-  Fp4Params p{c, a.gate_up_scales, (const uint16_t*)a.gate_up_bias, nullptr, a.roww, (uint16_t*)a.h};
-  return launch<0>(mA, mQ, p, a.num_sms, st);
+  Fp4Params p{c,       a.gate_up_scales, a.gate_scales, (const uint16_t*)a.gate_up_bias, (const uint16_t*)a.gate_bias,
+              nullptr, a.roww,           (uint16_t*)a.h};
+  return launch<0>(mA, mQ, mG, p, a.num_sms, st);
 }
 
 cudaError_t launch_fp4_down(const TcArgs& a, cudaStream_t st) {
@@ -427,8 +483,8 @@ cudaError_t launch_fp4_down(const TcArgs& a, cudaStream_t st) {
   bool ok = map_act(&mA, a.h, c.F, c.R, c.Fmax);
   ok = ok && map_codes_down(&mQ, a.down, c.F, c.d, c.E);
   if (!ok) return cudaErrorInvalidValue;
-  Fp4Params p{c, a.down_scales, nullptr, (const uint16_t*)a.down_bias, a.roww, (uint16_t*)a.Y};
-  return launch<1>(mA, mQ, p, a.num_sms, st);
+  Fp4Params p{c, a.down_scales, nullptr, nullptr, nullptr, (const uint16_t*)a.down_bias, a.roww, (uint16_t*)a.Y};
+  return launch<1>(mA, mQ, mQ, p, a.num_sms, st);
 }
 
 }  // namespace moe

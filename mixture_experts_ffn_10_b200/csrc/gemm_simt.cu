@@ -48,10 +48,20 @@ __global__ void __launch_bounds__(256) simt_gate_up_kernel(SimtArgs a) {
   const bool shared = ti.seg >= c.E;
   const int K = c.d;
   const int F = shared ? c.Fs : c.F;
-  const float* W = shared ? a.sh_gate_up : a.gate_up + (int64_t)ti.seg * 2 * c.F * c.d;
-  const float* bias = (!shared && a.gate_up_bias) ? a.gate_up_bias + (int64_t)ti.seg * 2 * c.F : nullptr;
+  // plain FFN: the 64 weight rows of a tile are 64 features of fc1 (columns of accg
+  // are features f0 + 2tx + j, of accu features f0 + 32 + 2tx + j); gated: 32 gate
+  // rows and their 32 up rows
+  const bool plain = c.ffn == MOE_FFN_PLAIN;
+  const bool unfused = !shared && !plain && c.gu_layout == MOE_GU_UNFUSED;
+  const int layout = (shared && c.gu_layout == MOE_GU_UNFUSED) ? MOE_GU_CONCAT : c.gu_layout;
+  const GuRows gr = gu_rows(layout, F);
+  const int64_t stack_rows = (plain || unfused) ? F : 2 * F;   // rows of one expert's gate_up stack
+  const float* W = shared ? a.sh_gate_up : a.gate_up + (int64_t)ti.seg * stack_rows * c.d;
+  const float* WG = unfused ? a.gate + (int64_t)ti.seg * F * c.d : W;   // the gate rows' stack
+  const float* bias = (!shared && a.gate_up_bias) ? a.gate_up_bias + (int64_t)ti.seg * stack_rows : nullptr;
+  const float* gbias = unfused ? (a.gate_bias ? a.gate_bias + (int64_t)ti.seg * F : nullptr) : bias;
   const int row_base = c.off[ti.seg];
-  const int f0 = ti.n_blk * kGuFeat;
+  const int f0 = ti.n_blk * kGuFeat * (plain ? 2 : 1);
 
   __shared__ float As[BK][BM + 4];
   __shared__ float Bs[BK][2 * kGuFeat + 4];
@@ -73,13 +83,13 @@ __global__ void __launch_bounds__(256) simt_gate_up_kernel(SimtArgs a) {
     }
     for (int q = threadIdx.x; q < 2 * kGuFeat * BK; q += 256) {
       const int r = q / BK, kk = q % BK;  // r < 32: gate feature r; else up feature r - 32
-      const int f = f0 + (r & (kGuFeat - 1));
+      const int f = plain ? f0 + r : f0 + (r & (kGuFeat - 1));
       const int k = k0 + kk;
       float v = 0.f;
       if (f < F && k < K) {
-        const int wrow = r < kGuFeat ? (c.gu_layout == MOE_GU_INTERLEAVED ? 2 * f : f)
-                                     : (c.gu_layout == MOE_GU_INTERLEAVED ? 2 * f + 1 : F + f);
-        v = W[(int64_t)wrow * K + k];
+        if (plain) v = W[(int64_t)f * K + k];
+        else if (r < kGuFeat) v = WG[(gr.gate0 + (int64_t)gr.stride * f) * K + k];
+        else v = W[(gr.up0 + (int64_t)gr.stride * f) * K + k];
       }
       Bs[kk][r] = v;
     }
@@ -107,14 +117,19 @@ __global__ void __launch_bounds__(256) simt_gate_up_kernel(SimtArgs a) {
     if (row >= ti.rows) continue;
 #pragma unroll
     for (int j = 0; j < 2; j++) {
+      float* hrow = a.h + (int64_t)(row_base + row) * c.Fmax;
+      if (plain) {
+        const int fa = f0 + tx * 2 + j, fb = fa + kGuFeat;
+        if (fa < F) hrow[fa] = plain_act(c.act, accg[i][j] + (bias ? bias[fa] : 0.f));
+        if (fb < F) hrow[fb] = plain_act(c.act, accu[i][j] + (bias ? bias[fb] : 0.f));
+        continue;
+      }
       const int f = f0 + tx * 2 + j;
       if (f >= F) continue;
       float g = accg[i][j], u = accu[i][j];
-      if (bias) {
-        g += bias[c.gu_layout == MOE_GU_INTERLEAVED ? 2 * f : f];
-        u += bias[c.gu_layout == MOE_GU_INTERLEAVED ? 2 * f + 1 : F + f];
-      }
-      a.h[(int64_t)(row_base + row) * c.Fmax + f] = gated_act(c.act, g, u);
+      if (gbias) g += gbias[gr.gate0 + (int64_t)gr.stride * f];
+      if (bias) u += bias[gr.up0 + (int64_t)gr.stride * f];
+      hrow[f] = gated_act(c.act, g, u);
     }
   }
 }

@@ -58,7 +58,8 @@ constexpr uint32_t IDESC = idesc_bf16_f32(BM, BNB);
 
 struct TcParams {
   GemmCommon c;
-  const uint16_t* gate_up_bias;  // [E, 2F] or null
+  const uint16_t* gate_up_bias;  // [E, 2F] ([E, F] unfused / plain) or null
+  const uint16_t* gate_bias;     // unfused: [E, F] or null
   const uint16_t* down_bias;     // [E, d] or null
   const float* roww;             // [R]
   uint16_t* out;                 // h [rows, Fmax] or Y [rows, d]
@@ -73,7 +74,7 @@ template <int MODE, int ABOX>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBs,
-                   const TcParams p) {
+                   const __grid_constant__ CUtensorMap tmG, const TcParams p) {
   constexpr int STAGES = Stage<ABOX>::COUNT, STAGE_BYTES = Stage<ABOX>::BYTES, A_BYTES = Stage<ABOX>::A_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -104,6 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmAs);
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmBs);
+    if (MODE == 0 && c.gu_layout == MOE_GU_UNFUSED) prefetch_tmap(&tmG);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -124,13 +126,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       auto issue = [&](const Tile& t, int kb, uint64_t* bar, uint8_t* sa) {
         const bool sh = t.seg >= c.E;
-        const int arow = sh ? t.m0 : c.off[t.seg] + t.m0;
+        const int arow = (sh || (MODE == 0 && c.direct_x)) ? t.m0 : c.off[t.seg] + t.m0;
         const CUtensorMap* mA = sh ? &tmAs : &tmA;
         const CUtensorMap* mB = sh ? &tmBs : &tmB;
         const int e = sh ? 0 : t.seg;
         const int k0 = kb * BK;
         tma_load_2d(mA, bar, sa, k0, arow);
-        if (MODE == 0) {
+        if (MODE == 0 && c.ffn == MOE_FFN_PLAIN) {
+          tma_load_3d(mB, bar, sa + A_BYTES, k0, t.n_blk * BNB, e);  // 256 rows of fc1 [E][F][d]
+        } else if (MODE == 0 && c.gu_layout == MOE_GU_UNFUSED && !sh) {
+          const int f0 = t.n_blk * (BNB / 2);  // 128 gate rows, then the 128 up rows
+          tma_load_3d(&tmG, bar, sa + A_BYTES, k0, f0, e);
+          tma_load_3d(mB, bar, sa + A_BYTES + B_BYTES / 2, k0, f0, e);
+        } else if (MODE == 0) {
           const int f0 = t.n_blk * (BNB / 2);
           const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
           for (int half = 0; half < 2; half++) {
@@ -214,8 +222,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
       const int row = t.m0 + r_in_tile;
-      const bool valid = row < t.rows;
-      const int64_t grow = (int64_t)c.off[t.seg] + row;
+      bool valid = row < t.rows;
+      int64_t grow = (int64_t)c.off[t.seg] + row;
+      float wi = 1.f;  // weigh-inputs scale of the accumulators (direct_x only)
+      if (MODE == 0 && c.direct_x && !sh) {
+        // accumulator row = token r_in_tile: its row of this expert, if it chose it
+        valid = false;
+        if (r_in_tile < c.T) {
+          for (int j = 0; j < c.k; j++)
+            if (c.topk_idx[(int64_t)r_in_tile * c.k + j] == t.seg) {
+              grow = c.pos[(int64_t)r_in_tile * c.k + j];
+              valid = true;
+            }
+        }
+        if (valid && c.weigh_inputs) wi = p.roww[grow];
+      }
       if (S > 1) {
         // split-K: this unit's fp32 partial accumulator row goes to the partial buffer
         if (__any_sync(0xffffffffu, valid)) {
@@ -236,11 +257,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else if (__any_sync(0xffffffffu, valid)) {
-        if (MODE == 0) {
+        if (MODE == 0 && c.ffn == MOE_FFN_PLAIN) {
+          const int F = sh ? c.Fs : c.F;
+          const int f0 = t.n_blk * BNB;
+          const uint16_t* bias = (!sh && p.gate_up_bias) ? p.gate_up_bias + (int64_t)t.seg * c.F : nullptr;
+          uint16_t* out = p.out + grow * c.Fmax;
+#pragma unroll 1
+          for (int ch = part; ch < BNB / 16; ch += kEpiGroups) {
+            uint32_t v[16];
+            tmem_ld16(tb + ch * 16, v);
+            tmem_ld_wait();
+            const int fb = f0 + ch * 16;
+            if (valid && fb < F) plain_chunk(v, bias, fb, F, c.act, wi, out);
+          }
+        } else if (MODE == 0) {
           const int F = sh ? c.Fs : c.F;
           const int f0 = t.n_blk * (BNB / 2);
-          const uint16_t* bias = (!sh && p.gate_up_bias) ? p.gate_up_bias + (int64_t)t.seg * 2 * c.F : nullptr;
-          const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
+          const GuBias gb = sh ? GuBias{nullptr, nullptr, 1}
+                               : gu_bias(c.gu_layout, c.F, t.seg, p.gate_up_bias, p.gate_bias);
           uint16_t* out = p.out + grow * c.Fmax;
 #pragma unroll 1
           for (int ch = part; ch < (BNB / 2) / 16; ch += kEpiGroups) {
@@ -249,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld16(tb + BNB / 2 + ch * 16, u);
             tmem_ld_wait();
             const int fb = f0 + ch * 16;
-            if (valid && fb < F) gate_up_chunk(g, u, bias, fb, F, il, c.act, out);
+            if (valid && fb < F) gate_up_chunk(g, u, gb.g, gb.u, gb.stride, fb, F, c.act, wi, out);
           }
         } else {
           const int n0 = t.n_blk * BNB;
@@ -320,13 +354,13 @@ bool map_down(CUtensorMap* m, const void* base, uint64_t F, uint64_t d, uint64_t
 
 template <int MODE, int ABOX>
 cudaError_t launch_box(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMap& b, const CUtensorMap& bs,
-                       const TcParams& p, int num_sms, cudaStream_t st) {
+                       const CUtensorMap& g, const TcParams& p, int num_sms, cudaStream_t st) {
   constexpr int smem = Stage<ABOX>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE, ABOX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int units = p.c.max_tiles * p.c.splits;
   const int grid = units < num_sms ? units : num_sms;
-  return launch_pdl(tc_gemm_kernel<MODE, ABOX>, (unsigned)grid, kThreads, smem, st, a, as, b, bs, p);
+  return launch_pdl(tc_gemm_kernel<MODE, ABOX>, (unsigned)grid, kThreads, smem, st, a, as, b, bs, g, p);
 }
 
 // Activation rows each stage loads: no segment has more rows than there are tokens.
@@ -334,10 +368,24 @@ int a_box_rows(const GemmCommon& c) { return c.T <= 32 ? 32 : c.T <= 64 ? 64 : B
 
 template <int MODE>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMap& b, const CUtensorMap& bs,
-                   const TcParams& p, int abox, int num_sms, cudaStream_t st) {
-  if (abox == 32) return launch_box<MODE, 32>(a, as, b, bs, p, num_sms, st);
-  if (abox == 64) return launch_box<MODE, 64>(a, as, b, bs, p, num_sms, st);
-  return launch_box<MODE, BM>(a, as, b, bs, p, num_sms, st);
+                   const CUtensorMap& g, const TcParams& p, int abox, int num_sms, cudaStream_t st) {
+  if (abox == 32) return launch_box<MODE, 32>(a, as, b, bs, g, p, num_sms, st);
+  if (abox == 64) return launch_box<MODE, 64>(a, as, b, bs, g, p, num_sms, st);
+  return launch_box<MODE, BM>(a, as, b, bs, g, p, num_sms, st);
+}
+
+// Maps of one gate_up weight stack (E experts of F features): a plain fc1 [E][F][d]
+// in boxes of 256 rows; an unfused gate or up stack [E][F][d] in boxes of 128 rows;
+// a fused stack [E][2F][d] through the 4-D view.
+bool map_fc1(CUtensorMap* m, const void* base, uint64_t d, uint64_t F, uint64_t E, int ffn, int layout) {
+  if (ffn == MOE_FFN_PLAIN) return map_down(m, base, d, F, E);  // same shape: {d, F, E}, box 64 x 256
+  if (layout == MOE_GU_UNFUSED) {
+    const uint64_t dims[3] = {d, F, E};
+    const uint64_t strides[2] = {d * 2, F * d * 2};
+    const uint32_t box[3] = {BK, BNB / 2, 1};
+    return make_map(m, base, 3, dims, strides, box);
+  }
+  return map_gate_up(m, base, d, F, E, layout);
 }
 
 }  // namespace
@@ -345,20 +393,26 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMa
 cudaError_t launch_tc_gate_up(const TcArgs& a, cudaStream_t st) {
   const GemmCommon& c = a.c;
   if (c.max_tiles == 0) return cudaSuccess;
-  CUtensorMap mA, mAs, mB, mBs;
+  CUtensorMap mA, mAs, mB, mBs, mG;
   const int abox = a_box_rows(c);
-  bool ok = map_rows(&mA, a.xg, c.d, c.R, c.d, abox);
-  ok = ok && map_gate_up(&mB, a.gate_up, c.d, c.F, c.E, c.gu_layout);
+  // small batches read the activation rows from x itself (direct_x), else the rows
+  // gathered into expert order
+  bool ok = c.direct_x ? map_rows(&mA, a.x, c.d, c.T, c.d, abox) : map_rows(&mA, a.xg, c.d, c.R, c.d, abox);
+  ok = ok && map_fc1(&mB, a.gate_up, c.d, c.F, c.E, c.ffn, c.gu_layout);
+  if (c.gu_layout == MOE_GU_UNFUSED) ok = ok && map_fc1(&mG, a.gate, c.d, c.F, c.E, c.ffn, c.gu_layout);
+  else mG = mB;
   if (c.Fs > 0) {
+    // the shared expert keeps one stack (gate rows first when the routed experts are unfused)
+    const int sh_layout = c.gu_layout == MOE_GU_UNFUSED ? MOE_GU_CONCAT : c.gu_layout;
     ok = ok && map_rows(&mAs, a.x, c.d, c.T, c.d, abox);
-    ok = ok && map_gate_up(&mBs, a.sh_gate_up, c.d, c.Fs, 1, c.gu_layout);
+    ok = ok && map_fc1(&mBs, a.sh_gate_up, c.d, c.Fs, 1, c.ffn, sh_layout);
   } else {
     mAs = mA;
     mBs = mB;
   }
   if (!ok) return cudaErrorInvalidValue;
-  TcParams p{c, (const uint16_t*)a.gate_up_bias, nullptr, a.roww, (uint16_t*)a.h};
-  return launch<0>(mA, mAs, mB, mBs, p, abox, a.num_sms, st);
+  TcParams p{c, (const uint16_t*)a.gate_up_bias, (const uint16_t*)a.gate_bias, nullptr, a.roww, (uint16_t*)a.h};
+  return launch<0>(mA, mAs, mB, mBs, mG, p, abox, a.num_sms, st);
 }
 
 cudaError_t launch_tc_down(const TcArgs& a, cudaStream_t st) {
@@ -376,8 +430,8 @@ cudaError_t launch_tc_down(const TcArgs& a, cudaStream_t st) {
     mBs = mB;
   }
   if (!ok) return cudaErrorInvalidValue;
-  TcParams p{c, nullptr, (const uint16_t*)a.down_bias, a.roww, (uint16_t*)a.Y};
-  return launch<1>(mA, mAs, mB, mBs, p, abox, a.num_sms, st);
+  TcParams p{c, nullptr, nullptr, (const uint16_t*)a.down_bias, a.roww, (uint16_t*)a.Y};
+  return launch<1>(mA, mAs, mB, mBs, mB, p, abox, a.num_sms, st);
 }
 
 }  // namespace moe

@@ -59,7 +59,8 @@ constexpr uint16_t kEvenCta = 0x1;
 
 struct Tc2Params {
   GemmCommon c;
-  const uint16_t* gate_up_bias;  // [E, 2F] or null
+  const uint16_t* gate_up_bias;  // [E, 2F] ([E, F] unfused / plain) or null
+  const uint16_t* gate_bias;     // unfused: [E, F] or null
   const uint16_t* down_bias;     // [E, d] or null
   const float* roww;             // [R]
   uint16_t* out;                 // h [rows, Fmax] or Y [rows, d]
@@ -74,7 +75,7 @@ template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBs,
-                    const Tc2Params p) {
+                    const __grid_constant__ CUtensorMap tmG, const Tc2Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
@@ -119,13 +120,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int S = 1;  // the plan never splits K for pair tiles (launch rejects it)
   const int total = c.tiles[c.NS];
+  const int first = c.tiles[c.seg_begin];  // tiles of segments seg_begin .. NS-1 only
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int unit = cluster; ok && unit < total; unit += nclusters) {
+      for (int unit = first + cluster; ok && unit < total; unit += nclusters) {
         const Tile t = decode_tile<BM2>(c, unit / S);
         const bool sh = t.seg >= c.E;
         const int nkb = (k_extent<MODE>(c, sh) + BK - 1) / BK;
@@ -150,7 +152,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint8_t* sa = smem + s * STAGE_BYTES;
           const int k0 = kb * BK;
           tma_load_2d_pair(mA, fb, sa, k0, arow);
-          if (MODE == 0) {
+          if (MODE == 0 && c.ffn == MOE_FFN_PLAIN) {
+            // CTA r: fc1 rows n_blk * 256 + 128 r .. + 127
+            tma_load_3d_pair(mB, fb, sa + A_BYTES, k0, t.n_blk * BNB + BNC * (int)rank, e);
+          } else if (MODE == 0 && c.gu_layout == MOE_GU_UNFUSED && !sh) {
+            // CTA 0: 128 rows of the gate stack, CTA 1: the matching up rows
+            tma_load_3d_pair(rank == 0 ? &tmG : mB, fb, sa + A_BYTES, k0, t.n_blk * BNC, e);
+          } else if (MODE == 0) {
             const int f0 = t.n_blk * BNC;
             const int half = (int)rank;  // CTA 0: gate rows, CTA 1: up rows
             const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
@@ -174,7 +182,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0 && rank == 0) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (int unit = cluster; ok && unit < total; unit += nclusters, tcount++) {
+      for (int unit = first + cluster; ok && unit < total; unit += nclusters, tcount++) {
         const Tile t = decode_tile<BM2>(c, unit / S);
         const int nkb = (k_extent<MODE>(c, t.seg >= c.E) + BK - 1) / BK;
         const int sp = unit % S, kb0 = sp * nkb / S, kb1 = (sp + 1) * nkb / S;
@@ -211,7 +219,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int r_in_tile = BMC * (int)rank + q * 32 + lane;
     const uint32_t tempty_even0 = mapa_shared(&tempty[0], 0), tempty_even1 = mapa_shared(&tempty[1], 0);
     uint32_t tcount = 0;
-    for (int unit = cluster; unit < total; unit += nclusters, tcount++) {
+    for (int unit = first + cluster; unit < total; unit += nclusters, tcount++) {
       const Tile t = decode_tile<BM2>(c, unit / S);
       const bool sh = t.seg >= c.E;
       const int acc = tcount & 1;
@@ -224,11 +232,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool valid = row < t.rows;
       const int64_t grow = (int64_t)c.off[t.seg] + row;
       if (__any_sync(0xffffffffu, valid)) {
-        if (MODE == 0) {
+        if (MODE == 0 && c.ffn == MOE_FFN_PLAIN) {
+          const int F = sh ? c.Fs : c.F;
+          const int f0 = t.n_blk * BNB;
+          const uint16_t* bias = (!sh && p.gate_up_bias) ? p.gate_up_bias + (int64_t)t.seg * c.F : nullptr;
+          uint16_t* out = p.out + grow * c.Fmax;
+#pragma unroll 1
+          for (int ch = 0; ch < BNB / 16; ch++) {
+            uint32_t v[16];
+            tmem_ld16(tb + ch * 16, v);
+            tmem_ld_wait();
+            const int fb = f0 + ch * 16;
+            if (valid && fb < F) plain_chunk(v, bias, fb, F, c.act, 1.f, out);
+          }
+        } else if (MODE == 0) {
           const int F = sh ? c.Fs : c.F;
           const int f0 = t.n_blk * BNC;
-          const uint16_t* bias = (!sh && p.gate_up_bias) ? p.gate_up_bias + (int64_t)t.seg * 2 * c.F : nullptr;
-          const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
+          const GuBias gb = sh ? GuBias{nullptr, nullptr, 1}
+                               : gu_bias(c.gu_layout, c.F, t.seg, p.gate_up_bias, p.gate_bias);
           uint16_t* out = p.out + grow * c.Fmax;
 #pragma unroll 1
           for (int ch = 0; ch < BNC / 16; ch++) {
@@ -237,7 +258,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tmem_ld16(tb + BNC + ch * 16, u);
             tmem_ld_wait();
             const int fb = f0 + ch * 16;
-            if (valid && fb < F) gate_up_chunk(g, u, bias, fb, F, il, c.act, out);
+            if (valid && fb < F) gate_up_chunk(g, u, gb.g, gb.u, gb.stride, fb, F, c.act, 1.f, out);
           }
         } else {
           const int n0 = t.n_blk * BNB;
@@ -307,6 +328,14 @@ bool map_down(CUtensorMap* m, const void* base, uint64_t F, uint64_t d, uint64_t
   return make_map(m, base, 3, dims, strides, box);
 }
 
+// One CTA's half of a gate_up weight stack (E experts of F features), box 128 rows:
+// a plain fc1 or an unfused gate or up stack [E][F][d] as 3-D; a fused stack
+// [E][2F][d] through the 4-D view.
+bool map_fc1(CUtensorMap* m, const void* base, uint64_t d, uint64_t F, uint64_t E, int ffn, int layout) {
+  if (ffn == MOE_FFN_PLAIN || layout == MOE_GU_UNFUSED) return map_down(m, base, d, F, E);
+  return map_gate_up(m, base, d, F, E, layout);
+}
+
 // Co-resident clusters of the kernel on the current device (cached per device and mode).
 template <int MODE>
 int max_clusters(int num_sms) {
@@ -330,7 +359,7 @@ int max_clusters(int num_sms) {
 
 template <int MODE>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMap& b, const CUtensorMap& bs,
-                   const Tc2Params& p, int num_sms, cudaStream_t st) {
+                   const CUtensorMap& g, const Tc2Params& p, int num_sms, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(tc2_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SMEM_BYTES);
   if (e != cudaSuccess) return e;
@@ -338,7 +367,7 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMa
   const int units = p.c.max_tiles;
   const int mc = max_clusters<MODE>(num_sms);
   const int clusters = units < mc ? units : mc;
-  return launch_pdl(tc2_gemm_kernel<MODE>, (unsigned)(2 * clusters), kThreads, SMEM_BYTES, st, a, as, b, bs, p);
+  return launch_pdl(tc2_gemm_kernel<MODE>, (unsigned)(2 * clusters), kThreads, SMEM_BYTES, st, a, as, b, bs, g, p);
 }
 
 }  // namespace
@@ -346,27 +375,44 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMa
 cudaError_t launch_tc2_gate_up(const TcArgs& a, cudaStream_t st) {
   const GemmCommon& c = a.c;
   if (c.max_tiles == 0) return cudaSuccess;
-  CUtensorMap mA, mAs, mB, mBs;
-  bool ok = map_rows(&mA, a.xg, c.d, c.R, c.d);
-  ok = ok && map_gate_up(&mB, a.gate_up, c.d, c.F, c.E, c.gu_layout);
+  CUtensorMap mA, mAs, mB, mBs, mG;
+  // the shared expert alone (beside MXFP4 experts) needs no maps of the routed stacks
+  const bool shared_only = c.seg_begin >= c.E;
+  bool ok = true;
+  if (!shared_only) {
+    ok = map_rows(&mA, a.xg, c.d, c.R, c.d);
+    ok = ok && map_fc1(&mB, a.gate_up, c.d, c.F, c.E, c.ffn, c.gu_layout);
+    if (c.gu_layout == MOE_GU_UNFUSED) ok = ok && map_fc1(&mG, a.gate, c.d, c.F, c.E, c.ffn, c.gu_layout);
+    else mG = mB;
+  }
   if (c.Fs > 0) {
+    // the shared expert keeps one stack (gate rows first when the routed experts are unfused)
+    const int sh_layout = c.gu_layout == MOE_GU_UNFUSED ? MOE_GU_CONCAT : c.gu_layout;
     ok = ok && map_rows(&mAs, a.x, c.d, c.T, c.d);
-    ok = ok && map_gate_up(&mBs, a.sh_gate_up, c.d, c.Fs, 1, c.gu_layout);
+    ok = ok && map_fc1(&mBs, a.sh_gate_up, c.d, c.Fs, 1, c.ffn, sh_layout);
   } else {
     mAs = mA;
     mBs = mB;
   }
+  if (shared_only) {
+    mA = mAs;
+    mB = mG = mBs;
+  }
   if (!ok) return cudaErrorInvalidValue;
-  Tc2Params p{c, (const uint16_t*)a.gate_up_bias, nullptr, a.roww, (uint16_t*)a.h};
-  return launch<0>(mA, mAs, mB, mBs, p, a.num_sms, st);
+  Tc2Params p{c, (const uint16_t*)a.gate_up_bias, (const uint16_t*)a.gate_bias, nullptr, a.roww, (uint16_t*)a.h};
+  return launch<0>(mA, mAs, mB, mBs, mG, p, a.num_sms, st);
 }
 
 cudaError_t launch_tc2_down(const TcArgs& a, cudaStream_t st) {
   const GemmCommon& c = a.c;
   if (c.max_tiles == 0) return cudaSuccess;
   CUtensorMap mA, mAs, mB, mBs;
-  bool ok = map_rows(&mA, a.h, c.F, c.R, c.Fmax);
-  ok = ok && map_down(&mB, a.down, c.F, c.d, c.E);
+  const bool shared_only = c.seg_begin >= c.E;  // beside MXFP4 experts
+  bool ok = true;
+  if (!shared_only) {
+    ok = map_rows(&mA, a.h, c.F, c.R, c.Fmax);
+    ok = ok && map_down(&mB, a.down, c.F, c.d, c.E);
+  }
   if (c.Fs > 0) {
     ok = ok && map_rows(&mAs, (const uint16_t*)a.h + (int64_t)c.R * c.Fmax, c.Fs, c.T, c.Fmax);
     ok = ok && map_down(&mBs, a.sh_down, c.Fs, c.d, 1);
@@ -374,9 +420,13 @@ cudaError_t launch_tc2_down(const TcArgs& a, cudaStream_t st) {
     mAs = mA;
     mBs = mB;
   }
+  if (shared_only) {
+    mA = mAs;
+    mB = mBs;
+  }
   if (!ok) return cudaErrorInvalidValue;
-  Tc2Params p{c, nullptr, (const uint16_t*)a.down_bias, a.roww, (uint16_t*)a.Y};
-  return launch<1>(mA, mAs, mB, mBs, p, a.num_sms, st);
+  Tc2Params p{c, nullptr, nullptr, (const uint16_t*)a.down_bias, a.roww, (uint16_t*)a.Y};
+  return launch<1>(mA, mAs, mB, mBs, mB, p, a.num_sms, st);
 }
 
 }  // namespace moe

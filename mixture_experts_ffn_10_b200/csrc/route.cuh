@@ -72,9 +72,10 @@ __device__ __forceinline__ float load_logit(const void* p, int bf16, int64_t i) 
   return bf16 ? bf16_to_f32(((const uint16_t*)p)[i]) : ((const float*)p)[i];
 }
 
-// Routes token t with the calling warp (lane = this thread's lane).
+// Routes token t with the calling warp (lane = this thread's lane).  The token's
+// logits are read from a.logits, or from lrow (fp32, E values) when it is given.
 template <int EPL>  // experts per lane: E <= 32 * EPL, expert e = lane + 32 * i
-__device__ __forceinline__ void route_token(const RouteArgs& a, int t, int lane) {
+__device__ __forceinline__ void route_token(const RouteArgs& a, int t, int lane, const float* lrow = nullptr) {
   const int E = a.E;
 
   float lp[EPL];
@@ -83,7 +84,7 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, int t, int lane)
     const int e = lane + 32 * i;
     float l = 0.f;
     if (e < E) {
-      l = load_logit(a.logits, a.logit_bf16, (int64_t)t * E + e);
+      l = lrow ? lrow[e] : load_logit(a.logits, a.logit_bf16, (int64_t)t * E + e);
       if (a.router_bias) l = l + load_logit(a.router_bias, a.logit_bf16, e);
     }
     lp[i] = l;
@@ -92,14 +93,15 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, int t, int lane)
   // ---- scores (double)
   double s[EPL];
   if (a.score == MOE_SCORE_SOFTMAX) {
-    float m = -INFINITY;
+    float m = -INFINITY;  // NaN logits never compare greater, so they never become the max
 #pragma unroll
     for (int i = 0; i < EPL; i++)
       if (lane + 32 * i < E && lp[i] > m) m = lp[i];
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      const float v = __shfl_xor_sync(0xffffffffu, m, o);
-      m = v > m ? v : m;
+    {  // warp max on the order-preserving image of the (non-NaN) fp32 values
+      uint32_t u = __float_as_uint(m);
+      u = (u >> 31) ? ~u : (u | 0x80000000u);
+      u = __reduce_max_sync(0xffffffffu, u);
+      m = __uint_as_float((u >> 31) ? (u & 0x7fffffffu) : ~u);
     }
     double den = 0.0;
 #pragma unroll
@@ -195,14 +197,15 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, int t, int lane)
         bi = e;
       }
     }
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) {
-      const uint64_t ok = __shfl_xor_sync(0xffffffffu, bk, m);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, m);
-      if (ahead(ok, oi, bk, bi)) {
-        bk = ok;
-        bi = oi;
-      }
+    // warp arg-best in three single-instruction warp reductions (same order as
+    // ahead()): the largest high word of the key images, the largest low word among
+    // the lanes holding it, then the lowest expert index among the lanes holding both
+    {
+      const uint32_t hi = (uint32_t)(bk >> 32), lo = (uint32_t)bk;
+      const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+      const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
+      const uint32_t cand = (hi == mhi && lo == mlo) ? (uint32_t)bi : (uint32_t)kNone;
+      bi = (int)__reduce_min_sync(0xffffffffu, cand);
     }
     // the winner's owner lane marks it taken and hands its score to lane j
     double sv = 0.0;

@@ -95,52 +95,67 @@ __global__ void __launch_bounds__(kScatterWarps * 32) scatter_kernel(SortArgs a)
   scatter_chunk(a, t0, (min(a.T, t0 + kChunkTokens) - t0) * a.k, a.off, a.hist + (int64_t)b * a.E, run);
 }
 
-// xg[r] = x[perm[r]] (times roww[r] for weigh-inputs), 16-byte vectors: one warp
-// per row and slice of the row; slice blockIdx.y of gridDim.y (more than one only
-// when there are too few rows to fill the GPU).
+// xg[pos[t, j]] = x[t] (times the row's routing weight for weigh-inputs), token
+// by token, so that x is read once and written k times: one warp per token and
+// slice of its row (slice blockIdx.y of gridDim.y; more than one only when there
+// are too few tokens to fill the GPU), 16-byte vectors.
 template <typename T>
 __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
-  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (r >= a.R) return;
-  const int t = a.perm[r];
-  if (t < 0 || t >= a.T) {
-    if (lane == 0) set_status(a.status, MOE_ERR_SHAPE);
-    return;
-  }
+  const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= a.T) return;
   constexpr int kVec = 16 / sizeof(T);
   const int nv = a.d / kVec;
   const int per = (nv + gridDim.y - 1) / gridDim.y;
   const int v0 = blockIdx.y * per, v1 = min(nv, v0 + per);
-  const uint4* src = reinterpret_cast<const uint4*>((const T*)a.x + (int64_t)t * a.d);
-  uint4* dst = reinterpret_cast<uint4*>((T*)a.xg + r * a.d);
-  const float w = a.weigh_inputs ? a.roww[r] : 1.f;
-  // four vectors per lane in flight: loads first, then the (scaled) stores
+  const uint4* src = reinterpret_cast<const uint4*>((const T*)a.x + t * a.d);
+  // each lane holds the row and weight of slot (lane mod k); shuffled to every lane
+  int my_row = 0;
+  float my_w = 1.f;
+  if (lane < a.k) {
+    my_row = a.pos[t * a.k + lane];
+    if (my_row < 0 || my_row >= a.R) {
+      set_status(a.status, MOE_ERR_SHAPE);
+      my_row = -1;
+    } else if (a.weigh_inputs) {
+      my_w = a.roww[my_row];
+    }
+  }
+  if (__any_sync(0xffffffffu, my_row < 0)) return;
+  // four vectors per lane in flight: loads first, then the k (scaled) stores of each;
+  // every lane runs every iteration (the shuffles below need the whole warp)
   constexpr int kBatch = 4;
-  for (int v = v0 + lane; v < v1; v += 32 * kBatch) {
+  for (int vb = v0; vb < v1; vb += 32 * kBatch) {
+    const int v = vb + lane;
     uint4 q[kBatch];
 #pragma unroll
     for (int b = 0; b < kBatch; b++)
       if (v + 32 * b < v1) q[b] = __ldg(src + v + 32 * b);
+    for (int j = 0; j < a.k; j++) {
+      const int row = __shfl_sync(0xffffffffu, my_row, j);
+      const float w = __shfl_sync(0xffffffffu, my_w, j);
+      uint4* dst = reinterpret_cast<uint4*>((T*)a.xg + (int64_t)row * a.d);
 #pragma unroll
-    for (int b = 0; b < kBatch; b++) {
-      if (v + 32 * b >= v1) break;
-      if (a.weigh_inputs) {
-        if constexpr (sizeof(T) == 2) {
-          uint32_t* u = reinterpret_cast<uint32_t*>(&q[b]);
+      for (int b = 0; b < kBatch; b++) {
+        if (v + 32 * b >= v1) break;
+        uint4 o = q[b];
+        if (a.weigh_inputs) {
+          if constexpr (sizeof(T) == 2) {
+            uint32_t* u = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-          for (int i = 0; i < 4; i++) {
-            const float lo = bf16_to_f32(u[i] & 0xffff) * w, hi = bf16_to_f32(u[i] >> 16) * w;
-            u[i] = pack_bf16x2(lo, hi);
+            for (int i = 0; i < 4; i++) {
+              const float lo = bf16_to_f32(u[i] & 0xffff) * w, hi = bf16_to_f32(u[i] >> 16) * w;
+              u[i] = pack_bf16x2(lo, hi);
+            }
+          } else {
+            float* f = reinterpret_cast<float*>(&o);
+#pragma unroll
+            for (int i = 0; i < 4; i++) f[i] *= w;
           }
-        } else {
-          float* f = reinterpret_cast<float*>(&q[b]);
-#pragma unroll
-          for (int i = 0; i < 4; i++) f[i] *= w;
         }
+        dst[v + 32 * b] = o;
       }
-      dst[v + 32 * b] = q[b];
     }
   }
 }
@@ -162,8 +177,8 @@ cudaError_t launch_sort(const SortArgs& a, cudaStream_t st) {
 
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t st) {
   if (a.R == 0) return cudaSuccess;
-  const int blocks = (a.R + 7) / 8;
-  // few rows: split each row into slices of at least 32 vectors until ~512 blocks
+  const int blocks = (a.T + 7) / 8;
+  // few tokens: split each row into slices of at least 32 vectors until ~512 blocks
   const int nv = a.d / (a.bf16 ? 8 : 4);
   int slices = 1;
   while (blocks * slices * 2 <= 512 && nv / (slices * 2) >= 32) slices *= 2;

@@ -31,6 +31,19 @@ __global__ void __launch_bounds__(128) reduce_gate_up_kernel(TcArgs a) {
   const int F = sh ? c.Fs : c.F;
   if (f >= F) return;
   const int rows = c.R + (c.Fs > 0 ? c.T : 0);
+  uint16_t* out = reinterpret_cast<uint16_t*>(a.h) + (int64_t)row * c.Fmax + f;
+  // weigh-inputs on x read in place (direct_x): W (w x) = w (W x)
+  const float wi = (!sh && c.direct_x && c.weigh_inputs) ? a.roww[row] : 1.f;
+  if (c.ffn == MOE_FFN_PLAIN) {  // tile columns are features: column f
+    float v = 0.f;
+    for (int sp = 0; sp < c.splits; sp++) v += c.partial[((int64_t)sp * rows + row) * c.partial_pitch + f];
+    v *= wi;
+    if (!sh && a.gate_up_bias) v += bf16_to_f32(((const uint16_t*)a.gate_up_bias)[(int64_t)seg * c.F + f]);
+    *out = f32_to_bf16_rn(plain_act_bf16(c.act, v));
+    return;
+  }
+  // gated: a tile of 128 features holds the gate values in columns 0..127 and the
+  // up values in 128..255
   const int64_t col = (int64_t)(f / 128) * 256 + (f % 128);
   float g = 0.f, u = 0.f;
   for (int sp = 0; sp < c.splits; sp++) {
@@ -38,13 +51,14 @@ __global__ void __launch_bounds__(128) reduce_gate_up_kernel(TcArgs a) {
     g += pr[col];
     u += pr[col + 128];
   }
-  const uint16_t* bias = (!sh && a.gate_up_bias) ? (const uint16_t*)a.gate_up_bias + (int64_t)seg * 2 * c.F : nullptr;
-  if (bias) {
-    const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
-    g += bf16_to_f32(bias[il ? 2 * f : f]);
-    u += bf16_to_f32(bias[il ? 2 * f + 1 : F + f]);
+  g *= wi;
+  u *= wi;
+  if (!sh) {
+    const GuBias gb = gu_bias(c.gu_layout, c.F, seg, (const uint16_t*)a.gate_up_bias, (const uint16_t*)a.gate_bias);
+    if (gb.g) g += bf16_to_f32(gb.g[(int64_t)gb.stride * f]);
+    if (gb.u) u += bf16_to_f32(gb.u[(int64_t)gb.stride * f]);
   }
-  reinterpret_cast<uint16_t*>(a.h)[(int64_t)row * c.Fmax + f] = f32_to_bf16_rn(gated_act_bf16(c.act, g, u));
+  *out = f32_to_bf16_rn(gated_act_bf16(c.act, g, u));
 }
 
 // One block per (row, 256 outputs); thread = output feature.

@@ -46,10 +46,10 @@ def test_library_exports_every_declared_symbol(moe):
 
 
 def test_struct_sizes_match_the_header(moe):
-    # int64 x 6 + int32 x 4; 12 x 4-byte fields; 17 pointers
+    # int64 x 6 + int32 x 4; 13 x 4-byte fields; 22 pointers
     assert C.sizeof(moe.moe_shape) == 64
-    assert C.sizeof(moe.moe_options) == 48
-    assert C.sizeof(moe.moe_tensors) == 17 * 8
+    assert C.sizeof(moe.moe_options) == 52
+    assert C.sizeof(moe.moe_tensors) == 22 * 8
 
 
 def test_options_defaults(moe):
@@ -107,6 +107,15 @@ def _tensors(moe, **kw):
     ({}, {}, dict(gate_up=FAKE + 8), 4),
     ({}, {}, dict(y=FAKE), 9),
     (dict(Fs=64), {}, {}, 1),
+    ({}, dict(gu_layout="unfused"), {}, 1),                           # no gate stack
+    ({}, dict(gu_layout="unfused", ffn="plain"), dict(gate=FAKE), 9),  # unfused needs a gated FFN
+    ({}, {}, dict(gate=FAKE), 9),                                      # gate given to a fused layout
+    (dict(w_dtype="mxfp4"), dict(gu_layout="unfused"),
+     dict(gate=FAKE, gate_up_scales=FAKE, down_scales=FAKE), 1),     # no gate_scales
+    ({}, {}, dict(router_weight=FAKE), 9),                             # logits and router weight
+    ({}, {}, dict(router_logits=None, router_weight=FAKE, x=None), 1),
+    ({}, {}, dict(logits_out=FAKE), 9),                                # logits_out without router weight
+    ({}, {}, dict(gate=FAKE + 8), 9),
 ])
 def test_validation_rejects_before_launch(moe, shape_kw, opt_kw, tens_kw, code):
     s = _valid(moe, **shape_kw)
@@ -114,6 +123,8 @@ def test_validation_rejects_before_launch(moe, shape_kw, opt_kw, tens_kw, code):
     t = _tensors(moe, **tens_kw)
     if tens_kw.get("y") == FAKE:
         t.x = FAKE  # y aliases x
+    else:
+        t.y = 2 * FAKE
     rc = moe.moe_forward(s, o, t, FAKE, 1 << 40, None)
     assert rc == code, (rc, moe.moe_last_error())
     assert moe.moe_last_error()
@@ -169,14 +180,14 @@ def test_binding_without_its_library_imports_but_every_entry_point_raises(tmp_pa
 
 
 @pytest.mark.parametrize("name,count", [
-    ("tiny_fp32", 6), ("decode_T1", 7), ("decode_T8", 6), ("decode_T64", 6), ("decode_T256", 8),
+    ("tiny_fp32", 6), ("decode_T1", 6), ("decode_T8", 5), ("decode_T64", 5), ("decode_T256", 8),
     ("mixtral_bf16", 8), ("gptoss_mxfp4", 8), ("deepseek_bf16", 8)])
 def test_kernel_count_of_each_workload(moe, name, count):
     """The launch plan on a 148-SM part (what the host assumes without a GPU): route,
     sort (one kernel for a single 64-token chunk, else histogram + scan + scatter),
-    gather, gate_up, down, combine, plus a reduction per GEMM whose K is split.  Decode
-    T=1 splits gate_up only (96 tiles of 64 k-blocks would leave 52 SMs idle); the
-    counts agree with the ncu launch lists of these workloads."""
+    gather (not for bf16 batches of at most 64 tokens, whose gate_up reads x in
+    place), gate_up, down, combine, plus a reduction per GEMM whose K is split.
+    Decode T=1 splits gate_up only (96 tiles of 64 k-blocks would leave 52 SMs idle)."""
     from workloads import CONFIGS
     cfg = CONFIGS[name]
     assert moe.moe_forward_kernel_count(moe.shape_of(cfg), moe.options_of(cfg)) == count
@@ -189,7 +200,7 @@ def test_split_k_choice_follows_the_cost_model(moe):
     -> 8 splits (cost 8 against 18).  T=65 (two sort chunks): gate_up 64 tiles -> 2
     splits (cost 38; 4 splits cost 40), down 128 tiles -> no split (18 against 24)."""
     o = moe.make_options()
-    assert moe.moe_forward_kernel_count(moe.make_shape(T=1, d=4096, F=1024, E=8, k=1), o) == 6 + 2
+    assert moe.moe_forward_kernel_count(moe.make_shape(T=1, d=4096, F=1024, E=8, k=1), o) == 5 + 2
     assert moe.moe_forward_kernel_count(moe.make_shape(T=65, d=4096, F=1024, E=8, k=1), o) == 8 + 1
     # fp32 problems run the SIMT GEMMs, which never split K
     f32 = moe.make_shape(T=1, d=4096, F=1024, E=8, k=1, act_dtype="f32", w_dtype="f32", logit_dtype="f32")

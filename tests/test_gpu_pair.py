@@ -31,6 +31,9 @@ CASES = {
     "pair_many_experts": small(MIX, name="pair_many_experts", E=64, k=8, T=200, d=256, F=256),
     "pair_skewed_top1": small(MIX, name="pair_skewed_top1", T=1024, d=512, F=256, E=2, k=1,
                               logits="zipf"),
+    # the unfused gate stack and the plain (non-gated) FFN ("MoE" graph-op fc3 / fusion_size 1)
+    "pair_unfused": small(DSK, name="pair_unfused", gu_layout="unfused", expert_bias=True, shared_gate=True),
+    "pair_plain": small(DSK, name="pair_plain", ffn="plain", act="gelu_erf", expert_bias=True, F=328),
 }
 
 
