@@ -629,7 +629,11 @@ def run_own(args, cfg):
         for name, ocfg in CONFIGS.items():
             if name == cfg.name:
                 continue
-            others[name] = measure_workload(ocfg, args.other_steps, 3, flush, stream)
+            try:
+                others[name] = measure_workload(ocfg, args.other_steps, 3, flush, stream)
+            except Exception as exc:  # report it on the line; the default workload's figures stand
+                others[name] = {"workload": workload_name(ocfg), "error": f"{type(exc).__name__}: {exc}"}
+            torch.cuda.synchronize()
             torch.cuda.empty_cache()
         out["other_workloads"] = others
         out["other_workloads_clocks"] = sampler2.stop()

@@ -220,6 +220,7 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
   sa.off = at<int32_t>(ws, p.o_off);
   sa.tile_gu = at<int32_t>(ws, p.o_tgu);
   sa.tile_dn = at<int32_t>(ws, p.o_tdn);
+  sa.order = p.interleave ? at<int32_t>(ws, p.o_ord) : nullptr;
   sa.bm = p.bm;
   sa.nt_gu_routed = p.nt_gu_routed;
   sa.nt_gu_shared = p.nt_gu_shared;
@@ -248,6 +249,7 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
   gc.T = (int)p.T;
   gc.cnt = sa.cnt;
   gc.off = sa.off;
+  gc.order = sa.order;
   gc.d = (int)p.d;
   gc.F = (int)p.F;
   gc.Fs = (int)p.Fs;
@@ -383,13 +385,15 @@ bool pdl_enabled() {
   return on;
 }
 
-// MXFP4 GEMMs on CTA pairs when every expert holds on average a tile's worth of rows
-// (128); MOE_B200_PAIR_FP4=0 or 1 overrides the choice.
+// MXFP4 GEMMs on CTA pairs only when asked for (MOE_B200_PAIR_FP4=1, and every expert
+// holds on average a tile's worth of rows, 128): measured slower than one CTA on the
+// gpt-oss-shaped layer.
 bool use_pair_fp4(int64_t R, int64_t E) {
   const char* env = std::getenv("MOE_B200_PAIR_FP4");
-  if (env && env[0] == '0') return false;
   if (env && env[0] == '1') return true;
-  return R >= (int64_t)kFp4PairMinRows * E;
+  (void)R;
+  (void)E;
+  return false;
 }
 
 // bf16 GEMMs with swapped operands on CTA pairs for large batches that the
@@ -403,6 +407,15 @@ bool use_swap_gemm(int64_t R, bool pair, int layout) {
   if (env && env[0] == '0') return false;
   if (env && env[0] == '1') return true;
   return !pair;
+}
+
+// The bf16 tensor-core GEMMs visit the experts in expert order; MOE_B200_INTERLEAVE=1
+// makes them visit the experts largest first, alternating with the smallest left
+// (sort.cuh: segment_scan) -- measured no faster (DeepSeek-shaped layer 8.48 vs 8.80
+// ms, decode and Mixtral within noise), so not the default.
+bool interleave_segments() {
+  const char* env = std::getenv("MOE_B200_INTERLEAVE");
+  return env && env[0] == '1';
 }
 
 bool use_pair_gemm(int64_t R, int64_t E) {
@@ -433,6 +446,7 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   p->pair_fp4 = s->w_dtype == MOE_MXFP4 && use_pair_fp4(p->R, s->E);
   p->swap = p->tc && s->w_dtype == MOE_BF16 && use_swap_gemm(p->R, p->pair, o->gu_layout);
   if (p->swap) p->pair = false;
+  p->interleave = p->tc && s->w_dtype == MOE_BF16 && interleave_segments();
   // h features per gate_up tile: a gated tile holds each feature's gate and up
   // rows, a plain one a single row per feature (twice the features)
   const int plain = o->ffn == MOE_FFN_PLAIN ? 2 : 1;
@@ -490,6 +504,7 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   p->o_off = take((p->NS + 1) * 4);
   p->o_tgu = take((p->NS + 1) * 4);
   p->o_tdn = take((p->NS + 1) * 4);
+  p->o_ord = take(p->NS * 4);
   p->o_pos = take(p->R * 4);
   p->o_perm = take(p->R * 4);
   p->o_roww = take(p->R * 4);

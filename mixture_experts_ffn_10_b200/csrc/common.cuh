@@ -44,12 +44,13 @@ struct Plan {
   bool direct_x;      // gate_up reads x in place (small batches, single-CTA bf16 GEMMs)
   bool pair_fp4;      // MXFP4 GEMMs on CTA pairs (256 weight rows over two SMs)
   bool swap;          // bf16 GEMMs on CTA pairs with the weights as M (256 weight rows x <= 256 tokens)
+  bool interleave;    // bf16 GEMMs visit the experts in interleaved order (sort.cuh: segment_scan)
   int bm;             // GEMM tile rows
   int nt_gu_routed, nt_gu_shared, nt_dn_routed, nt_dn_shared;  // N tiles per segment
   int splits_gu, splits_dn;  // split-K factors of the two GEMMs (1 = none)
   int64_t partial_pitch;     // floats per row of the split-K partial buffer
   // byte offsets into the workspace
-  size_t o_status, o_idx, o_w, o_hist, o_cnt, o_off, o_tgu, o_tdn, o_pos, o_perm, o_roww,
+  size_t o_status, o_idx, o_w, o_hist, o_cnt, o_off, o_tgu, o_tdn, o_ord, o_pos, o_perm, o_roww,
       o_sgate, o_x, o_h, o_y, o_part, total;
 };
 
@@ -171,8 +172,9 @@ struct SortArgs {
   int32_t* hist;        // [nchunks, E]
   int32_t* cnt;         // [NS]
   int32_t* off;         // [NS + 1]
-  int32_t* tile_gu;     // [NS + 1]
+  int32_t* tile_gu;     // [NS + 1] (by visiting position when order is set)
   int32_t* tile_dn;     // [NS + 1]
+  int32_t* order;       // [NS] segment visited at each position, or null (segment order)
   int bm, nt_gu_routed, nt_gu_shared, nt_dn_routed, nt_dn_shared;
   int32_t* pos;         // [T, k] -> row
   int32_t* perm;        // [R] row -> token
@@ -207,7 +209,8 @@ struct GemmCommon {
   int NS, E, R, T;
   const int32_t* cnt;       // [NS]
   const int32_t* off;       // [NS + 1]
-  const int32_t* tiles;     // [NS + 1] tile prefix for this GEMM
+  const int32_t* tiles;     // [NS + 1] tile prefix for this GEMM (by visiting position)
+  const int32_t* order;     // [NS] segment at each visiting position, or null (identity)
   int max_tiles;            // host upper bound of tiles[NS] - tiles[seg_begin]
   int seg_begin;            // CTA-pair bf16 kernel: walk segments seg_begin .. NS-1 only (else 0)
   int d, F, Fs, Fmax;

@@ -19,13 +19,15 @@
 // Warp roles:
 //   warp 0      TMA producer of activations 256 x 64 (bf16, 128B swizzle)
 //   warp 1      TMEM owner and MMA issuer (M=128 N<=256 K=16)
-//   warp 26     TMA producer of the codes, 128 x 32 bytes, running up to 6 stages ahead
+//   warp 13     TMA producer of the codes, 128 x 32 bytes, running up to 6 stages ahead
 //   warps 2-9   epilogue: two warps per TMEM lane quadrant, alternate 16-token chunks;
 //               for gate_up, weight rows 2j and 2j+1 are the gate and up rows of one
 //               feature, so neighbouring lanes pair up with one shuffle
-//   warps 10-25 converters in four groups, group g owning stages it % 4 == g:
-//               codes + scale -> bf16 in the 128B-swizzled K-major layout the MMA
-//               descriptor reads (mxfp4.cuh), then a proxy fence and one arrive per warp.
+//   warps 10-24 except 13, 17, 21: converters in three groups of four, group g
+//               owning stages it % 3 == g: codes + scale -> bf16 in the 128B-swizzled
+//               K-major layout the MMA descriptor reads (mxfp4.cuh), then a proxy
+//               fence and one arrive per warp.  None shares the MMA issuer's
+//               scheduler (warp w issues on scheduler w % 4); warps 17 and 21 idle.
 #include "epilogue.cuh"
 #include "mxfp4.cuh"
 #include "sm100.cuh"
@@ -43,7 +45,7 @@ constexpr int BNB = 128;                // weight rows per tile
 // Three rings, so that decoding never holds an activation slot:
 constexpr int AST = 4;                  // activations: 256 x 64 bf16, freed by the MMA
 constexpr int QST = 6;                  // e2m1 codes: 128 x 32 bytes, freed once converted
-constexpr int WST = 4;                  // decoded bf16 weights: 128 x 64, freed by the MMA
+constexpr int WST = 3;                  // decoded bf16 weights: 128 x 64, freed by the MMA
 constexpr int A_BYTES = BM * BK * 2;    // 32 KiB
 constexpr int Q_BYTES = BNB * BK / 2;   // 4 KiB
 constexpr int W_BYTES = BNB * BK * 2;   // 16 KiB
@@ -52,13 +54,23 @@ constexpr int ACC_COLS = BM;            // one column per activation row
 constexpr int TMEM_COLS = 2 * ACC_COLS; // double-buffered
 constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, alternate token chunks
 constexpr int kEpiGroups = kEpiWarps / 4;
-constexpr int kCvtWarps = 16;
-constexpr int kCvtGroups = 4;                // converter groups, each owning every 4th stage
+constexpr int kCvtWarps = 12;
+constexpr int kCvtGroups = 3;                // converter groups, each owning every 3rd stage
 constexpr int kCvtGroupWarps = kCvtWarps / kCvtGroups;
-constexpr int kThreads = 64 + (kEpiWarps + kCvtWarps + 1) * 32;  // + the codes producer warp
+// Warps 0 .. 24.  Warp w runs on the SM's scheduler w % 4; the MMA issuer (warp 1)
+// shares its scheduler only with warps that issue few instructions (two epilogue
+// warps and the code producer), never with a converter, so that its MMAs issue on
+// time: converters are the warps 10 .. 24 other than 13, 17 and 21.
+constexpr int kWarps = 25;
+constexpr int kThreads = kWarps * 32;
+constexpr int kCodesWarp = 13;
+__host__ __device__ constexpr int converter_index(int w) {  // -1: not a converter
+  return (w < 10 || w >= kWarps || w % 4 == 1) ? -1 : w - 10 - (w > 13) - (w > 17) - (w > 21);
+}
 constexpr int SMEM_BYTES = RING_BYTES + 1024 + 512;
 static_assert(kCvtGroupWarps * 32 == BNB, "one converter thread per weight row in a group");
 static_assert(WST % kCvtGroups == 0, "a group's stages map to its own decoded-weight slots");
+static_assert(converter_index(24) == kCvtWarps - 1, "twelve converter warps");
 
 struct Fp4Params {
   GemmCommon c;
@@ -127,7 +139,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const GemmCommon& c = p.c;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kCodesWarp = 2 + kEpiWarps + kCvtWarps;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < AST; s++) {
@@ -334,14 +345,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
-  } else if (warp < kCodesWarp) {
+  } else if (converter_index(warp) >= 0) {
     // ------------------------------------------------------------ converters
     // Four groups of four warps; group g converts the stages it with it % 4 == g,
     // so four stages are in conversion at once.  In a group, thread = weight row:
     // it loads the row's 32 code bytes, decodes 64 elements with the row's two
     // block scales and writes the 128-byte row in the swizzled layout (the 8
     // consecutive rows of a quarter-warp hit distinct banks).
-    const int cw = warp - 2 - kEpiWarps;         // 0 .. kCvtWarps-1
+    const int cw = converter_index(warp);        // 0 .. kCvtWarps-1
     const int group = cw / kCvtGroupWarps;       // 0 .. kCvtGroups-1
     const int r = (cw % kCvtGroupWarps) * 32 + lane;  // weight row inside the tile
     const int kblocks = K / 32;                  // scale bytes per weight row

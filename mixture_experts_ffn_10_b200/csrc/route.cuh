@@ -18,42 +18,10 @@
 namespace moe {
 namespace routing {
 
-struct Cand {
-  double key;
-  int idx;  // -1 = none
-  double s;
-};
-
-// a outranks b: larger key, NaN below every number, then the lower index; -1 = none.
-__device__ __forceinline__ bool outranks(double ka, int ia, double kb, int ib) {
-  if (ib < 0) return ia >= 0;
-  if (ia < 0) return false;
-  const bool na = isnan(ka), nb = isnan(kb);
-  if (na || nb) return (na && nb) ? ia < ib : nb;
-  if (ka != kb) return ka > kb;
-  return ia < ib;
-}
-
-__device__ __forceinline__ Cand shfl_cand(const Cand& c, int src_lane_xor) {
-  Cand o;
-  o.key = __shfl_xor_sync(0xffffffffu, c.key, src_lane_xor);
-  o.idx = __shfl_xor_sync(0xffffffffu, c.idx, src_lane_xor);
-  o.s = __shfl_xor_sync(0xffffffffu, c.s, src_lane_xor);
-  return o;
-}
-
-__device__ __forceinline__ Cand warp_best(Cand c) {
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) {
-    Cand o = shfl_cand(c, m);
-    if (outranks(o.key, o.idx, c.key, c.idx)) c = o;
-  }
-  return c;
-}
-
-// Order-preserving 64-bit image of a key for the top-k: larger keys map to larger
-// integers, NaN to 0 (below every number), -0 to the image of +0 (so equal keys,
-// +-0 included, fall to the index tie-break as in outranks()).
+// Order-preserving 64-bit image of a key: larger keys map to larger integers, NaN to
+// 0 (below every number), -0 to the image of +0.  Experts (and groups) rank by image,
+// larger first, equal images to the lower index (ahead()): the order the oracle
+// defines on the keys themselves.
 __device__ __forceinline__ uint64_t ord_key(double k) {
   if (isnan(k)) return 0ull;
   if (k == 0.0) k = 0.0;
@@ -70,6 +38,24 @@ __device__ __forceinline__ bool ahead(uint64_t ka, int ia, uint64_t kb, int ib) 
 
 __device__ __forceinline__ float load_logit(const void* p, int bf16, int64_t i) {
   return bf16 ? bf16_to_f32(((const uint16_t*)p)[i]) : ((const float*)p)[i];
+}
+
+// The key whose image is k (ord_key inverted; NaN comes back as a NaN, -0 as +0).
+__device__ __forceinline__ double key_of_image(uint64_t k) {
+  const uint64_t b = (k >> 63) ? (k & 0x7fffffffffffffffull) : ~k;
+  return __longlong_as_double((long long)b);
+}
+
+// Warp arg-best over (image, expert) candidates, one per lane (kNone = none): the
+// largest image, then the lowest index, in three single-instruction warp reductions.
+// Returns the best image; *winner = its index (kNone if every lane offered none).
+__device__ __forceinline__ uint64_t warp_argbest(uint64_t k, int idx, int* winner) {
+  const uint32_t hi = (uint32_t)(k >> 32), lo = (uint32_t)k;
+  const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+  const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
+  const uint32_t cand = (hi == mhi && lo == mlo) ? (uint32_t)idx : (uint32_t)kNone;
+  *winner = (int)__reduce_min_sync(0xffffffffu, cand);
+  return ((uint64_t)mhi << 32) | mlo;
 }
 
 // Routes token t with the calling warp (lane = this thread's lane).  The token's
@@ -137,45 +123,53 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, int t, int lane,
     per = E / a.n_group;
     double my_gscore = 0.0;
     for (int g = 0; g < a.n_group; g++) {
-      // lane-local best two of group g, then a warp merge of the pairs
-      Cand b1{0.0, -1, 0.0}, b2{0.0, -1, 0.0};
+      // lane-local best two of group g on the key images, then the warp's best and
+      // second best by single-instruction warp reductions
+      uint64_t k1 = 0ull, k2 = 0ull;
+      int i1 = kNone, i2 = kNone;
 #pragma unroll
       for (int i = 0; i < EPL; i++) {
         const int e = lane + 32 * i;
         if (e < E && e / per == g) {
-          if (outranks(key[i], e, b1.key, b1.idx)) {
-            b2 = b1;
-            b1 = Cand{key[i], e, 0.0};
-          } else if (outranks(key[i], e, b2.key, b2.idx)) {
-            b2 = Cand{key[i], e, 0.0};
+          const uint64_t ke = ord_key(key[i]);
+          if (ahead(ke, e, k1, i1)) {
+            k2 = k1;
+            i2 = i1;
+            k1 = ke;
+            i1 = e;
+          } else if (ahead(ke, e, k2, i2)) {
+            k2 = ke;
+            i2 = e;
           }
         }
       }
-#pragma unroll
-      for (int m = 16; m >= 1; m >>= 1) {
-        const Cand o1 = shfl_cand(b1, m), o2 = shfl_cand(b2, m);
-        if (outranks(b1.key, b1.idx, o1.key, o1.idx)) {
-          if (outranks(o1.key, o1.idx, b2.key, b2.idx)) b2 = o1;
-        } else {
-          b2 = outranks(b1.key, b1.idx, o2.key, o2.idx) ? b1 : o2;
-          b1 = o1;
-        }
+      int w1;
+      const uint64_t best = warp_argbest(k1, i1, &w1);
+      double gs = key_of_image(best);
+      if (per >= 2) {
+        // the lane that held the winner offers its second best instead
+        const bool had = i1 == w1;
+        int w2;
+        const uint64_t second = warp_argbest(had ? k2 : k1, had ? i2 : i1, &w2);
+        gs = gs + key_of_image(second);
       }
-      const double gs = per >= 2 ? b1.key + b2.key : b1.key;
       if (lane == g) my_gscore = gs;
     }
     kept_groups = 0;
     bool gtaken = false;
+    const uint64_t gk = ord_key(my_gscore);
     for (int r = 0; r < a.topk_group; r++) {
-      Cand c{my_gscore, (lane < a.n_group && !gtaken) ? lane : -1, 0.0};
-      c = warp_best(c);
-      kept_groups |= 1u << c.idx;
-      if (lane == c.idx) gtaken = true;
+      // lane g offers group g until it is kept; other lanes offer the empty candidate
+      const bool offer = lane < a.n_group && !gtaken;
+      int wg;
+      warp_argbest(offer ? gk : 0ull, offer ? lane : kNone, &wg);
+      if (wg != kNone) kept_groups |= 1u << wg;
+      if (lane == wg) gtaken = true;
     }
   }
 
   // ---- top-k: k rounds of a warp arg-best over the eligible, untaken experts,
-  // on the keys' order-preserving integer images (same order as outranks())
+  // on the keys' order-preserving integer images
   uint64_t okey[EPL];
   bool avail[EPL];  // eligible and not yet taken
 #pragma unroll
@@ -197,16 +191,8 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, int t, int lane,
         bi = e;
       }
     }
-    // warp arg-best in three single-instruction warp reductions (same order as
-    // ahead()): the largest high word of the key images, the largest low word among
-    // the lanes holding it, then the lowest expert index among the lanes holding both
-    {
-      const uint32_t hi = (uint32_t)(bk >> 32), lo = (uint32_t)bk;
-      const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
-      const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
-      const uint32_t cand = (hi == mhi && lo == mlo) ? (uint32_t)bi : (uint32_t)kNone;
-      bi = (int)__reduce_min_sync(0xffffffffu, cand);
-    }
+    // warp arg-best in three single-instruction warp reductions (same order as ahead())
+    warp_argbest(bk, bi, &bi);
     // the winner's owner lane marks it taken and hands its score to lane j
     double sv = 0.0;
     const int slot = bi >> 5;

@@ -36,6 +36,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(SortArgs a) {
   __shared__ int32_t cnt[kMaxE + 1];
   __shared__ int32_t tg[kMaxE + 1];
   __shared__ int32_t td[kMaxE + 1];
+  __shared__ int32_t ord[kMaxE + 1];
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t tot;
   pdl_enter();
@@ -49,7 +50,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(SortArgs a) {
     }
     cnt[e] = run;
   }
-  segment_scan<2>(a, cnt, tg, td, warp_tot, &tot);
+  segment_scan<2>(a, cnt, tg, td, warp_tot, &tot, ord);
 }
 
 // The whole sort for a single chunk of tokens (T <= kChunkTokens) in one block:
@@ -59,6 +60,7 @@ __global__ void __launch_bounds__(1024) sort_one_chunk_kernel(SortArgs a) {
   __shared__ int32_t tg[kMaxE + 1];
   __shared__ int32_t td[kMaxE + 1];
   __shared__ int32_t run[kMaxE];
+  __shared__ int32_t ord[kMaxE + 1];
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t tot;
   pdl_enter();
@@ -74,7 +76,7 @@ __global__ void __launch_bounds__(1024) sort_one_chunk_kernel(SortArgs a) {
     else set_status(a.status, MOE_ERR_SHAPE);
   }
   __syncthreads();
-  segment_scan<2>(a, cnt, tg, td, warp_tot, &tot);
+  segment_scan<2>(a, cnt, tg, td, warp_tot, &tot, ord);
   __syncthreads();
   if (threadIdx.x < 32) scatter_chunk(a, 0, n_ent, cnt, nullptr, run);
 }

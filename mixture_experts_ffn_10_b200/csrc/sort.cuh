@@ -53,9 +53,15 @@ __device__ void block_exclusive_scan(int32_t* v, int n, int32_t* total, int32_t*
 // Segment offsets and per-GEMM tile prefixes from the per-expert row counts in
 // cnt[0..E) (shared memory; one block).  Leaves the segments'
 // first rows (exclusive prefix) in cnt.
+//
+// With a.order set, the GEMMs visit the segments in an interleaved order: by rows,
+// the largest first, each followed by the smallest one left (order[p] = segment at
+// position p; the tile prefixes follow the positions).  Tiles of experts with few
+// rows stream their weights from memory while those of large experts keep the
+// tensor cores busy, so that SMs working at the same time mix the two.
 template <int kItems>  // blockDim.x * kItems >= NS
 __device__ void segment_scan(const SortArgs& a, int32_t* cnt, int32_t* tg, int32_t* td, int32_t* warp_tot,
-                             int32_t* tot) {
+                             int32_t* tot, int32_t* ord) {
   if (threadIdx.x == 0 && a.NS > a.E) cnt[a.E] = a.shared_rows;
   __syncthreads();
   for (int s = threadIdx.x; s < a.NS; s += blockDim.x) {
@@ -66,6 +72,39 @@ __device__ void segment_scan(const SortArgs& a, int32_t* cnt, int32_t* tg, int32
     td[s] = mt * (sh ? a.nt_dn_shared : a.nt_dn_routed);
   }
   __syncthreads();
+  if (a.order) {
+    // rank by rows (descending, ties to the lower segment), then interleave the ranks
+    for (int s = threadIdx.x; s < a.NS; s += blockDim.x) {
+      const int32_t cs = cnt[s];
+      int rank = 0;
+      for (int q = 0; q < a.NS; q++) {
+        const int32_t cq = cnt[q];
+        rank += (cq > cs || (cq == cs && q < s)) ? 1 : 0;
+      }
+      const int h = (a.NS + 1) / 2;
+      const int pos = rank < h ? 2 * rank : 2 * (a.NS - 1 - rank) + 1;
+      ord[pos] = s;
+      a.order[pos] = s;
+    }
+    __syncthreads();
+    int32_t g[kItems], dd[kItems];
+#pragma unroll
+    for (int i = 0; i < kItems; i++) {
+      const int pos = threadIdx.x + i * blockDim.x;
+      g[i] = pos < a.NS ? tg[ord[pos]] : 0;
+      dd[i] = pos < a.NS ? td[ord[pos]] : 0;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kItems; i++) {
+      const int pos = threadIdx.x + i * blockDim.x;
+      if (pos < a.NS) {
+        tg[pos] = g[i];
+        td[pos] = dd[i];
+      }
+    }
+    __syncthreads();
+  }
   block_exclusive_scan<kItems>(cnt, a.NS, tot, warp_tot);
   for (int s = threadIdx.x; s < a.NS; s += blockDim.x) a.off[s] = cnt[s];
   if (threadIdx.x == 0) {

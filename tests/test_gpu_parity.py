@@ -307,3 +307,17 @@ def test_every_token_on_the_same_two_experts():
     logits[:, 3] += 4.0
     logits[:, 5] += 3.0
     parity(cfg, override={"logits": logits.to(torch.bfloat16)})
+
+
+@pytest.mark.parametrize("cfg", [DSK, MIX, small(DEC, T=5)], ids=["deepseek", "mixtral", "decode"])
+def test_expert_visiting_order_does_not_change_results(cfg, monkeypatch):
+    """The GEMMs' interleaved expert order (largest first, alternating with the
+    smallest) only reorders independent tiles: results are bitwise those of the
+    expert order."""
+    inputs = make_inputs(cfg, "cuda")
+    monkeypatch.setenv("MOE_B200_INTERLEAVE", "0")
+    y0, i0, _ = run_gpu(cfg, inputs)
+    monkeypatch.setenv("MOE_B200_INTERLEAVE", "1")
+    y1, i1, _ = run_gpu(cfg, inputs)
+    torch.cuda.synchronize()
+    assert torch.equal(i0, i1) and torch.equal(y0, y1)
