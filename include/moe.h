@@ -192,11 +192,19 @@ MOE_API size_t moe_workspace_size(const moe_shape *shape, const moe_options *opt
  * Errors: MOE_ERR_NULL / SHAPE / DTYPE / ALIGN / ARG / UNSUPPORTED / WORKSPACE
  * before any launch; MOE_ERR_CUDA if a launch fails.  T == 0 is a no-op.
  * Results are bitwise reproducible run to run for the same inputs.
- * Kernel choice: with bf16 weights and on average >= 512 routed rows per
- * expert (and T*k > 4096) the GEMMs run on CTA pairs (256-row tiles over two
- * SMs); the environment variable MOE_B200_PAIR_GEMM=0 or =1, read at every
- * call, forces the single-CTA or the pair kernels.  Set it before
- * moe_workspace_size: the two choices may need different workspace sizes.
+ * Kernel choice (environment variables read at every call; set them before
+ * moe_workspace_size, the choices may need different workspace sizes):
+ *   - bf16 weights, T*k > 4096, fused or plain layout: CTA pairs with the weight
+ *     rows as the MMA's M (256 over two SMs) and the token rows as N, padded to 16
+ *     (MOE_B200_SWAP_GEMM=0 turns them off);
+ *   - otherwise bf16: token tiles, on CTA pairs (256 rows over two SMs) when the
+ *     experts average >= 512 routed rows and T*k > 4096, else one CTA per 128-row
+ *     tile, with split-K for small batches (MOE_B200_PAIR_GEMM=0 or =1 forces
+ *     one or the other);
+ *   - MXFP4 weights: one CTA per tile; MOE_B200_PAIR_FP4=1 picks CTA pairs with
+ *     256 decoded weight rows (slower on the shapes measured);
+ *   - MOE_B200_INTERLEAVE=1: the bf16 GEMMs visit the experts largest first,
+ *     alternating with the smallest (results unchanged).
  * Launches: every kernel after the first may be scheduled while its
  * predecessor in the stream still runs (programmatic dependent launch) and
  * waits on the device for the predecessor's results; MOE_B200_PDL=0, read

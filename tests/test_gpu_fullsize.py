@@ -94,10 +94,13 @@ def test_full_size_parity(name):
     _full_size(name)
 
 
-def test_full_size_mixtral_single_cta_gemm(monkeypatch):
-    """The large-batch workload again with the single-CTA GEMMs forced (the library
-    picks the CTA-pair GEMMs for it by default)."""
-    monkeypatch.setenv("MOE_B200_PAIR_GEMM", "0")
+@pytest.mark.parametrize("pair", ["0", "1"], ids=["single_cta", "token_tile_pair"])
+def test_full_size_mixtral_token_tile_gemms(monkeypatch, pair):
+    """The large-batch workload again on the token-tile GEMMs (the library picks the
+    swapped-operand CTA-pair GEMMs for it by default): one CTA per 128-row tile, and
+    CTA pairs per 256-row tile."""
+    monkeypatch.setenv("MOE_B200_SWAP_GEMM", "0")
+    monkeypatch.setenv("MOE_B200_PAIR_GEMM", pair)
     _full_size("mixtral_bf16")
 
 

@@ -39,6 +39,7 @@ CASES = {
 
 @pytest.fixture
 def force_pair(monkeypatch):
+    monkeypatch.setenv("MOE_B200_SWAP_GEMM", "0")
     monkeypatch.setenv("MOE_B200_PAIR_GEMM", "1")
 
 
@@ -54,6 +55,7 @@ def test_pair_and_single_cta_agree(monkeypatch):
     p = oracle.Problem(cfg, host(inputs))
     ref = p.forward()
     errs = {}
+    monkeypatch.setenv("MOE_B200_SWAP_GEMM", "0")
     for flag in ("0", "1"):
         monkeypatch.setenv("MOE_B200_PAIR_GEMM", flag)
         y, _, _ = run_gpu(cfg, inputs)

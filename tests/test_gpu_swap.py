@@ -1,9 +1,8 @@
 """GPU parity of the bf16 GEMMs with swapped operands on CTA pairs (256 weight rows
 over two SMs as the MMA's M, the tile's token rows as its N, padded to 16 only).
 
-The library picks them by itself for batches of more than 4096 routed rows that
-the 256-row token-tile pair kernel does not take (fewer than 512 rows per expert
-on average); MOE_B200_SWAP_GEMM=1 forces them for larger experts too.  Cases span
+The library picks them by itself for batches of more than 4096 routed rows (with
+a fused or plain layout); MOE_B200_SWAP_GEMM=0 turns them off.  Cases span
 token tiles of every height (1 .. 256 rows, the MMA's N split evenly across the
 pair), ragged d and F against the 256-row weight tiles and the 64-deep K step,
 both fused layouts (gate and up rows of a feature adjacent through a feature-outer
