@@ -29,6 +29,7 @@ import argparse
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -41,19 +42,41 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE layer tokens/s; achieved TFLOP/s or HBM GB/s as % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a workload's
-# dominant GEMM, each from one ncu capture of that kernel, keyed with the hash of the CUDA
-# sources the captured library was built from (kernel_sources_hash).  A figure whose hash
-# is not the current sources' belongs to an older kernel and is reported as null.
-NCU_TRAFFIC = {}
+# dominant GEMM, each from one ncu capture of that kernel, with the kernel's source file and
+# the hash of that file and the headers it includes (kernel_sources_hash) at capture time.
+# A figure whose hash is not the current sources' belongs to an older kernel: reported null.
+#   mixtral_bf16 gate_up: full-size capture, median of two launches (2.7992 GB read + 0.2312
+#     GB written).
+#   deepseek_bf16 gate_up: captured at E=32 T=1024 (same 256 routed rows per expert and one
+#     shared row per token, one eighth of every operand) and scaled by 8: 2.1719 GB read +
+#     0.0373 GB written per launch there.
+#   gptoss_mxfp4 gate_up: full-size capture, 0.3297 GB read + 0.0389 GB written.
+NCU_TRAFFIC = {
+    ("mixtral_bf16", "gate_up"): (3030478336, "gemm_tcs.cu", "c8f80540d88e"),
+    ("deepseek_bf16", "gate_up"): (8 * (2171850000 + 37275392), "gemm_tcs.cu", "c8f80540d88e"),
+    ("gptoss_mxfp4", "gate_up"): (329742592 + 38918400, "gemm_fp4.cu", "667efd3d31dc"),
+}
 
 
-def kernel_sources_hash() -> str:
-    """Short hash of the library's CUDA sources (csrc/*.cu, *.cuh) and its header."""
+def kernel_sources_hash(kernel_file: str = None) -> str:
+    """Short hash of one kernel source file of the library and every local header it
+    includes (transitively, plus include/moe.h); without a file, of all of csrc/."""
     import hashlib
-    h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixture_experts_ffn_10_b200", "csrc")
-    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
-    for f in files + [os.path.join(ROOT, "include", "moe.h")]:
+    if kernel_file is None:
+        files = sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    else:
+        files, todo = [], [kernel_file]
+        while todo:
+            f = todo.pop()
+            if f in files or not os.path.exists(os.path.join(csrc, f)):
+                continue
+            files.append(f)
+            with open(os.path.join(csrc, f)) as fh:
+                todo += re.findall(r'^#include "([^"]+)"', fh.read(), flags=re.M)
+        files.sort()
+    h = hashlib.sha256()
+    for f in [os.path.join(csrc, f) for f in files] + [os.path.join(ROOT, "include", "moe.h")]:
         h.update(os.path.basename(f).encode())
         with open(f, "rb") as fh:
             h.update(fh.read())
@@ -61,12 +84,18 @@ def kernel_sources_hash() -> str:
 
 
 def ncu_traffic(workload: str, stage: str):
-    """ncu DRAM bytes per launch for this workload and stage, or None if not captured
-    for the current sources."""
+    """ncu DRAM bytes per launch for this workload's stage, or None if not captured for the
+    current sources of the kernel that ran it."""
     rec = NCU_TRAFFIC.get((workload, stage))
-    if rec is None or rec[1] != kernel_sources_hash():
+    if rec is None or rec[2] != kernel_sources_hash(rec[1]):
         return None
     return rec[0]
+
+
+def traffic_kernel_sources(workload: str, stage: str):
+    """(kernel file, current hash) of the kernel a traffic figure belongs to, or None."""
+    rec = NCU_TRAFFIC.get((workload, stage))
+    return None if rec is None else {"file": rec[1], "hash": kernel_sources_hash(rec[1])}
 
 
 def peaks():
@@ -568,7 +597,7 @@ def run_own(args, cfg):
                 "frac_vs_sustained_peak": (achieved / sustained) if sustained else None,
                 # the figures belong to the kernels the library picks by itself
                 "traffic": None if os.environ.get("MOE_B200_PAIR_GEMM") else ncu_traffic(cfg.name, dom),
-                "kernel_sources": kernel_sources_hash(),
+                "kernel_sources": traffic_kernel_sources(cfg.name, dom) or kernel_sources_hash(),
                 "algorithmic_per_launch": m["flops"] if bound == "tensor" else m["bytes"],
                 "kernel_ms": dom_ms,
                 "timed": "CUDA events around this stage only (GEMM + split-K reduction), "

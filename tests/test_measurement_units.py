@@ -5,10 +5,14 @@ FLOPs of a forward = 2 * (T*k routed rows) * 3*d*F + 2 * T * 3*d*Fs; bytes = the
 touched experts' weights (+ MXFP4 scales, + expert biases) + shared weights + x,
 logits and y.
 """
+import os
+
 import pytest
 
 import bench
 from workloads import CONFIGS, algorithmic_bytes, flops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 # name: (experts touched, FLOPs, bytes), each worked out by hand:
 HAND = {
@@ -50,3 +54,25 @@ def test_stage_bytes_count_each_weight_once():
     # gate_up reads 2/3 of the weights, the gathered rows (d) and writes h (F); down the rest
     assert m["gate_up"]["bytes"] == 2 * w / 3 + R * (cfg.d + cfg.F) * 2
     assert m["down"]["bytes"] == w / 3 + R * (cfg.F + cfg.d) * 2
+
+
+def test_traffic_figures_follow_their_kernel_sources(monkeypatch):
+    # each stored DRAM figure is reported only while its kernel's sources are unchanged
+    for (wl, st), (nbytes, kfile, h) in bench.NCU_TRAFFIC.items():
+        assert bench.ncu_traffic(wl, st) == (nbytes if h == bench.kernel_sources_hash(kfile) else None)
+    key = ("mixtral_bf16", "gate_up")
+    nbytes, kfile, _ = bench.NCU_TRAFFIC[key]
+    monkeypatch.setitem(bench.NCU_TRAFFIC, key, (nbytes, kfile, "0" * 12))
+    assert bench.ncu_traffic(*key) is None
+    assert bench.ncu_traffic("mixtral_bf16", "combine") is None
+
+
+def test_kernel_hash_covers_included_headers_only():
+    import hashlib
+    csrc = os.path.join(ROOT, "mixture_experts_ffn_10_b200", "csrc")
+    files = ["common.cuh", "epilogue.cuh", "gemm_tcs.cu", "sm100.cuh", "tmap.cuh"]
+    h = hashlib.sha256()
+    for f in [os.path.join(csrc, f) for f in files] + [os.path.join(ROOT, "include", "moe.h")]:
+        h.update(os.path.basename(f).encode())
+        h.update(open(f, "rb").read())
+    assert bench.kernel_sources_hash("gemm_tcs.cu") == h.hexdigest()[:12]
