@@ -167,7 +167,11 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
 cudaError_t launch_sort(const SortArgs& a, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   if (a.nchunks == 1) {  // small batches: one launch instead of three
-    return launch_pdl(sort_one_chunk_kernel, 1, 1024, 0, st, a);
+    // as few threads as the segment scan needs (two segments per thread): its block
+    // barriers are the kernel's latency
+    int threads = ((a.NS + 1) / 2 + 31) / 32 * 32;
+    threads = threads < 128 ? 128 : (threads > 1024 ? 1024 : threads);
+    return launch_pdl(sort_one_chunk_kernel, 1, threads, 0, st, a);
   }
   cudaError_t e = launch_pdl(hist_kernel, (unsigned)a.nchunks, 256, a.E * sizeof(int32_t), st, a);
   if (e == cudaSuccess) e = launch_pdl(scan_kernel, 1, 1024, 0, st, a);
