@@ -9,8 +9,8 @@ Mixtral-shaped bf16 prefill layer (T=4096, d=4096, F=14336, E=8, k=2).
 
 Timing: W warm-up steps, then K steps timed on the device with one CUDA event
 pair per step on the launching stream, each step a replay of a CUDA graph of
-the moe_forward call (--no-graph: eager calls); the L2 is flushed (512 MiB
-write) before every timed step, outside the events.  A second pass of K steps
+the moe_forward call (--no-graph: eager calls); the L2 is flushed (a 512 MiB
+buffer written, then read back) before every timed step, outside the events.  A second pass of K steps
 has the library record an event at every stage boundary (inside the replayed
 graph, so without host launch gaps); it gives the per-kernel times behind the
 roofline figure.
@@ -41,6 +41,25 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer tokens/s; achieved TFLOP/s or HBM GB/s as % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_NOTE = "flushed before every timed step: a 512 MiB buffer written, then read back"
+
+
+class L2Flush:
+    """Evicts the inputs from the 126 MB L2 before a timed step: writes a 512 MiB buffer,
+    then reads it back, so that the L2 holds only clean lines of that buffer (a write
+    alone would leave ~126 MB of dirty lines, whose write-back the timed step would pay
+    for: 13 us of a 82 us decode step)."""
+
+    def __init__(self, torch):
+        self.buf = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+        self.acc = torch.empty((), dtype=torch.int64, device="cuda")
+        self.torch = torch
+
+    def __call__(self):
+        self.buf.zero_()
+        self.torch.sum(self.buf.view(self.torch.int64), 0, out=self.acc)
+
+
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a workload's
 # dominant GEMM, each from one ncu capture of that kernel, with the kernel's source file and
 # the hash of that file and the headers it includes (kernel_sources_hash) at capture time.
@@ -132,7 +151,7 @@ def workload_name(cfg):
 def config_dict(cfg, extra=None):
     d = {"workload": workload_name(cfg), "T": cfg.T, "d": cfg.d, "F": cfg.F, "E": cfg.E, "k": cfg.k,
          "Fs": cfg.Fs, "global_batch": cfg.T, "parallelism": "replicas",
-         "l2": "flushed (512 MiB write) before every timed step"}
+         "l2": L2_NOTE}
     if extra:
         d.update(extra)
     return d
@@ -270,6 +289,17 @@ def stage_model(cfg, distinct):
     }
 
 
+def fuse_stages(model):
+    """The stage model when gate_up and down are one launch: the gate_up stage (events
+    3 .. 4) then spans both GEMMs and the down stage is empty."""
+    both = {k: model["gate_up"][k] + model["down"][k] for k in ("flops", "bytes")}
+    return {"gate_up": both, "down": {"flops": 0.0, "bytes": 0.0}}
+
+
+def stage_label(dom, fused):
+    return "gate_up + down grouped GEMMs (one launch)" if fused else f"{dom} grouped GEMM"
+
+
 def measure_workload(cfg, steps, warmup, flush, stream):
     """Device-timed summary of one more workload (rank-local): CUDA-graph replays of
     moe_forward with the L2 flushed before each, then each GEMM stage alone between
@@ -303,7 +333,7 @@ def measure_workload(cfg, steps, warmup, flush, stream):
 
     with torch.cuda.stream(stream):
         for _ in range(warmup):
-            flush.zero_()
+            flush()
             call()
     torch.cuda.synchronize()
     graphs = [capture()]
@@ -322,13 +352,13 @@ def measure_workload(cfg, steps, warmup, flush, stream):
     stage_ms = {"gate_up": 0.0, "down": 0.0}
     with torch.cuda.stream(stream):
         for i in range(steps):
-            flush.zero_()
+            flush()
             t0s[i].record(stream)
             graphs[0].replay()
             t1s[i].record(stream)
         for gi, st in ((1, "gate_up"), (2, "down")):
             for _ in range(steps):
-                flush.zero_()
+                flush()
                 graphs[gi].replay()
                 torch.cuda.synchronize()
                 stage_ms[st] += stage_ev[st][0].elapsed_time(stage_ev[st][1]) / steps
@@ -341,6 +371,9 @@ def measure_workload(cfg, steps, warmup, flush, stream):
     rows = torch.bincount(idx.flatten().long(), minlength=cfg.E)
     pk, pk_src = peaks()
     model = stage_model(cfg, distinct)
+    fused = moe.moe_forward_fused_gemms(shape, opts) == 1
+    if fused:
+        model = fuse_stages(model)
     dom = max(stage_ms, key=stage_ms.get)
     m, t_dom = model[dom], stage_ms[dom] / 1e3
     tensor = m["flops"] / pk["bf16_tflops"] / 1e12 >= m["bytes"] / pk["hbm_gbs"] / 1e9
@@ -350,7 +383,7 @@ def measure_workload(cfg, steps, warmup, flush, stream):
     del graphs
     return {"workload": workload_name(cfg), "ms_per_step": ms, "tokens_per_s": cfg.T / (ms / 1e3),
             "stage_ms": stage_ms,
-            "roofline": {"kernel": f"{dom} grouped GEMM", "bound": "tensor" if tensor else "hbm",
+            "roofline": {"kernel": stage_label(dom, fused), "bound": "tensor" if tensor else "hbm",
                          "achieved": achieved, "unit": "TFLOP/s" if tensor else "GB/s", "peak": peak,
                          "frac": achieved / peak, "peak_source": f"{pk_src} (burst)",
                          "traffic": ncu_traffic(cfg.name, dom)},
@@ -390,7 +423,7 @@ def run_own(args, cfg):
     y = torch.empty_like(inputs["x"])
     idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
     tens = moe.tensors_of(inputs, y, idx, None)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush(torch)
     nev = moe.MOE_STAGE_EVENTS
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
     for row in events:
@@ -410,7 +443,7 @@ def run_own(args, cfg):
     sampler = ClockSampler(physical_gpu_index(local))
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            flush.zero_()
+            flush()
             step()
     torch.cuda.synchronize()
     status = moe.moe_debug_status(ws.ptr, sptr)
@@ -432,7 +465,7 @@ def run_own(args, cfg):
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             t0s[i].record(stream)
             if graph is not None:
                 graph.replay()
@@ -467,7 +500,7 @@ def run_own(args, cfg):
 
     with torch.cuda.stream(stream):
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             if stage_graph is not None:
                 stage_graph.replay()
                 torch.cuda.synchronize()
@@ -482,7 +515,7 @@ def run_own(args, cfg):
     stage_launch = "cuda graph" if stage_graph is not None else "eager"
 
     # Pass 3 (the roofline's kernel time): the same call with only the two events
-    # around the dominant GEMM stage (GEMM + its split-K reduction, if any), so
+    # around the dominant GEMM stage (its GEMM launch), so
     # that no other event node adds to that stage's time.
     names = list(moe.STAGES)
     dom = max(("gate_up", "down"), key=lambda n: stage_ms[names.index(n)])
@@ -501,7 +534,7 @@ def run_own(args, cfg):
     dom_ms = 0.0
     with torch.cuda.stream(stream):
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             if dom_graph is not None:
                 dom_graph.replay()
             else:
@@ -584,6 +617,9 @@ def run_own(args, cfg):
     rows_per_expert = torch.bincount(idx.flatten().long(), minlength=cfg.E)
     pk, pk_src = peaks()
     model = stage_model(cfg, distinct)
+    fused = moe.moe_forward_fused_gemms(shape, opts) == 1
+    if fused:
+        model = fuse_stages(model)
     t_dom = dom_ms / 1e3
     m = model[dom]
     t_tc, t_hbm = m["flops"] / (pk["bf16_tflops"] * 1e12), m["bytes"] / (pk["hbm_gbs"] * 1e9)
@@ -592,7 +628,7 @@ def run_own(args, cfg):
     else:
         achieved, peak, unit, bound = m["bytes"] / t_dom / 1e9, pk["hbm_gbs"], "GB/s", "hbm"
     sustained = pk["bf16_tflops_sustained"] if bound == "tensor" else None
-    roofline = {"bound": bound, "kernel": f"{dom} grouped GEMM", "achieved": achieved, "peak": peak,
+    roofline = {"bound": bound, "kernel": stage_label(dom, fused), "achieved": achieved, "peak": peak,
                 "unit": unit, "frac": achieved / peak, "peak_source": f"{pk_src} (burst)",
                 "frac_vs_sustained_peak": (achieved / sustained) if sustained else None,
                 # the figures belong to the kernels the library picks by itself
@@ -600,7 +636,7 @@ def run_own(args, cfg):
                 "kernel_sources": traffic_kernel_sources(cfg.name, dom) or kernel_sources_hash(),
                 "algorithmic_per_launch": m["flops"] if bound == "tensor" else m["bytes"],
                 "kernel_ms": dom_ms,
-                "timed": "CUDA events around this stage only (GEMM + split-K reduction), "
+                "timed": "CUDA events around this stage only (its GEMM launch), "
                          + ("graph replay" if dom_graph is not None else "eager calls") + ", L2 flushed"}
     layer_flops = flops(cfg)
     layer_bytes = algorithmic_bytes(cfg, distinct)

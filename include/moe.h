@@ -200,7 +200,9 @@ MOE_API size_t moe_workspace_size(const moe_shape *shape, const moe_options *opt
  *   - otherwise bf16: token tiles, on CTA pairs (256 rows over two SMs) when the
  *     experts average >= 512 routed rows and T*k > 4096, else one CTA per 128-row
  *     tile, with split-K for small batches (MOE_B200_PAIR_GEMM=0 or =1 forces
- *     one or the other);
+ *     one or the other); for T <= 64 gate_up reads x in place and, unless
+ *     MOE_B200_FUSED_FFN=0 or MOE_B200_INTERLEAVE=1, gate_up and down run as one
+ *     launch whose down tiles start once their expert's h rows are complete;
  *   - MXFP4 weights: one CTA per tile; MOE_B200_PAIR_FP4=1 picks CTA pairs with
  *     256 decoded weight rows (slower on the shapes measured);
  *   - MOE_B200_INTERLEAVE=1: the bf16 GEMMs visit the experts largest first,
@@ -229,6 +231,8 @@ MOE_API int moe_route(const moe_shape *shape, const moe_options *opts, const moe
  *   events[1] after routing           events[5] after the down GEMM
  *   events[2] after sort/scan/scatter events[6] after the combine
  *   events[3] after the row gather
+ * (events[4] and events[5] both after the one launch of the two GEMMs when
+ * moe_forward_fused_gemms says they are fused.)
  * n_events <= MOE_STAGE_EVENTS; NULL entries are skipped.  Same results,
  * errors and workspace rules as moe_forward.  Called under stream capture,
  * the events become event-record nodes of the graph and time every replay.
@@ -276,6 +280,19 @@ MOE_API size_t moe_noalloc_workspace_bytes(void);
 /* Number of CUDA kernels one moe_forward of this problem launches (-1 if the
  * arguments are invalid; 0 for T == 0).  For launch accounting. */
 MOE_API int moe_forward_kernel_count(const moe_shape *shape, const moe_options *opts);
+
+/* The split-K factors moe_forward uses for the gate_up and down GEMMs of this
+ * problem (1 = K not split; more only for bf16 batches of at most 4096 routed rows
+ * on the single-CTA GEMMs, when the tiles alone would leave SMs idle).  Returns
+ * MOE_OK or the argument error of moe_forward. */
+MOE_API int moe_forward_split_k(const moe_shape *shape, const moe_options *opts, int *splits_gate_up,
+                                int *splits_down);
+
+/* 1 if moe_forward of this problem runs gate_up and down as one kernel launch
+ * (batches of at most 64 tokens with bf16 weights; MOE_B200_FUSED_FFN=0 turns it
+ * off), 0 if not, -1 if the arguments are invalid.  Stage events 4 and 5 are then
+ * both recorded after that launch. */
+MOE_API int moe_forward_fused_gemms(const moe_shape *shape, const moe_options *opts);
 
 /* Message of the last failed call on this thread ("" if none). */
 MOE_API const char *moe_last_error(void);

@@ -86,6 +86,10 @@ def _bind(lib: C.CDLL) -> C.CDLL:
     lib.moe_noalloc_workspace_bytes.restype = C.c_size_t
     lib.moe_forward_kernel_count.argtypes = [_P(moe_shape), _P(moe_options)]
     lib.moe_forward_kernel_count.restype = C.c_int
+    lib.moe_forward_split_k.argtypes = [_P(moe_shape), _P(moe_options), _P(C.c_int), _P(C.c_int)]
+    lib.moe_forward_split_k.restype = C.c_int
+    lib.moe_forward_fused_gemms.argtypes = [_P(moe_shape), _P(moe_options)]
+    lib.moe_forward_fused_gemms.restype = C.c_int
     lib.moe_last_error.argtypes = []
     lib.moe_last_error.restype = C.c_char_p
     lib.moe_debug_status.argtypes = [C.c_void_p, C.c_void_p]
@@ -96,26 +100,35 @@ def _bind(lib: C.CDLL) -> C.CDLL:
 
 
 class _UnbuiltLibrary:
-    """Stands in for the CUDA library until it exists.  The package stays importable
-    without it, so that its build step can run; every entry point then loads the
-    library on first use and raises ImportError while it has not been built.  There
-    is no fallback: nothing here computes without the CUDA library."""
+    """Stands in for the CUDA library until its first use.  The package imports
+    without loading it, so that its build step can run (and replace a library built
+    from older sources); the first entry point called loads and binds it, raising
+    ImportError while it is missing or lacks an entry point of these bindings.
+    There is no fallback: nothing here computes without the CUDA library."""
 
     def __getattr__(self, name):
         global _lib
         if not os.path.exists(LIB_PATH):
             raise ImportError(f"{LIB_PATH} is missing: build it with `python "
                               f"{os.path.join(_HERE, 'build.py')}` (nvcc, sm_100a)")
-        _lib = _bind(C.CDLL(LIB_PATH))
+        handle = C.CDLL(LIB_PATH)
+        try:
+            lib = _bind(handle)
+        except AttributeError as e:
+            import _ctypes
+            _ctypes.dlclose(handle._handle)  # a rebuilt library then loads afresh
+            raise ImportError(f"{LIB_PATH} was built from older sources ({e}): rebuild it with "
+                              f"`python {os.path.join(_HERE, 'build.py')}`") from None
+        _lib = lib
         return getattr(_lib, name)
 
 
-_lib = _bind(C.CDLL(LIB_PATH)) if os.path.exists(LIB_PATH) else _UnbuiltLibrary()
+_lib = _UnbuiltLibrary()
 
 EXPORTED = ("moe_options_init", "moe_workspace_size", "moe_forward", "moe_route",
             "moe_forward_events", "moe_forward_noalloc", "moe_noalloc_debug_status",
-            "moe_noalloc_workspace_bytes", "moe_forward_kernel_count",
-            "moe_last_error", "moe_debug_status", "moe_version")
+            "moe_noalloc_workspace_bytes", "moe_forward_kernel_count", "moe_forward_split_k",
+            "moe_forward_fused_gemms", "moe_last_error", "moe_debug_status", "moe_version")
 
 
 class MoeError(RuntimeError):
@@ -170,6 +183,19 @@ def moe_noalloc_workspace_bytes() -> int:
 
 def moe_forward_kernel_count(shape, opts) -> int:
     return _lib.moe_forward_kernel_count(C.byref(shape), C.byref(opts))
+
+
+def moe_forward_split_k(shape, opts):
+    """(gate_up splits, down splits) of the forward's GEMMs; raises MoeError on bad arguments."""
+    sg, sd = C.c_int(0), C.c_int(0)
+    rc = _lib.moe_forward_split_k(C.byref(shape), C.byref(opts), C.byref(sg), C.byref(sd))
+    if rc != 0:
+        raise MoeError(rc, moe_last_error())
+    return sg.value, sd.value
+
+
+def moe_forward_fused_gemms(shape, opts) -> int:
+    return _lib.moe_forward_fused_gemms(C.byref(shape), C.byref(opts))
 
 
 def moe_last_error() -> str:

@@ -229,6 +229,8 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
   sa.pos = at<int32_t>(ws, p.o_pos);
   sa.perm = at<int32_t>(ws, p.o_perm);
   sa.roww = at<float>(ws, p.o_roww);
+  sa.sync = at<int32_t>(ws, p.o_sync);
+  sa.n_sync = (int)p.n_sync;
   sa.status = status;
   if ((e = launch_sort(sa, st)) != cudaSuccess) return cuda_fail(e, "sort kernels");
   if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
@@ -266,16 +268,23 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
   gc.splits = 1;
   gc.partial = at<float>(ws, p.o_part);
   gc.partial_pitch = (int)p.partial_pitch;
-  // Upper bound of the M tiles: every non-empty expert adds at most one partial tile.
   const int64_t mt_routed = p.R / p.bm + std::min<int64_t>(p.E, p.R);
   const int64_t mt_shared = p.Fs > 0 ? cdiv(p.T, p.bm) : 0;
   GemmCommon gu = gc, dn = gc;
   gu.tiles = sa.tile_gu;
   gu.splits = p.splits_gu;
-  gu.max_tiles = (int)(mt_routed * p.nt_gu_routed + mt_shared * p.nt_gu_shared);
+  gu.max_tiles = (int)p.max_tiles_gu;
   dn.tiles = sa.tile_dn;
   dn.splits = p.splits_dn;
-  dn.max_tiles = (int)(mt_routed * p.nt_dn_routed + mt_shared * p.nt_dn_shared);
+  dn.max_tiles = (int)p.max_tiles_dn;
+  // the sort cleared these counters: split-K arrivals of gate_up, of down, then the
+  // finished h regions per segment of the fused launch
+  int32_t* sync = at<int32_t>(ws, p.o_sync);
+  gu.fix = p.splits_gu > 1 ? sync : nullptr;
+  if (p.splits_gu > 1) sync += p.max_tiles_gu * kFixRegions;
+  dn.fix = p.splits_dn > 1 ? sync : nullptr;
+  if (p.splits_dn > 1) sync += p.max_tiles_dn * kFixRegions;
+  int32_t* ready = p.fused_ffn ? sync : nullptr;
 
   if (p.tc) {
     TcArgs ta{};
@@ -308,33 +317,35 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
       gu_shared.max_tiles = (int)(mt_shared * p.nt_gu_shared);
     }
     ta.c = fp4 ? gu_routed : gu;
-    e = fp4 ? (p.pair_fp4 ? launch_fp4p_gate_up(ta, st) : launch_fp4_gate_up(ta, st))
-            : p.swap ? launch_tcs_gate_up(ta, st) : p.pair ? launch_tc2_gate_up(ta, st) : launch_tc_gate_up(ta, st);
-    if (e != cudaSuccess) return cuda_fail(e, "tensor-core gate_up GEMM");
-    if (fp4 && p.Fs > 0) {
-      ta.c = gu_shared;
-      if ((e = launch_tc2_gate_up(ta, st)) != cudaSuccess) return cuda_fail(e, "shared expert gate_up GEMM");
+    if (p.fused_ffn) {
+      // gate_up and down in one launch: stage event 4 goes with event 5, after it
+      if ((e = launch_tc_ffn(ta, dn, ready, st)) != cudaSuccess) return cuda_fail(e, "fused gate_up + down GEMMs");
+      if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    } else {
+      e = fp4 ? (p.pair_fp4 ? launch_fp4p_gate_up(ta, st) : launch_fp4_gate_up(ta, st))
+              : p.swap ? launch_tcs_gate_up(ta, st) : p.pair ? launch_tc2_gate_up(ta, st) : launch_tc_gate_up(ta, st);
+      if (e != cudaSuccess) return cuda_fail(e, "tensor-core gate_up GEMM");
+      if (fp4 && p.Fs > 0) {
+        ta.c = gu_shared;
+        if ((e = launch_tc2_gate_up(ta, st)) != cudaSuccess) return cuda_fail(e, "shared expert gate_up GEMM");
+      }
+      if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+      GemmCommon dn_routed = dn, dn_shared = dn;
+      if (fp4 && p.Fs > 0) {
+        dn_routed.NS = (int)p.E;
+        dn_routed.max_tiles = (int)(mt_routed * p.nt_dn_routed);
+        dn_shared.seg_begin = (int)p.E;
+        dn_shared.max_tiles = (int)(mt_shared * p.nt_dn_shared);
+      }
+      ta.c = fp4 ? dn_routed : dn;
+      e = fp4 ? (p.pair_fp4 ? launch_fp4p_down(ta, st) : launch_fp4_down(ta, st))
+              : p.swap ? launch_tcs_down(ta, st) : p.pair ? launch_tc2_down(ta, st) : launch_tc_down(ta, st);
+      if (e != cudaSuccess) return cuda_fail(e, "tensor-core down GEMM");
+      if (fp4 && p.Fs > 0) {
+        ta.c = dn_shared;
+        if ((e = launch_tc2_down(ta, st)) != cudaSuccess) return cuda_fail(e, "shared expert down GEMM");
+      }
     }
-    if (gu.splits > 1 && (e = launch_splitk_gate_up_reduce(ta, st)) != cudaSuccess)
-      return cuda_fail(e, "split-K gate_up reduction");
-    if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    GemmCommon dn_routed = dn, dn_shared = dn;
-    if (fp4 && p.Fs > 0) {
-      dn_routed.NS = (int)p.E;
-      dn_routed.max_tiles = (int)(mt_routed * p.nt_dn_routed);
-      dn_shared.seg_begin = (int)p.E;
-      dn_shared.max_tiles = (int)(mt_shared * p.nt_dn_shared);
-    }
-    ta.c = fp4 ? dn_routed : dn;
-    e = fp4 ? (p.pair_fp4 ? launch_fp4p_down(ta, st) : launch_fp4_down(ta, st))
-            : p.swap ? launch_tcs_down(ta, st) : p.pair ? launch_tc2_down(ta, st) : launch_tc_down(ta, st);
-    if (e != cudaSuccess) return cuda_fail(e, "tensor-core down GEMM");
-    if (fp4 && p.Fs > 0) {
-      ta.c = dn_shared;
-      if ((e = launch_tc2_down(ta, st)) != cudaSuccess) return cuda_fail(e, "shared expert down GEMM");
-    }
-    if (dn.splits > 1 && (e = launch_splitk_down_reduce(ta, st)) != cudaSuccess)
-      return cuda_fail(e, "split-K down reduction");
   } else {
     SimtArgs sm{};
     sm.x = (const float*)t->x;
@@ -418,6 +429,14 @@ bool interleave_segments() {
   return env && env[0] == '1';
 }
 
+// Small batches that read x in place run gate_up and down as one launch (the down
+// phase's weight loads start while the last h tiles are written);
+// MOE_B200_FUSED_FFN=0 launches them separately.
+bool use_fused_ffn() {
+  const char* env = std::getenv("MOE_B200_FUSED_FFN");
+  return !(env && env[0] == '0');
+}
+
 bool use_pair_gemm(int64_t R, int64_t E) {
   const char* env = std::getenv("MOE_B200_PAIR_GEMM");
   if (env && env[0] == '0') return false;
@@ -489,6 +508,15 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
     if (p->splits_gu > 1 || p->splits_dn > 1)
       p->partial_pitch = (int64_t)std::max({p->nt_gu_routed, p->nt_gu_shared, p->nt_dn_routed}) * 256;
   }
+  // Upper bounds of the GEMMs' tile counts: every non-empty expert adds at most one
+  // partial M tile.
+  const int64_t mt_routed = p->R / p->bm + std::min<int64_t>(p->E, p->R);
+  const int64_t mt_shared = p->Fs > 0 ? cdiv(p->T, p->bm) : 0;
+  p->max_tiles_gu = mt_routed * p->nt_gu_routed + mt_shared * p->nt_gu_shared;
+  p->max_tiles_dn = mt_routed * p->nt_dn_routed + mt_shared * p->nt_dn_shared;
+  p->fused_ffn = p->direct_x && !p->interleave && use_fused_ffn();
+  p->n_sync = (p->splits_gu > 1 ? p->max_tiles_gu * kFixRegions : 0) +
+              (p->splits_dn > 1 ? p->max_tiles_dn * kFixRegions : 0) + (p->fused_ffn ? p->NS : 0);
   const size_t elt = p->tc ? 2 : 4;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -514,6 +542,7 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   p->o_y = take(p->rows * p->d * elt);
   p->o_part = take((size_t)std::max(p->splits_gu, p->splits_dn) * p->rows * p->partial_pitch * 4 *
                    (p->partial_pitch > 0 ? 1 : 0));
+  p->o_sync = take(p->n_sync * 4);
   p->total = off;
   return off;
 }
@@ -560,10 +589,29 @@ int moe_forward_kernel_count(const moe_shape* s, const moe_options* o) {
   if (s->T == 0) return 0;
   moe::Plan p;
   moe::make_plan(s, o, &p);
-  // route, histogram, scan, scatter, gather (not for direct_x), gate_up, down, combine
-  // (+ split-K reductions); a single 64-token chunk sorts in one kernel
-  return (p.nchunks == 1 ? 4 : 6) + (p.direct_x ? 0 : 1) + 1 + (p.splits_gu > 1) + (p.splits_dn > 1) +
+  // route, histogram, scan, scatter, gather (not for direct_x), gate_up, down (one
+  // launch with gate_up when fused), combine; a single 64-token chunk sorts in one kernel
+  return (p.nchunks == 1 ? 4 : 6) + (p.direct_x ? 0 : 1) + 1 - (p.fused_ffn ? 1 : 0) +
          (s->w_dtype == MOE_MXFP4 && p.Fs > 0 ? 2 : 0);  // the shared expert beside MXFP4 experts
+}
+
+int moe_forward_split_k(const moe_shape* s, const moe_options* o, int* splits_gate_up, int* splits_down) {
+  if (!splits_gate_up || !splits_down) return moe::fail(MOE_ERR_NULL, "split outputs must not be NULL");
+  const int rc = moe::check_shape_opts(s, o);
+  if (rc != MOE_OK) return rc;
+  moe::Plan p;
+  moe::make_plan(s, o, &p);
+  *splits_gate_up = p.splits_gu;
+  *splits_down = p.splits_dn;
+  return MOE_OK;
+}
+
+int moe_forward_fused_gemms(const moe_shape* s, const moe_options* o) {
+  if (moe::check_shape_opts(s, o) != MOE_OK) return -1;
+  if (s->T == 0) return 0;
+  moe::Plan p;
+  moe::make_plan(s, o, &p);
+  return p.fused_ffn ? 1 : 0;
 }
 
 const char* moe_last_error(void) { return moe::g_err.c_str(); }

@@ -22,6 +22,7 @@ constexpr int kPairMinRows = 512; // CTA pairs when routed rows per expert avera
 constexpr int kTcGuBN = 128;      // h features per gate_up tile (gate rows + up rows = 256)
 constexpr int kTcDnBN = 256;      // output features per down tile
 constexpr int kTcBK = 64;         // K elements per pipeline stage of the bf16 tensor-core GEMMs
+constexpr int kFixRegions = 8;      // split-K arrival counters per tile (one per epilogue warp, at most 8)
 constexpr int kSplitMaxRows = 4096;  // split-K only for problems with at most this many routed rows
 constexpr int kDirectMaxTokens = 64; // batches whose gate_up reads x in place (one 64-row A tile)
 
@@ -45,13 +46,16 @@ struct Plan {
   bool pair_fp4;      // MXFP4 GEMMs on CTA pairs (256 weight rows over two SMs)
   bool swap;          // bf16 GEMMs on CTA pairs with the weights as M (256 weight rows x <= 256 tokens)
   bool interleave;    // bf16 GEMMs visit the experts in interleaved order (sort.cuh: segment_scan)
+  bool fused_ffn;     // direct_x: gate_up and down in one launch (launch_tc_ffn)
   int bm;             // GEMM tile rows
   int nt_gu_routed, nt_gu_shared, nt_dn_routed, nt_dn_shared;  // N tiles per segment
   int splits_gu, splits_dn;  // split-K factors of the two GEMMs (1 = none)
   int64_t partial_pitch;     // floats per row of the split-K partial buffer
+  int64_t max_tiles_gu, max_tiles_dn;  // upper bounds of the GEMMs' tile counts
+  int64_t n_sync;            // GEMM counters the sort clears (GemmCommon::fix, ready)
   // byte offsets into the workspace
   size_t o_status, o_idx, o_w, o_hist, o_cnt, o_off, o_tgu, o_tdn, o_ord, o_pos, o_perm, o_roww,
-      o_sgate, o_x, o_h, o_y, o_part, total;
+      o_sgate, o_x, o_h, o_y, o_part, o_sync, total;
 };
 
 // Fills `p` from validated arguments; returns the workspace size.
@@ -179,6 +183,8 @@ struct SortArgs {
   int32_t* pos;         // [T, k] -> row
   int32_t* perm;        // [R] row -> token
   float* roww;          // [R] row -> routing weight
+  int32_t* sync;        // [n_sync] counters of the GEMMs (split-K arrivals, finished h
+  int n_sync;           // regions), set to zero here, before the GEMMs run
   int* status;
 };
 cudaError_t launch_sort(const SortArgs& a, cudaStream_t st);
@@ -230,10 +236,14 @@ struct GemmCommon {
   int* status;
   // split-K: each tile's K range is cut into `splits` parts whose fp32 partial
   // accumulators go to partial[split][row][n_blk * 256 + col] (pitch floats per
-  // row); a reduce kernel then sums them in split order and runs the epilogue.
+  // row).  Each epilogue warp of a tile owns one region of it (its TMEM lane
+  // quadrant, its column chunks) and counts its split done in fix[tile * kFixRegions
+  // + region]; the last of the splits to arrive sums the region's partials in split
+  // order and runs the epilogue.  The counters start at zero (the sort clears them).
   int splits;
   float* partial;
   int partial_pitch;
+  int32_t* fix;
 };
 
 struct SimtArgs {
@@ -282,9 +292,10 @@ cudaError_t launch_tcs_down(const TcArgs& a, cudaStream_t st);
 constexpr int kSwapBM = 256;      // token rows per swapped-operand pair tile (the MMA's N, trimmed)
 cudaError_t launch_tc2_gate_up(const TcArgs& a, cudaStream_t st);  // CTA-pair variants
 cudaError_t launch_tc2_down(const TcArgs& a, cudaStream_t st);
-// Split-K reductions (partials -> epilogue) for the bf16 tensor-core GEMMs.
-cudaError_t launch_splitk_gate_up_reduce(const TcArgs& a, cudaStream_t st);
-cudaError_t launch_splitk_down_reduce(const TcArgs& a, cudaStream_t st);
+// Small batches with x read in place (direct_x): gate_up and down in one launch of the
+// single-CTA kernel.  a.c is the gate_up GEMM, dn the down GEMM; ready [NS] counts the
+// finished h regions of each segment (zero before the launch).
+cudaError_t launch_tc_ffn(const TcArgs& a, const GemmCommon& dn, int32_t* ready, cudaStream_t st);
 // Split count for a GEMM of at most `tiles` tiles of `nkb` k-blocks on `sms` SMs.
 int choose_splits(int64_t tiles, int nkb, int sms);
 // MXFP4 expert stacks (gate_up / down are e2m1 codes), routed segments only (a shared
@@ -326,6 +337,26 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// launch_pdl for a kernel whose CTAs wait on one another: a cooperative launch too,
+// which fails instead of starting when the grid cannot be resident all at once.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_coop_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                   Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 

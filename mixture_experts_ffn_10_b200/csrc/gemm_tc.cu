@@ -57,24 +57,175 @@ constexpr int kThreads = 64 + kEpiWarps * 32;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BNB);
 
 struct TcParams {
-  GemmCommon c;
+  GemmCommon c;                  // gate_up (MODE 0 and 2) or down (MODE 1)
   const uint16_t* gate_up_bias;  // [E, 2F] ([E, F] unfused / plain) or null
   const uint16_t* gate_bias;     // unfused: [E, F] or null
   const uint16_t* down_bias;     // [E, d] or null
   const float* roww;             // [R]
-  uint16_t* out;                 // h [rows, Fmax] or Y [rows, d]
+  uint16_t* out;                 // h [rows, Fmax] (MODE 0 and 2) or Y [rows, d] (MODE 1)
+  GemmCommon c2;                 // MODE 2: the down GEMM of the same forward
+  uint16_t* out2;                // MODE 2: Y [rows, d]
+  int32_t* ready;                // MODE 2: [NS] finished h regions per segment
+};
+
+// A work unit: split sp (of S) of tile `tile` of the gate_up GEMM or (dn) of the down
+// GEMM, K blocks kb0 .. kb1-1.  MODE 2 numbers the gate_up units first, then the
+// down units (u1 = the number of gate_up units).
+struct Unit {
+  Tile t;
+  int tile, sp, S, kb0, kb1;
+  bool dn;
 };
 
 template <int MODE>
-__device__ __forceinline__ int k_extent(const GemmCommon& c, bool shared) {
-  return MODE == 0 ? c.d : (shared ? c.Fs : c.F);
+__device__ __forceinline__ Unit unit_of(const TcParams& p, int unit, int u1) {
+  Unit u;
+  u.dn = MODE == 1 || (MODE == 2 && unit >= u1);
+  const GemmCommon& c = (MODE == 2 && u.dn) ? p.c2 : p.c;
+  const int local = (MODE == 2 && u.dn) ? unit - u1 : unit;
+  u.S = c.splits;
+  u.tile = local / u.S;
+  u.sp = local % u.S;
+  u.t = decode_tile<BM>(c, u.tile);
+  const bool sh = u.t.seg >= c.E;
+  const int K = u.dn ? (sh ? c.Fs : c.F) : c.d;
+  const int nkb = (K + BK - 1) / BK;
+  u.kb0 = u.sp * nkb / u.S;
+  u.kb1 = (u.sp + 1) * nkb / u.S;
+  return u;
 }
 
+// h regions (one per epilogue warp and gate_up tile) of segment `seg` that the MODE 2
+// down tiles of the segment wait for (the segment's tiles are visited in segment order).
+__device__ __forceinline__ int h_regions(const GemmCommon& gu, int seg) {
+  return (gu.tiles[seg + 1] - gu.tiles[seg]) * kEpiWarps;
+}
+
+// Bounded wait until *ctr >= need.  On a timeout it records MOE_ERR_TIMEOUT and
+// returns: the h rows then read are not final, and the forward reports the error.
+__device__ __forceinline__ void wait_count(const int32_t* ctr, int need, int* status) {
+  if (ld_acquire_gpu(ctr) >= need) return;
+  const uint64_t t0 = global_timer();
+  while (ld_acquire_gpu(ctr) < need) {
+    if (global_timer() - t0 > kTimeoutNs) {
+      set_status(status, MOE_ERR_TIMEOUT);
+      return;
+    }
+    __nanosleep(64);
+  }
+}
+
+// Whole warp: counts this warp's split of a region done (after its partial stores);
+// true in every lane for the last of the S splits, which then sees all partials.
+__device__ __forceinline__ bool split_arrive(int32_t* ctr, int S, int lane) {
+  __threadfence();
+  __syncwarp();
+  int old = 0;
+  if (lane == 0) old = atomicAdd(ctr, 1);
+  old = __shfl_sync(0xffffffffu, old, 0);
+  if (old != S - 1) return false;
+  __threadfence();
+  return true;
+}
+
+// Whole warp: publishes this warp's finished h region (after its stores) to the
+// MODE 2 down tiles, whose h loads go through the async proxy.
+__device__ __forceinline__ void signal_region(int32_t* ctr, int lane) {
+  __threadfence();
+  fence_proxy_async_all();
+  __syncwarp();
+  if (lane == 0) atomicAdd(ctr, 1);
+}
+
+// 16 accumulator columns of one row summed over the S (<= 8) split partials in split
+// order, as fp32 bits; the loads of four splits at a time are issued before their sums
+// (not inlined: the gate and up sums of a chunk then do not hold their loads at once).
+__device__ __noinline__ void sum_splits(const float* row, int64_t split_stride, int S, uint32_t (&v)[16]) {
+  float a[16];
+#pragma unroll
+  for (int i = 0; i < 16; i++) a[i] = 0.f;
+#pragma unroll 1
+  for (int s0 = 0; s0 < S; s0 += 4) {
+    float4 q[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; j++)
+      if (s0 + j < S) {
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+          q[j][i] = __ldcg(reinterpret_cast<const float4*>(row + (s0 + j) * split_stride) + i);
+      }
+#pragma unroll
+    for (int j = 0; j < 4; j++)
+      if (s0 + j < S) {
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+          a[4 * i] += q[j][i].x;
+          a[4 * i + 1] += q[j][i].y;
+          a[4 * i + 2] += q[j][i].z;
+          a[4 * i + 3] += q[j][i].w;
+        }
+      }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; i++) v[i] = __float_as_uint(a[i]);
+}
+
+// Column chunks of a tile's accumulator row: a gated gate_up chunk ch is gate columns
+// 16ch .. 16ch+15 with their up partners 128 columns on (8 chunks); plain gate_up and
+// down chunks are 16 columns each (16 chunks).
+__device__ __forceinline__ int chunks_of(const GemmCommon& c, bool dn) {
+  return (!dn && c.ffn != MOE_FFN_PLAIN) ? (BNB / 2) / 16 : BNB / 16;
+}
+
+// The epilogue of chunk ch of one accumulator row (output row grow, weigh-inputs
+// scale wi), stored if `store`; fetch(col, v) yields columns col .. col+15 of the row
+// (called whether or not the chunk is stored: TMEM loads are whole-warp).
+template <typename Fetch>
+__device__ __forceinline__ void emit_chunk(const TcParams& p, const GemmCommon& c, bool dn, uint16_t* out,
+                                           const Tile& t, bool store, int64_t grow, float wi, int ch,
+                                           Fetch&& fetch) {
+  const bool sh = t.seg >= c.E;
+  if (!dn && c.ffn == MOE_FFN_PLAIN) {
+    const int F = sh ? c.Fs : c.F;
+    const uint16_t* bias = (!sh && p.gate_up_bias) ? p.gate_up_bias + (int64_t)t.seg * c.F : nullptr;
+    uint32_t v[16];
+    fetch(ch * 16, v);
+    const int fb = t.n_blk * BNB + ch * 16;
+    if (store && fb < F) plain_chunk(v, bias, fb, F, c.act, wi, out + grow * c.Fmax);
+  } else if (!dn) {
+    const int F = sh ? c.Fs : c.F;
+    const GuBias gb = sh ? GuBias{nullptr, nullptr, 1} : gu_bias(c.gu_layout, c.F, t.seg, p.gate_up_bias, p.gate_bias);
+    uint32_t g[16], u[16];
+    fetch(ch * 16, g);
+    fetch(BNB / 2 + ch * 16, u);
+    const int fb = t.n_blk * (BNB / 2) + ch * 16;
+    if (store && fb < F) gate_up_chunk(g, u, gb.g, gb.u, gb.stride, fb, F, c.act, wi, out + grow * c.Fmax);
+  } else {
+    const uint16_t* bias = (!sh && p.down_bias) ? p.down_bias + (int64_t)t.seg * c.d : nullptr;
+    uint32_t v[16];
+    fetch(ch * 16, v);
+    const int ob = t.n_blk * BNB + ch * 16;
+    if (store && ob < c.d) {
+      const float w = (sh || c.weigh_inputs) ? 1.f : p.roww[grow];
+      down_chunk(v, bias, ob, c.d, w, out + grow * c.d);
+    }
+  }
+}
+
+// MODE 0: gate_up; 1: down; 2: gate_up then down in one launch (small batches with x
+// read in place).  In MODE 2 a CTA's producer, reaching a down tile of a segment
+// whose h rows are not all written yet, loads the weights of the tile's first stages
+// and waits for the segment's count of finished h regions before loading the h rows.
+// Every CTA takes its gate_up units before its down units, and a gate_up unit waits
+// on no other CTA, so the waits end once every CTA runs (one per SM, a cooperative
+// launch).
 template <int MODE, int ABOX>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBs,
-                   const __grid_constant__ CUtensorMap tmG, const TcParams p) {
+                   const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmA2,
+                   const __grid_constant__ CUtensorMap tmAs2, const __grid_constant__ CUtensorMap tmB2,
+                   const __grid_constant__ CUtensorMap tmBs2, const TcParams p) {
   constexpr int STAGES = Stage<ABOX>::COUNT, STAGE_BYTES = Stage<ABOX>::BYTES, A_BYTES = Stage<ABOX>::A_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -86,8 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const GemmCommon& c = p.c;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* const status = p.c.status;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; s++) {
@@ -105,7 +256,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmAs);
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmBs);
-    if (MODE == 0 && c.gu_layout == MOE_GU_UNFUSED) prefetch_tmap(&tmG);
+    if (MODE != 1 && p.c.gu_layout == MOE_GU_UNFUSED) prefetch_tmap(&tmG);
+    if (MODE == 2) {
+      prefetch_tmap(&tmA2);
+      prefetch_tmap(&tmAs2);
+      prefetch_tmap(&tmB2);
+      prefetch_tmap(&tmBs2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -116,53 +273,83 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   pdl_enter();
   const uint32_t tmem_base = *tmem_slot;
-  // Work units: (tile, split).  Split sp of a tile covers k-blocks
-  // [sp * nkb / S, (sp + 1) * nkb / S) of the tile's K range.
-  const int S = c.splits;
-  const int total = c.tiles[c.NS] * S;
+  // Work units: (tile, split) of the GEMM (MODE 2: of gate_up, then of down).  Split
+  // sp of a tile covers k-blocks [sp * nkb / S, (sp + 1) * nkb / S) of its K range.
+  const int u1 = p.c.tiles[p.c.NS] * p.c.splits;
+  const int total = u1 + (MODE == 2 ? p.c2.tiles[p.c2.NS] * p.c2.splits : 0);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      auto issue = [&](const Tile& t, int kb, uint64_t* bar, uint8_t* sa) {
-        const bool sh = t.seg >= c.E;
-        const int arow = (sh || (MODE == 0 && c.direct_x)) ? t.m0 : c.off[t.seg] + t.m0;
-        const CUtensorMap* mA = sh ? &tmAs : &tmA;
-        const CUtensorMap* mB = sh ? &tmBs : &tmB;
-        const int e = sh ? 0 : t.seg;
+      // the activation rows of k-block kb (x, gathered rows, or h)
+      auto issue_a = [&](const Unit& u, int kb, uint64_t* bar, uint8_t* sa) {
+        const GemmCommon& c = (MODE == 2 && u.dn) ? p.c2 : p.c;
+        const bool sh = u.t.seg >= c.E;
+        const int arow = (sh || (!u.dn && c.direct_x)) ? u.t.m0 : c.off[u.t.seg] + u.t.m0;
+        const CUtensorMap* m = (MODE == 2 && u.dn) ? (sh ? &tmAs2 : &tmA2) : (sh ? &tmAs : &tmA);
+        tma_load_2d(m, bar, sa, kb * BK, arow);
+      };
+      // the 256 weight rows of k-block kb
+      auto issue_b = [&](const Unit& u, int kb, uint64_t* bar, uint8_t* sb) {
+        const GemmCommon& c = (MODE == 2 && u.dn) ? p.c2 : p.c;
+        const bool sh = u.t.seg >= c.E;
+        const int e = sh ? 0 : u.t.seg;
         const int k0 = kb * BK;
-        tma_load_2d(mA, bar, sa, k0, arow);
-        if (MODE == 0 && c.ffn == MOE_FFN_PLAIN) {
-          tma_load_3d(mB, bar, sa + A_BYTES, k0, t.n_blk * BNB, e);  // 256 rows of fc1 [E][F][d]
-        } else if (MODE == 0 && c.gu_layout == MOE_GU_UNFUSED && !sh) {
-          const int f0 = t.n_blk * (BNB / 2);  // 128 gate rows, then the 128 up rows
-          tma_load_3d(&tmG, bar, sa + A_BYTES, k0, f0, e);
-          tma_load_3d(mB, bar, sa + A_BYTES + B_BYTES / 2, k0, f0, e);
-        } else if (MODE == 0) {
-          const int f0 = t.n_blk * (BNB / 2);
+        if (u.dn) {
+          const CUtensorMap* m = MODE == 2 ? (sh ? &tmBs2 : &tmB2) : (sh ? &tmBs : &tmB);
+          tma_load_3d(m, bar, sb, k0, u.t.n_blk * BNB, e);  // 256 rows of down [E][d][F]
+        } else if (c.ffn == MOE_FFN_PLAIN) {
+          tma_load_3d(sh ? &tmBs : &tmB, bar, sb, k0, u.t.n_blk * BNB, e);  // 256 rows of fc1 [E][F][d]
+        } else if (c.gu_layout == MOE_GU_UNFUSED && !sh) {
+          const int f0 = u.t.n_blk * (BNB / 2);  // 128 gate rows, then the 128 up rows
+          tma_load_3d(&tmG, bar, sb, k0, f0, e);
+          tma_load_3d(&tmB, bar, sb + B_BYTES / 2, k0, f0, e);
+        } else {
+          const int f0 = u.t.n_blk * (BNB / 2);
           const bool il = c.gu_layout == MOE_GU_INTERLEAVED;
           for (int half = 0; half < 2; half++) {
             const int c1 = il ? half : f0, c2 = il ? f0 : half;
-            tma_load_4d(mB, bar, sa + A_BYTES + half * (B_BYTES / 2), k0, c1, c2, e);
+            tma_load_4d(sh ? &tmBs : &tmB, bar, sb + half * (B_BYTES / 2), k0, c1, c2, e);
           }
-        } else {
-          tma_load_3d(mB, bar, sa + A_BYTES, k0, t.n_blk * BNB, e);
         }
       };
       uint32_t it = 0;
       bool ok = true;
       for (int unit = blockIdx.x; ok && unit < total; unit += gridDim.x) {
-        const Tile t = decode_tile<BM>(c, unit / S);
-        const int nkb = (k_extent<MODE>(c, t.seg >= c.E) + BK - 1) / BK;
-        const int sp = unit % S, kb1 = (sp + 1) * nkb / S;
-        for (int kb = sp * nkb / S; kb < kb1; kb++, it++) {
+        const Unit u = unit_of<MODE>(p, unit, u1);
+        // MODE 2 down unit whose h rows are not complete: the first `pre` stages get
+        // their weights now and their h tiles once the rows are ready
+        int pre = 0, need = 0;
+        if (MODE == 2 && u.dn && u.t.seg < p.c.NS) {
+          need = h_regions(p.c, u.t.seg);
+          if (ld_acquire_gpu(p.ready + u.t.seg) < need) pre = min(u.kb1 - u.kb0, STAGES);
+        }
+        for (int kb = u.kb0; kb < u.kb1; kb++, it++) {
           const int s = it % STAGES;
-          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, c.status)) {
+          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, status)) {
+            // stages that hold weights without their h tile get it, so that every
+            // issued stage completes before the CTA exits
+            const int held = kb - u.kb0 < pre ? kb - u.kb0 : 0;
+            for (int j = 0; j < held; j++) {
+              const uint32_t i2 = it - held + j;
+              issue_a(u, u.kb0 + j, &full[i2 % STAGES], smem + (i2 % STAGES) * STAGE_BYTES);
+            }
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-          issue(t, kb, &full[s], smem + s * STAGE_BYTES);
+          uint8_t* sa = smem + s * STAGE_BYTES;
+          issue_b(u, kb, &full[s], sa + A_BYTES);
+          if (kb - u.kb0 >= pre) {
+            issue_a(u, kb, &full[s], sa);
+          } else if (kb - u.kb0 == pre - 1) {
+            wait_count(p.ready + u.t.seg, need, status);
+            fence_proxy_async_all();
+            for (int j = 0; j < pre; j++) {
+              const uint32_t i2 = it - (pre - 1) + j;
+              issue_a(u, u.kb0 + j, &full[i2 % STAGES], smem + (i2 % STAGES) * STAGE_BYTES);
+            }
+          }
         }
       }
       // every load issued into a stage has landed before the CTA may exit
@@ -178,17 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       for (int unit = blockIdx.x; ok && unit < total; unit += gridDim.x, tcount++) {
-        const Tile t = decode_tile<BM>(c, unit / S);
-        const bool sh = t.seg >= c.E;
-        const int nkb = (k_extent<MODE>(c, sh) + BK - 1) / BK;
-        const int sp = unit % S, kb0 = sp * nkb / S, kb1 = (sp + 1) * nkb / S;
+        const Unit u = unit_of<MODE>(p, unit, u1);
         const int acc = tcount & 1;
-        if (!mbar_wait(&tempty[acc], ((tcount >> 1) & 1) ^ 1, abort_flag, c.status)) break;
+        if (!mbar_wait(&tempty[acc], ((tcount >> 1) & 1) ^ 1, abort_flag, status)) break;
         tc_fence_after();
         const uint32_t dt = tmem_base + acc * ACC_COLS;
-        for (int kb = kb0; kb < kb1; kb++, it++) {
+        for (int kb = u.kb0; kb < u.kb1; kb++, it++) {
           const int s = it % STAGES;
-          if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag, c.status)) {
+          if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag, status)) {
             ok = false;
             break;
           }
@@ -197,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t ad = sdesc_k_sw128(sa), bd = sdesc_k_sw128(sa + A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; kk++)
-            mma_bf16(dt, ad + 2 * kk, bd + 2 * kk, IDESC, (kb > kb0 || kk > 0) ? 1u : 0u);
+            mma_bf16(dt, ad + 2 * kk, bd + 2 * kk, IDESC, (kb > u.kb0 || kk > 0) ? 1u : 0u);
           mma_commit(&empty[s]);
         }
         if (ok) mma_commit(&tfull[acc]);
@@ -212,20 +396,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;            // this warp may read TMEM lanes 32q .. 32q+31
     const int part = (warp - 2) / 4;   // which alternate column chunks this warp drains
+    const int region = warp - 2;       // this warp's region of a tile (split-K, h readiness)
     const int r_in_tile = q * 32 + lane;
     uint32_t tcount = 0;
     for (int unit = blockIdx.x; unit < total; unit += gridDim.x, tcount++) {
-      const Tile t = decode_tile<BM>(c, unit / S);
+      const Unit u = unit_of<MODE>(p, unit, u1);
+      const GemmCommon& c = (MODE == 2 && u.dn) ? p.c2 : p.c;
+      uint16_t* out = (MODE == 2 && u.dn) ? p.out2 : p.out;
+      const Tile& t = u.t;
       const bool sh = t.seg >= c.E;
       const int acc = tcount & 1;
-      if (!mbar_wait(&tfull[acc], (tcount >> 1) & 1, abort_flag, c.status)) break;
+      if (!mbar_wait(&tfull[acc], (tcount >> 1) & 1, abort_flag, status)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * ACC_COLS;
       const int row = t.m0 + r_in_tile;
       bool valid = row < t.rows;
       int64_t grow = (int64_t)c.off[t.seg] + row;
       float wi = 1.f;  // weigh-inputs scale of the accumulators (direct_x only)
-      if (MODE == 0 && c.direct_x && !sh) {
+      if (!u.dn && c.direct_x && !sh) {
         // accumulator row = token r_in_tile: its row of this expert, if it chose it
         valid = false;
         if (r_in_tile < c.T) {
@@ -237,11 +425,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (valid && c.weigh_inputs) wi = p.roww[grow];
       }
-      if (S > 1) {
-        // split-K: this unit's fp32 partial accumulator row goes to the partial buffer
-        if (__any_sync(0xffffffffu, valid)) {
-          float* prow = c.partial + ((int64_t)(unit % S) * (c.R + (c.Fs > 0 ? c.T : 0)) + grow) * c.partial_pitch +
-                        t.n_blk * ACC_COLS;
+      const bool any = __any_sync(0xffffffffu, valid);
+      auto from_tmem = [&](int col, uint32_t (&v)[16]) {
+        tmem_ld16(tb + col, v);
+        tmem_ld_wait();
+      };
+      bool final_region = true;  // this warp's region of the tile holds its final output
+      if (u.S > 1) {
+        // split-K: this split's fp32 partial accumulators, then the last split of
+        // the region to arrive sums them all and runs the epilogue
+        const int64_t split_stride = (int64_t)(c.R + (c.Fs > 0 ? c.T : 0)) * c.partial_pitch;
+        float* prow = c.partial + (int64_t)u.sp * split_stride + grow * c.partial_pitch + t.n_blk * ACC_COLS;
+        if (any) {
 #pragma unroll 1
           for (int ch = part; ch < ACC_COLS / 16; ch += kEpiGroups) {
             uint32_t v[16];
@@ -256,52 +451,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-      } else if (__any_sync(0xffffffffu, valid)) {
-        if (MODE == 0 && c.ffn == MOE_FFN_PLAIN) {
-          const int F = sh ? c.Fs : c.F;
-          const int f0 = t.n_blk * BNB;
-          const uint16_t* bias = (!sh && p.gate_up_bias) ? p.gate_up_bias + (int64_t)t.seg * c.F : nullptr;
-          uint16_t* out = p.out + grow * c.Fmax;
-#pragma unroll 1
-          for (int ch = part; ch < BNB / 16; ch += kEpiGroups) {
-            uint32_t v[16];
-            tmem_ld16(tb + ch * 16, v);
-            tmem_ld_wait();
-            const int fb = f0 + ch * 16;
-            if (valid && fb < F) plain_chunk(v, bias, fb, F, c.act, wi, out);
-          }
-        } else if (MODE == 0) {
-          const int F = sh ? c.Fs : c.F;
-          const int f0 = t.n_blk * (BNB / 2);
-          const GuBias gb = sh ? GuBias{nullptr, nullptr, 1}
-                               : gu_bias(c.gu_layout, c.F, t.seg, p.gate_up_bias, p.gate_bias);
-          uint16_t* out = p.out + grow * c.Fmax;
-#pragma unroll 1
-          for (int ch = part; ch < (BNB / 2) / 16; ch += kEpiGroups) {
-            uint32_t g[16], u[16];
-            tmem_ld16(tb + ch * 16, g);
-            tmem_ld16(tb + BNB / 2 + ch * 16, u);
-            tmem_ld_wait();
-            const int fb = f0 + ch * 16;
-            if (valid && fb < F) gate_up_chunk(g, u, gb.g, gb.u, gb.stride, fb, F, c.act, wi, out);
-          }
-        } else {
-          const int n0 = t.n_blk * BNB;
-          const uint16_t* bias = (!sh && p.down_bias) ? p.down_bias + (int64_t)t.seg * c.d : nullptr;
-          const float w = (sh || c.weigh_inputs || !valid) ? 1.f : p.roww[grow];
-          uint16_t* out = p.out + grow * c.d;
-#pragma unroll 1
-          for (int ch = part; ch < BNB / 16; ch += kEpiGroups) {
-            uint32_t v[16];
-            tmem_ld16(tb + ch * 16, v);
-            tmem_ld_wait();
-            const int ob = n0 + ch * 16;
-            if (valid && ob < c.d) down_chunk(v, bias, ob, c.d, w, out);
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+        final_region = split_arrive(c.fix + (int64_t)u.tile * kFixRegions + region, u.S, lane);
+        if (final_region && any) {
+          // (row, chunk) items of the region spread over the lanes, so that the
+          // partials of up to 32 chunks are in flight at once
+          const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+          const int nch = (chunks_of(c, u.dn) - part + kEpiGroups - 1) / kEpiGroups;
+          const int items = __popc(vmask) * nch;
+          for (int base = 0; base < items; base += 32) {
+            const int item = base + lane;
+            const int ri = item < items ? item / nch : 0;
+            uint32_t m = vmask;  // the lane holding the ri-th valid row
+            for (int i = 0; i < ri; i++) m &= m - 1;
+            const int src = __ffs(m) - 1;
+            const int64_t g_row = __shfl_sync(0xffffffffu, grow, src);
+            const float w_row = __shfl_sync(0xffffffffu, wi, src);
+            if (item < items) {
+              const float* row0 = c.partial + g_row * c.partial_pitch + t.n_blk * ACC_COLS;
+              emit_chunk(p, c, u.dn, out, t, true, g_row, w_row, part + (item % nch) * kEpiGroups,
+                         [&](int col, uint32_t (&v)[16]) { sum_splits(row0 + col, split_stride, u.S, v); });
+            }
           }
         }
+      } else {
+        if (any) {
+#pragma unroll 1
+          for (int ch = part; ch < chunks_of(c, u.dn); ch += kEpiGroups)
+            emit_chunk(p, c, u.dn, out, t, valid, grow, wi, ch, from_tmem);
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      if (MODE == 2 && !u.dn && final_region) signal_region(p.ready + t.seg, lane);
     }
   }
 
@@ -352,26 +535,35 @@ bool map_down(CUtensorMap* m, const void* base, uint64_t F, uint64_t d, uint64_t
   return make_map(m, base, 3, dims, strides, box);
 }
 
+// The kernel's tensor maps: gate_up (a, as, b, bs, g) and, for MODE 2, down (a2 .. bs2).
+// Maps a mode does not read are copies of a used one.
+struct Maps {
+  CUtensorMap a, as, b, bs, g, a2, as2, b2, bs2;
+};
+
 template <int MODE, int ABOX>
-cudaError_t launch_box(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMap& b, const CUtensorMap& bs,
-                       const CUtensorMap& g, const TcParams& p, int num_sms, cudaStream_t st) {
+cudaError_t launch_box(const Maps& m, const TcParams& p, int num_sms, cudaStream_t st) {
   constexpr int smem = Stage<ABOX>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE, ABOX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int units = p.c.max_tiles * p.c.splits;
+  const int units = p.c.max_tiles * p.c.splits + (MODE == 2 ? p.c2.max_tiles * p.c2.splits : 0);
   const int grid = units < num_sms ? units : num_sms;
-  return launch_pdl(tc_gemm_kernel<MODE, ABOX>, (unsigned)grid, kThreads, smem, st, a, as, b, bs, g, p);
+  if (MODE == 2)  // CTAs wait for h regions that other CTAs write: all must be resident
+    return launch_coop_pdl(tc_gemm_kernel<MODE, ABOX>, (unsigned)grid, kThreads, smem, st, m.a, m.as, m.b, m.bs,
+                           m.g, m.a2, m.as2, m.b2, m.bs2, p);
+  return launch_pdl(tc_gemm_kernel<MODE, ABOX>, (unsigned)grid, kThreads, smem, st, m.a, m.as, m.b, m.bs, m.g, m.a2,
+                    m.as2, m.b2, m.bs2, p);
 }
 
 // Activation rows each stage loads: no segment has more rows than there are tokens.
 int a_box_rows(const GemmCommon& c) { return c.T <= 32 ? 32 : c.T <= 64 ? 64 : BM; }
 
 template <int MODE>
-cudaError_t launch(const CUtensorMap& a, const CUtensorMap& as, const CUtensorMap& b, const CUtensorMap& bs,
-                   const CUtensorMap& g, const TcParams& p, int abox, int num_sms, cudaStream_t st) {
-  if (abox == 32) return launch_box<MODE, 32>(a, as, b, bs, g, p, num_sms, st);
-  if (abox == 64) return launch_box<MODE, 64>(a, as, b, bs, g, p, num_sms, st);
-  return launch_box<MODE, BM>(a, as, b, bs, g, p, num_sms, st);
+cudaError_t launch(const Maps& m, const TcParams& p, int abox, int num_sms, cudaStream_t st) {
+  if (abox == 32) return launch_box<MODE, 32>(m, p, num_sms, st);
+  if (abox == 64) return launch_box<MODE, 64>(m, p, num_sms, st);
+  if (MODE == 2) return cudaErrorInvalidValue;  // only batches of at most 64 tokens
+  return launch_box<MODE == 2 ? 0 : MODE, BM>(m, p, num_sms, st);
 }
 
 // Maps of one gate_up weight stack (E experts of F features): a plain fc1 [E][F][d]
@@ -390,48 +582,78 @@ bool map_fc1(CUtensorMap* m, const void* base, uint64_t d, uint64_t F, uint64_t 
 
 }  // namespace
 
-cudaError_t launch_tc_gate_up(const TcArgs& a, cudaStream_t st) {
+namespace {
+
+// gate_up maps: activation rows (x itself for direct_x, else the gathered rows), the
+// weight stack, the shared expert's rows and stack, the unfused gate stack.
+bool gate_up_maps(const TcArgs& a, int abox, Maps* m) {
   const GemmCommon& c = a.c;
-  if (c.max_tiles == 0) return cudaSuccess;
-  CUtensorMap mA, mAs, mB, mBs, mG;
-  const int abox = a_box_rows(c);
-  // small batches read the activation rows from x itself (direct_x), else the rows
-  // gathered into expert order
-  bool ok = c.direct_x ? map_rows(&mA, a.x, c.d, c.T, c.d, abox) : map_rows(&mA, a.xg, c.d, c.R, c.d, abox);
-  ok = ok && map_fc1(&mB, a.gate_up, c.d, c.F, c.E, c.ffn, c.gu_layout);
-  if (c.gu_layout == MOE_GU_UNFUSED) ok = ok && map_fc1(&mG, a.gate, c.d, c.F, c.E, c.ffn, c.gu_layout);
-  else mG = mB;
+  bool ok = c.direct_x ? map_rows(&m->a, a.x, c.d, c.T, c.d, abox) : map_rows(&m->a, a.xg, c.d, c.R, c.d, abox);
+  ok = ok && map_fc1(&m->b, a.gate_up, c.d, c.F, c.E, c.ffn, c.gu_layout);
+  if (c.gu_layout == MOE_GU_UNFUSED) ok = ok && map_fc1(&m->g, a.gate, c.d, c.F, c.E, c.ffn, c.gu_layout);
+  else m->g = m->b;
   if (c.Fs > 0) {
     // the shared expert keeps one stack (gate rows first when the routed experts are unfused)
     const int sh_layout = c.gu_layout == MOE_GU_UNFUSED ? MOE_GU_CONCAT : c.gu_layout;
-    ok = ok && map_rows(&mAs, a.x, c.d, c.T, c.d, abox);
-    ok = ok && map_fc1(&mBs, a.sh_gate_up, c.d, c.Fs, 1, c.ffn, sh_layout);
+    ok = ok && map_rows(&m->as, a.x, c.d, c.T, c.d, abox);
+    ok = ok && map_fc1(&m->bs, a.sh_gate_up, c.d, c.Fs, 1, c.ffn, sh_layout);
   } else {
-    mAs = mA;
-    mBs = mB;
+    m->as = m->a;
+    m->bs = m->b;
   }
-  if (!ok) return cudaErrorInvalidValue;
+  return ok;
+}
+
+// down maps: h rows (routed, then the shared expert's at R), the down stacks.
+bool down_maps(const TcArgs& a, const GemmCommon& c, int abox, CUtensorMap* mA, CUtensorMap* mAs, CUtensorMap* mB,
+               CUtensorMap* mBs) {
+  bool ok = map_rows(mA, a.h, c.F, c.R, c.Fmax, abox);
+  ok = ok && map_down(mB, a.down, c.F, c.d, c.E);
+  if (c.Fs > 0) {
+    ok = ok && map_rows(mAs, (const uint16_t*)a.h + (int64_t)c.R * c.Fmax, c.Fs, c.T, c.Fmax, abox);
+    ok = ok && map_down(mBs, a.sh_down, c.Fs, c.d, 1);
+  } else {
+    *mAs = *mA;
+    *mBs = *mB;
+  }
+  return ok;
+}
+
+}  // namespace
+
+cudaError_t launch_tc_gate_up(const TcArgs& a, cudaStream_t st) {
+  const GemmCommon& c = a.c;
+  if (c.max_tiles == 0) return cudaSuccess;
+  Maps m;
+  const int abox = a_box_rows(c);
+  if (!gate_up_maps(a, abox, &m)) return cudaErrorInvalidValue;
+  m.a2 = m.as2 = m.b2 = m.bs2 = m.b;
   TcParams p{c, (const uint16_t*)a.gate_up_bias, (const uint16_t*)a.gate_bias, nullptr, a.roww, (uint16_t*)a.h};
-  return launch<0>(mA, mAs, mB, mBs, mG, p, abox, a.num_sms, st);
+  return launch<0>(m, p, abox, a.num_sms, st);
 }
 
 cudaError_t launch_tc_down(const TcArgs& a, cudaStream_t st) {
   const GemmCommon& c = a.c;
   if (c.max_tiles == 0) return cudaSuccess;
-  CUtensorMap mA, mAs, mB, mBs;
+  Maps m;
   const int abox = a_box_rows(c);
-  bool ok = map_rows(&mA, a.h, c.F, c.R, c.Fmax, abox);
-  ok = ok && map_down(&mB, a.down, c.F, c.d, c.E);
-  if (c.Fs > 0) {
-    ok = ok && map_rows(&mAs, (const uint16_t*)a.h + (int64_t)c.R * c.Fmax, c.Fs, c.T, c.Fmax, abox);
-    ok = ok && map_down(&mBs, a.sh_down, c.Fs, c.d, 1);
-  } else {
-    mAs = mA;
-    mBs = mB;
-  }
-  if (!ok) return cudaErrorInvalidValue;
+  if (!down_maps(a, c, abox, &m.a, &m.as, &m.b, &m.bs)) return cudaErrorInvalidValue;
+  m.g = m.a2 = m.as2 = m.b2 = m.bs2 = m.b;
   TcParams p{c, nullptr, nullptr, (const uint16_t*)a.down_bias, a.roww, (uint16_t*)a.Y};
-  return launch<1>(mA, mAs, mB, mBs, mB, p, abox, a.num_sms, st);
+  return launch<1>(m, p, abox, a.num_sms, st);
+}
+
+cudaError_t launch_tc_ffn(const TcArgs& a, const GemmCommon& dn, int32_t* ready, cudaStream_t st) {
+  const GemmCommon& c = a.c;
+  if (c.max_tiles == 0) return cudaSuccess;
+  Maps m;
+  const int abox = a_box_rows(c);
+  if (!c.direct_x || c.order || !ready || abox > 64) return cudaErrorInvalidValue;
+  if (!gate_up_maps(a, abox, &m) || !down_maps(a, dn, abox, &m.a2, &m.as2, &m.b2, &m.bs2))
+    return cudaErrorInvalidValue;
+  TcParams p{c, (const uint16_t*)a.gate_up_bias, (const uint16_t*)a.gate_bias, (const uint16_t*)a.down_bias,
+             a.roww, (uint16_t*)a.h, dn, (uint16_t*)a.Y, ready};
+  return launch<2>(m, p, abox, a.num_sms, st);
 }
 
 }  // namespace moe

@@ -14,10 +14,12 @@ namespace {
 using namespace sorting;
 
 // Per-chunk expert histogram: hist[b][e] = #(t in chunk b, j) with idx[t][j] == e.
+// Also clears the GEMMs' counters (SortArgs::sync).
 __global__ void __launch_bounds__(256) hist_kernel(SortArgs a) {
   pdl_enter();
   extern __shared__ int32_t sh[];
   const int b = blockIdx.x;
+  for (int i = b * blockDim.x + threadIdx.x; i < a.n_sync; i += gridDim.x * blockDim.x) a.sync[i] = 0;
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) sh[e] = 0;
   __syncthreads();
   const int t0 = b * kChunkTokens;
@@ -54,7 +56,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(SortArgs a) {
 }
 
 // The whole sort for a single chunk of tokens (T <= kChunkTokens) in one block:
-// histogram in shared memory, the segment scan, and the in-order scatter.
+// histogram in shared memory, the segment scan, and the in-order scatter (and the
+// GEMMs' counters cleared).
 __global__ void __launch_bounds__(1024) sort_one_chunk_kernel(SortArgs a) {
   __shared__ int32_t cnt[kMaxE + 1];
   __shared__ int32_t tg[kMaxE + 1];
@@ -64,6 +67,7 @@ __global__ void __launch_bounds__(1024) sort_one_chunk_kernel(SortArgs a) {
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t tot;
   pdl_enter();
+  for (int i = threadIdx.x; i < a.n_sync; i += blockDim.x) a.sync[i] = 0;
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
     cnt[e] = 0;
     run[e] = 0;

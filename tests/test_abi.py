@@ -27,7 +27,8 @@ def test_header_declares_the_entry_points():
     assert _declared() == sorted(["moe_options_init", "moe_workspace_size", "moe_forward",
                                   "moe_route", "moe_forward_events", "moe_forward_noalloc",
                                   "moe_noalloc_debug_status", "moe_noalloc_workspace_bytes",
-                                  "moe_forward_kernel_count", "moe_last_error", "moe_debug_status",
+                                  "moe_forward_kernel_count", "moe_forward_split_k",
+                                  "moe_forward_fused_gemms", "moe_last_error", "moe_debug_status",
                                   "moe_version"])
 
 
@@ -180,28 +181,48 @@ def test_binding_without_its_library_imports_but_every_entry_point_raises(tmp_pa
 
 
 @pytest.mark.parametrize("name,count", [
-    ("tiny_fp32", 6), ("decode_T1", 6), ("decode_T8", 5), ("decode_T64", 5), ("decode_T256", 8),
+    ("tiny_fp32", 6), ("decode_T1", 4), ("decode_T8", 4), ("decode_T64", 4), ("decode_T256", 8),
     ("mixtral_bf16", 8), ("gptoss_mxfp4", 8), ("deepseek_bf16", 8)])
 def test_kernel_count_of_each_workload(moe, name, count):
     """The launch plan on a 148-SM part (what the host assumes without a GPU): route,
     sort (one kernel for a single 64-token chunk, else histogram + scan + scatter),
     gather (not for bf16 batches of at most 64 tokens, whose gate_up reads x in
-    place), gate_up, down, combine, plus a reduction per GEMM whose K is split.
-    Decode T=1 splits gate_up only (96 tiles of 64 k-blocks would leave 52 SMs idle)."""
+    place), gate_up, down (one launch with gate_up for those batches), combine.
+    Split-K adds no launch: the last split of a tile region reduces it."""
     from workloads import CONFIGS
     cfg = CONFIGS[name]
     assert moe.moe_forward_kernel_count(moe.shape_of(cfg), moe.options_of(cfg)) == count
 
 
+@pytest.mark.parametrize("name,fused", [
+    ("tiny_fp32", 0), ("decode_T1", 1), ("decode_T8", 1), ("decode_T64", 1), ("decode_T256", 0),
+    ("mixtral_bf16", 0), ("gptoss_mxfp4", 0), ("deepseek_bf16", 0)])
+def test_fused_gemms_for_small_bf16_batches(moe, name, fused, monkeypatch):
+    from workloads import CONFIGS
+    cfg = CONFIGS[name]
+    shape, opts = moe.shape_of(cfg), moe.options_of(cfg)
+    assert moe.moe_forward_fused_gemms(shape, opts) == fused
+    monkeypatch.setenv("MOE_B200_FUSED_FFN", "0")
+    assert moe.moe_forward_fused_gemms(shape, opts) == 0
+    assert moe.moe_forward_kernel_count(shape, opts) == (5 if fused else moe.moe_forward_kernel_count(shape, opts))
+
+
 def test_split_k_choice_follows_the_cost_model(moe):
-    """choose_splits: cost = waves * (k-blocks per unit + 2) + 4 for the reduction.
-    T=1, E=8, k=1, d=4096, F=1024: gate_up has 8 tiles x 64 k-blocks -> 8 splits (one
-    wave of 64 units of 8 k-blocks: cost 14 against 66); down has 16 tiles x 16 k-blocks
-    -> 8 splits (cost 8 against 18).  T=65 (two sort chunks): gate_up 64 tiles -> 2
-    splits (cost 38; 4 splits cost 40), down 128 tiles -> no split (18 against 24)."""
+    """choose_splits: cost = waves * (k-blocks per unit + 2) + 4 for the read-back of
+    the partials.  T=1, E=8, k=1, d=4096, F=1024: gate_up has 8 tiles x 64 k-blocks ->
+    8 splits (one wave of 64 units of 8 k-blocks: cost 14 against 66); down has 16
+    tiles x 16 k-blocks -> 8 splits (cost 8 against 18).  T=65 (two sort chunks):
+    gate_up 64 tiles -> 2 splits (cost 38; 4 splits cost 40), down 128 tiles -> no
+    split (18 against 24).  Decode T=1 (E=128, k=8, d=4096, F=1536): gate_up 96 tiles x
+    64 k-blocks -> 3 splits (2 waves of 22: cost 52 against 66), down 128 tiles x 24 ->
+    none (26 against 32)."""
     o = moe.make_options()
-    assert moe.moe_forward_kernel_count(moe.make_shape(T=1, d=4096, F=1024, E=8, k=1), o) == 5 + 2
-    assert moe.moe_forward_kernel_count(moe.make_shape(T=65, d=4096, F=1024, E=8, k=1), o) == 8 + 1
+    assert moe.moe_forward_split_k(moe.make_shape(T=1, d=4096, F=1024, E=8, k=1), o) == (8, 8)
+    assert moe.moe_forward_split_k(moe.make_shape(T=65, d=4096, F=1024, E=8, k=1), o) == (2, 1)
+    assert moe.moe_forward_split_k(moe.make_shape(T=1, d=4096, F=1536, E=128, k=8), o) == (3, 1)
     # fp32 problems run the SIMT GEMMs, which never split K
     f32 = moe.make_shape(T=1, d=4096, F=1024, E=8, k=1, act_dtype="f32", w_dtype="f32", logit_dtype="f32")
+    assert moe.moe_forward_split_k(f32, o) == (1, 1)
     assert moe.moe_forward_kernel_count(f32, o) == 6
+    with pytest.raises(moe.MoeError):
+        moe.moe_forward_split_k(moe.make_shape(T=1, d=4096, F=1024, E=8, k=0), o)
