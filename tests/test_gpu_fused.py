@@ -26,6 +26,9 @@ CASES = {
     "T64_ragged": small(DEC, name="T64_ragged", T=64, d=200, F=136, E=12, k=3, Fs=72),
     "T3_sigmoid_groups": small(CONFIGS["deepseek_bf16"], name="T3_sigmoid_groups", T=3, d=256, F=128, E=64,
                                k=8, Fs=128),
+    # the router weight in front of the routing
+    "T40_router": small(DEC, name="T40_router", T=40, router="weight", router_bias=True),
+    "T64_router_many_experts": small(DEC, name="T64_router_many_experts", T=64, E=700, k=5, router="weight"),
 }
 
 
