@@ -315,6 +315,10 @@ def measure_workload(cfg, steps, warmup, flush, stream):
     y = torch.empty_like(inputs["x"])
     idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
     tens = moe.tensors_of(inputs, y, idx, None)
+    # the inputs are generated, and these buffers allocated, on the default stream, whose
+    # kernels may still be writing memory the allocator handed out; the forwards run on
+    # `stream`: let that work finish first
+    torch.cuda.synchronize()
     sptr = stream.cuda_stream
     names = list(moe.STAGES)
 
@@ -424,6 +428,10 @@ def run_own(args, cfg):
     idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
     tens = moe.tensors_of(inputs, y, idx, None)
     flush = L2Flush(torch)
+    # the inputs are generated, and these buffers allocated, on the default stream, whose
+    # kernels may still be writing memory the allocator handed out (temporaries of the
+    # input generation); the forwards run on `stream`: let that work finish first
+    torch.cuda.synchronize()
     nev = moe.MOE_STAGE_EVENTS
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
     for row in events:

@@ -101,13 +101,16 @@ __device__ __forceinline__ int h_regions(const GemmCommon& gu, int seg) {
   return (gu.tiles[seg + 1] - gu.tiles[seg]) * kEpiWarps;
 }
 
-// Bounded wait until *ctr >= need.  On a timeout it records MOE_ERR_TIMEOUT and
-// returns: the h rows then read are not final, and the forward reports the error.
-__device__ __forceinline__ void wait_count(const int32_t* ctr, int need, int* status) {
-  if (ld_acquire_gpu(ctr) >= need) return;
+// Bounded wait until *ctr >= need.  On a timeout it records MOE_ERR_TIMEOUT and sets
+// the CTA's abort flag (later waits then return at once, and the other roles stop);
+// the h rows then read are not final, and the forward reports the error.
+__device__ __forceinline__ void wait_count(const int32_t* ctr, int need, volatile int* abort, int* status) {
+  if (ld_acquire_gpu(ctr) >= need || *abort) return;
   const uint64_t t0 = global_timer();
   while (ld_acquire_gpu(ctr) < need) {
+    if (*abort) return;
     if (global_timer() - t0 > kTimeoutNs) {
+      *abort = 1;
       set_status(status, MOE_ERR_TIMEOUT);
       return;
     }
@@ -170,6 +173,48 @@ __device__ __noinline__ void sum_splits(const float* row, int64_t split_stride, 
   for (int i = 0; i < 16; i++) v[i] = __float_as_uint(a[i]);
 }
 
+// The same for two 16-column groups of the row at once (a gate chunk and its up
+// partner): the loads of three slots of both at a time are issued before their sums.
+__device__ __noinline__ void sum_splits_pair(const float* ra, const float* rb, int64_t split_stride, int S,
+                                             uint32_t (&va)[16], uint32_t (&vb)[16]) {
+  float a[16], b[16];
+#pragma unroll
+  for (int i = 0; i < 16; i++) a[i] = b[i] = 0.f;
+#pragma unroll 1
+  for (int s0 = 0; s0 < S; s0 += 3) {
+    float4 qa[3][4], qb[3][4];
+#pragma unroll
+    for (int j = 0; j < 3; j++)
+      if (s0 + j < S) {
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+          qa[j][i] = __ldcg(reinterpret_cast<const float4*>(ra + (s0 + j) * split_stride) + i);
+          qb[j][i] = __ldcg(reinterpret_cast<const float4*>(rb + (s0 + j) * split_stride) + i);
+        }
+      }
+#pragma unroll
+    for (int j = 0; j < 3; j++)
+      if (s0 + j < S) {
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+          a[4 * i] += qa[j][i].x;
+          a[4 * i + 1] += qa[j][i].y;
+          a[4 * i + 2] += qa[j][i].z;
+          a[4 * i + 3] += qa[j][i].w;
+          b[4 * i] += qb[j][i].x;
+          b[4 * i + 1] += qb[j][i].y;
+          b[4 * i + 2] += qb[j][i].z;
+          b[4 * i + 3] += qb[j][i].w;
+        }
+      }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; i++) {
+    va[i] = __float_as_uint(a[i]);
+    vb[i] = __float_as_uint(b[i]);
+  }
+}
+
 // Column chunks of a tile's accumulator row: a gated gate_up chunk ch is gate columns
 // 16ch .. 16ch+15 with their up partners 128 columns on (8 chunks); plain gate_up and
 // down chunks are 16 columns each (16 chunks).
@@ -178,12 +223,13 @@ __device__ __forceinline__ int chunks_of(const GemmCommon& c, bool dn) {
 }
 
 // The epilogue of chunk ch of one accumulator row (output row grow, weigh-inputs
-// scale wi), stored if `store`; fetch(col, v) yields columns col .. col+15 of the row
-// (called whether or not the chunk is stored: TMEM loads are whole-warp).
-template <typename Fetch>
+// scale wi), stored if `store`; fetch(col, v) yields columns col .. col+15 of the row,
+// fetch2(c1, c2, v1, v2) two such groups (called whether or not the chunk is stored:
+// TMEM loads are whole-warp).
+template <typename Fetch, typename Fetch2>
 __device__ __forceinline__ void emit_chunk(const TcParams& p, const GemmCommon& c, bool dn, uint16_t* out,
                                            const Tile& t, bool store, int64_t grow, float wi, int ch,
-                                           Fetch&& fetch) {
+                                           Fetch&& fetch, Fetch2&& fetch2) {
   const bool sh = t.seg >= c.E;
   if (!dn && c.ffn == MOE_FFN_PLAIN) {
     const int F = sh ? c.Fs : c.F;
@@ -196,8 +242,7 @@ __device__ __forceinline__ void emit_chunk(const TcParams& p, const GemmCommon& 
     const int F = sh ? c.Fs : c.F;
     const GuBias gb = sh ? GuBias{nullptr, nullptr, 1} : gu_bias(c.gu_layout, c.F, t.seg, p.gate_up_bias, p.gate_bias);
     uint32_t g[16], u[16];
-    fetch(ch * 16, g);
-    fetch(BNB / 2 + ch * 16, u);
+    fetch2(ch * 16, BNB / 2 + ch * 16, g, u);
     const int fb = t.n_blk * (BNB / 2) + ch * 16;
     if (store && fb < F) gate_up_chunk(g, u, gb.g, gb.u, gb.stride, fb, F, c.act, wi, out + grow * c.Fmax);
   } else {
@@ -343,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kb - u.kb0 >= pre) {
             issue_a(u, kb, &full[s], sa);
           } else if (kb - u.kb0 == pre - 1) {
-            wait_count(p.ready + u.t.seg, need, status);
+            wait_count(p.ready + u.t.seg, need, abort_flag, status);
             fence_proxy_async_all();
             for (int j = 0; j < pre; j++) {
               const uint32_t i2 = it - (pre - 1) + j;
@@ -430,6 +475,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld16(tb + col, v);
         tmem_ld_wait();
       };
+      auto from_tmem2 = [&](int c1, int c2, uint32_t (&v1)[16], uint32_t (&v2)[16]) {
+        tmem_ld16(tb + c1, v1);
+        tmem_ld16(tb + c2, v2);
+        tmem_ld_wait();
+      };
       bool final_region = true;  // this warp's region of the tile holds its final output
       if (u.S > 1) {
         // split-K: this split's fp32 partial accumulators, then the last split of
@@ -437,17 +487,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t split_stride = (int64_t)(c.R + (c.Fs > 0 ? c.T : 0)) * c.partial_pitch;
         float* prow = c.partial + (int64_t)u.sp * split_stride + grow * c.partial_pitch + t.n_blk * ACC_COLS;
         if (any) {
+          // two chunks per TMEM wait
+          constexpr int kGroup = 2;
 #pragma unroll 1
-          for (int ch = part; ch < ACC_COLS / 16; ch += kEpiGroups) {
-            uint32_t v[16];
-            tmem_ld16(tb + ch * 16, v);
+          for (int c0 = part; c0 < ACC_COLS / 16; c0 += kGroup * kEpiGroups) {
+            uint32_t v[kGroup][16];
+#pragma unroll
+            for (int j = 0; j < kGroup; j++)
+              if (c0 + j * kEpiGroups < ACC_COLS / 16) tmem_ld16(tb + (c0 + j * kEpiGroups) * 16, v[j]);
             tmem_ld_wait();
             if (valid) {
-              float4* dst = reinterpret_cast<float4*>(prow + ch * 16);
 #pragma unroll
-              for (int i = 0; i < 4; i++)
-                dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                     __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+              for (int j = 0; j < kGroup; j++) {
+                const int ch = c0 + j * kEpiGroups;
+                if (ch >= ACC_COLS / 16) break;
+                float4* dst = reinterpret_cast<float4*>(prow + ch * 16);
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                  dst[i] = make_float4(__uint_as_float(v[j][4 * i]), __uint_as_float(v[j][4 * i + 1]),
+                                       __uint_as_float(v[j][4 * i + 2]), __uint_as_float(v[j][4 * i + 3]));
+              }
             }
           }
         }
@@ -471,7 +530,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (item < items) {
               const float* row0 = c.partial + g_row * c.partial_pitch + t.n_blk * ACC_COLS;
               emit_chunk(p, c, u.dn, out, t, true, g_row, w_row, part + (item % nch) * kEpiGroups,
-                         [&](int col, uint32_t (&v)[16]) { sum_splits(row0 + col, split_stride, u.S, v); });
+                         [&](int col, uint32_t (&v)[16]) { sum_splits(row0 + col, split_stride, u.S, v); },
+                         [&](int c1, int c2, uint32_t (&v1)[16], uint32_t (&v2)[16]) {
+                           sum_splits_pair(row0 + c1, row0 + c2, split_stride, u.S, v1, v2);
+                         });
             }
           }
         }
@@ -479,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (any) {
 #pragma unroll 1
           for (int ch = part; ch < chunks_of(c, u.dn); ch += kEpiGroups)
-            emit_chunk(p, c, u.dn, out, t, valid, grow, wi, ch, from_tmem);
+            emit_chunk(p, c, u.dn, out, t, valid, grow, wi, ch, from_tmem, from_tmem2);
         }
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
