@@ -64,16 +64,19 @@ class L2Flush:
 # dominant GEMM, each from one ncu capture of that kernel, with the kernel's source file and
 # the hash of that file and the headers it includes (kernel_sources_hash) at capture time.
 # A figure whose hash is not the current sources' belongs to an older kernel: reported null.
-#   mixtral_bf16 gate_up: full-size capture, median of two launches (2.7992 GB read + 0.2312
-#     GB written).
+#   mixtral_bf16 gate_up: full-size capture (2.8381 GB read + 0.2332 GB written).
 #   deepseek_bf16 gate_up: captured at E=32 T=1024 (same 256 routed rows per expert and one
-#     shared row per token, one eighth of every operand) and scaled by 8: 2.1719 GB read +
-#     0.0373 GB written per launch there.
-#   gptoss_mxfp4 gate_up: full-size capture, 0.3297 GB read + 0.0389 GB written.
+#     shared row per token, one eighth of every operand) and scaled by 8: 2.1751 GB read +
+#     0.0363 GB written per launch there.
+#   gptoss_mxfp4 gate_up: full-size capture, 0.3299 GB read + 0.0384 GB written.
+#   decode_T1 / decode_T8: the one launch of both GEMMs, full size (median of 18 launches):
+#     0.3042 GB + 0.8 MB and 0.9445 GB + 1.2 MB.
 NCU_TRAFFIC = {
-    ("mixtral_bf16", "gate_up"): (3030478336, "gemm_tcs.cu", "c8f80540d88e"),
-    ("deepseek_bf16", "gate_up"): (8 * (2171850000 + 37275392), "gemm_tcs.cu", "c8f80540d88e"),
-    ("gptoss_mxfp4", "gate_up"): (329742592 + 38918400, "gemm_fp4.cu", "667efd3d31dc"),
+    ("mixtral_bf16", "gate_up"): (2838147328 + 233207040, "gemm_tcs.cu", "40335cf4263a"),
+    ("deepseek_bf16", "gate_up"): (8 * (2175083776 + 36308480), "gemm_tcs.cu", "40335cf4263a"),
+    ("gptoss_mxfp4", "gate_up"): (329914368 + 38359296, "gemm_fp4.cu", "9a1e7a69371c"),
+    ("decode_T1", "gate_up"): (304210304 + 772224, "gemm_tc.cu", "232e4161c62f"),
+    ("decode_T8", "gate_up"): (944453376 + 1232768, "gemm_tc.cu", "232e4161c62f"),
 }
 
 
