@@ -246,6 +246,17 @@ struct GemmCommon {
   int32_t* fix;
 };
 
+// The GEMM's tile count from the device-side prefix, at most the host's bound
+// max_tiles past tiles[seg_begin]: a larger count means the workspace was changed
+// under the call (MOE_ERR_SHAPE recorded, the walk clamped to the bound).
+__device__ __forceinline__ int tile_total(const GemmCommon& c) {
+  const int first = c.tiles[c.seg_begin];
+  const int total = c.tiles[c.NS];
+  if (total >= first && total - first <= c.max_tiles) return total;
+  set_status(c.status, MOE_ERR_SHAPE);
+  return total < first ? first : first + c.max_tiles;
+}
+
 struct SimtArgs {
   GemmCommon c;
   const float* x;           // [T, d] (shared rows read x directly)

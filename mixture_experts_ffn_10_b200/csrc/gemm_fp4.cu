@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   pdl_enter();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = c.tiles[c.NS];
+  const int total = tile_total(c);
   const int K = k_extent<MODE>(c);
   const int nkb = (K + BK - 1) / BK;
 

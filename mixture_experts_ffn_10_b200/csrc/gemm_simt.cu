@@ -22,7 +22,7 @@ struct TileInfo {
 };
 
 __device__ __forceinline__ bool find_tile(const GemmCommon& c, int tile, TileInfo* ti) {
-  const int total = c.tiles[c.NS];
+  const int total = tile_total(c);
   if (tile >= total) return false;
   int lo = 0, hi = c.NS - 1;  // last s with tiles[s] <= tile
   while (lo < hi) {

@@ -320,8 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   // Work units: (tile, split) of the GEMM (MODE 2: of gate_up, then of down).  Split
   // sp of a tile covers k-blocks [sp * nkb / S, (sp + 1) * nkb / S) of its K range.
-  const int u1 = p.c.tiles[p.c.NS] * p.c.splits;
-  const int total = u1 + (MODE == 2 ? p.c2.tiles[p.c2.NS] * p.c2.splits : 0);
+  const int u1 = tile_total(p.c) * p.c.splits;
+  const int total = u1 + (MODE == 2 ? tile_total(p.c2) * p.c2.splits : 0);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer

@@ -119,7 +119,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   pdl_enter();
   const uint32_t tmem_base = *tmem_slot;
   const int S = 1;  // the plan never splits K for pair tiles (launch rejects it)
-  const int total = c.tiles[c.NS];
+  const int total = tile_total(c);
   const int first = c.tiles[c.seg_begin];  // tiles of segments seg_begin .. NS-1 only
 
   if (warp == 0) {

@@ -115,7 +115,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   pdl_enter();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = c.tiles[c.NS];
+  const int total = tile_total(c);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
