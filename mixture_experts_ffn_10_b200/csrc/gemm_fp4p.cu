@@ -26,7 +26,8 @@
 //               CTAs' barriers;
 //   warps 2-9   epilogue of this CTA's 128 accumulator lanes (its weight rows);
 //   warps 10-25 converters (four groups of four warps): codes + scales -> bf16 in
-//               the 128B-swizzled K-major layout, a proxy fence, a local barrier of
+//               the 128B-swizzled K-major layout, a proxy fence for this CTA's
+//               shared memory, a local barrier of
 //               the group's warps, then one arrival per group and stage on the even
 //               CTA's decoded-slot barrier (remote, with release at cluster scope,
 //               from the odd CTA);
@@ -428,7 +429,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           break;
         }
         decode_row_sw128(q0, q1, sc, ringW + sw * W_BYTES + r * (BK * 2), r);
-        fence_proxy_async_all();
+        // this CTA's shared memory, which the pair MMAs read through the async proxy
+        // (the all-state-space fence cost ~1200 cycles per stage here)
+        fence_proxy_async_smem();
         __syncwarp();
         // the group's four warps meet on a local barrier, then its first warp signals
         // the slot to the MMA issuer (one remote arrival per stage from the odd CTA)

@@ -135,7 +135,7 @@ __device__ __forceinline__ bool split_arrive(int32_t* ctr, int S, int lane) {
 // MODE 2 down tiles, whose h loads go through the async proxy.
 __device__ __forceinline__ void signal_region(int32_t* ctr, int lane) {
   __threadfence();
-  fence_proxy_async_all();
+  fence_proxy_async_global();
   __syncwarp();
   if (lane == 0) atomicAdd(ctr, 1);
 }
@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_a(u, kb, &full[s], sa);
           } else if (kb - u.kb0 == pre - 1) {
             wait_count(p.ready + u.t.seg, need, abort_flag, status);
-            fence_proxy_async_all();
+            fence_proxy_async_global();
             for (int j = 0; j < pre; j++) {
               const uint32_t i2 = it - (pre - 1) + j;
               issue_a(u, u.kb0 + j, &full[i2 % STAGES], smem + (i2 % STAGES) * STAGE_BYTES);

@@ -108,6 +108,9 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // read through the cluster window included).
 __device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
 
+// The same for global memory only (rows other CTAs' TMA loads read).
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
 // Load with acquire semantics at GPU scope (a counter other CTAs release into).
 __device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
   int32_t v;
