@@ -23,11 +23,12 @@
 //   warps 2-9   epilogue: two warps per TMEM lane quadrant, alternate 16-token chunks;
 //               for gate_up, weight rows 2j and 2j+1 are the gate and up rows of one
 //               feature, so neighbouring lanes pair up with one shuffle
-//   warps 10-24 except 13, 17, 21: converters in three groups of four, group g
-//               owning stages it % 3 == g: codes + scale -> bf16 in the 128B-swizzled
-//               K-major layout the MMA descriptor reads (mxfp4.cuh), then a proxy
-//               fence and one arrive per warp.  None shares the MMA issuer's
-//               scheduler (warp w issues on scheduler w % 4); warps 17 and 21 idle.
+//   warps 10-30 except 13, 17, 21, 25, 29: converters in four groups of four, group
+//               g owning stages it % 4 == g: codes + scale -> bf16 in the
+//               128B-swizzled K-major layout the MMA descriptor reads (mxfp4.cuh),
+//               then a proxy fence and one arrive per warp.  None shares the MMA
+//               issuer's scheduler (warp w issues on scheduler w % 4); warps 17, 21,
+//               25 and 29 idle.
 #include "epilogue.cuh"
 #include "mxfp4.cuh"
 #include "sm100.cuh"
@@ -45,7 +46,7 @@ constexpr int BNB = 128;                // weight rows per tile
 // Three rings, so that decoding never holds an activation slot:
 constexpr int AST = 4;                  // activations: 256 x 64 bf16, freed by the MMA
 constexpr int QST = 6;                  // e2m1 codes: 128 x 32 bytes, freed once converted
-constexpr int WST = 3;                  // decoded bf16 weights: 128 x 64, freed by the MMA
+constexpr int WST = 4;                  // decoded bf16 weights: 128 x 64, freed by the MMA
 constexpr int A_BYTES = BM * BK * 2;    // 32 KiB
 constexpr int Q_BYTES = BNB * BK / 2;   // 4 KiB
 constexpr int W_BYTES = BNB * BK * 2;   // 16 KiB
@@ -54,23 +55,27 @@ constexpr int ACC_COLS = BM;            // one column per activation row
 constexpr int TMEM_COLS = 2 * ACC_COLS; // double-buffered
 constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, alternate token chunks
 constexpr int kEpiGroups = kEpiWarps / 4;
-constexpr int kCvtWarps = 12;
-constexpr int kCvtGroups = 3;                // converter groups, each owning every 3rd stage
+constexpr int kCvtWarps = 16;
+constexpr int kCvtGroups = 4;                // converter groups, each owning every 4th stage
 constexpr int kCvtGroupWarps = kCvtWarps / kCvtGroups;
-// Warps 0 .. 24.  Warp w runs on the SM's scheduler w % 4; the MMA issuer (warp 1)
+// Warps 0 .. 30.  Warp w runs on the SM's scheduler w % 4; the MMA issuer (warp 1)
 // shares its scheduler only with warps that issue few instructions (two epilogue
 // warps and the code producer), never with a converter, so that its MMAs issue on
-// time: converters are the warps 10 .. 24 other than 13, 17 and 21.
-constexpr int kWarps = 25;
+// time: converters are the warps 10 .. 30 other than 13, 17, 21, 25 and 29.  Four
+// groups with a decoded slot each: a group's slot comes free three stages of MMAs
+// after it was filled (with three groups the converters waited ~400 cycles per stage
+// for it: 0.545 -> 0.527 ms per gpt-oss layer).
+constexpr int kWarps = 31;
 constexpr int kThreads = kWarps * 32;
 constexpr int kCodesWarp = 13;
 __host__ __device__ constexpr int converter_index(int w) {  // -1: not a converter
-  return (w < 10 || w >= kWarps || w % 4 == 1) ? -1 : w - 10 - (w > 13) - (w > 17) - (w > 21);
+  return (w < 10 || w >= kWarps || w % 4 == 1) ? -1
+                                               : w - 10 - (w > 13) - (w > 17) - (w > 21) - (w > 25) - (w > 29);
 }
 constexpr int SMEM_BYTES = RING_BYTES + 1024 + 512;
 static_assert(kCvtGroupWarps * 32 == BNB, "one converter thread per weight row in a group");
 static_assert(WST % kCvtGroups == 0, "a group's stages map to its own decoded-weight slots");
-static_assert(converter_index(24) == kCvtWarps - 1, "twelve converter warps");
+static_assert(converter_index(30) == kCvtWarps - 1, "sixteen converter warps");
 
 struct Fp4Params {
   GemmCommon c;
