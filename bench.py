@@ -64,19 +64,20 @@ class L2Flush:
 # dominant GEMM, each from one ncu capture of that kernel, with the kernel's source file and
 # the hash of that file and the headers it includes (kernel_sources_hash) at capture time.
 # A figure whose hash is not the current sources' belongs to an older kernel: reported null.
-#   mixtral_bf16 gate_up: full-size capture (2.8381 GB read + 0.2332 GB written).
+#   mixtral_bf16 gate_up: full-size capture (2.4584 GB read + 0.2333 GB written; other
+#     boxes read up to 2.84 GB: how many repeated weight-tile fetches hit L2 varies).
 #   deepseek_bf16 gate_up: captured at E=32 T=1024 (same 256 routed rows per expert and one
-#     shared row per token, one eighth of every operand) and scaled by 8: 2.1751 GB read +
-#     0.0363 GB written per launch there.
-#   gptoss_mxfp4 gate_up: full-size capture, 0.3299 GB read + 0.0384 GB written.
+#     shared row per token, one eighth of every operand) and scaled by 8: 2.1469 GB read +
+#     0.0359 GB written per launch there.
+#   gptoss_mxfp4 gate_up: full-size capture, 0.3297 GB read + 0.0375 GB written.
 #   decode_T1 / decode_T8: the one launch of both GEMMs, full size (the fourth launch of
-#     that kernel): 0.3040 GB + 0.8 MB and 0.9444 GB + 1.2 MB.
+#     that kernel): 0.3041 GB + 1.4 MB and 0.9444 GB + 1.2 MB.
 NCU_TRAFFIC = {
-    ("mixtral_bf16", "gate_up"): (2838147328 + 233207040, "gemm_tcs.cu", "40335cf4263a"),
-    ("deepseek_bf16", "gate_up"): (8 * (2175083776 + 36308480), "gemm_tcs.cu", "40335cf4263a"),
-    ("gptoss_mxfp4", "gate_up"): (329914368 + 38359296, "gemm_fp4.cu", "9a1e7a69371c"),
-    ("decode_T1", "gate_up"): (304019968 + 790272, "gemm_tc.cu", "232e4161c62f"),
-    ("decode_T8", "gate_up"): (944413440 + 1203968, "gemm_tc.cu", "232e4161c62f"),
+    ("mixtral_bf16", "gate_up"): (2458378496 + 233282048, "gemm_tcs.cu", "bccc21e5b5ea"),
+    ("deepseek_bf16", "gate_up"): (8 * (2146914048 + 35875072), "gemm_tcs.cu", "bccc21e5b5ea"),
+    ("gptoss_mxfp4", "gate_up"): (329699840 + 37458432, "gemm_fp4.cu", "5a9b55fdd5ed"),
+    ("decode_T1", "gate_up"): (304128768 + 1417728, "gemm_tc.cu", "25f399db458c"),
+    ("decode_T8", "gate_up"): (944408832 + 1224192, "gemm_tc.cu", "25f399db458c"),
 }
 
 
