@@ -202,7 +202,8 @@ MOE_API size_t moe_workspace_size(const moe_shape *shape, const moe_options *opt
  *     tile, with split-K for small batches (MOE_B200_PAIR_GEMM=0 or =1 forces
  *     one or the other); for T <= 64 gate_up reads x in place and, unless
  *     MOE_B200_FUSED_FFN=0 or MOE_B200_INTERLEAVE=1, gate_up and down run as one
- *     launch whose down tiles start once their expert's h rows are complete;
+ *     launch whose down tiles start once their expert's h rows are complete (a
+ *     cooperative launch; where its CTAs cannot all be resident, two launches);
  *   - MXFP4 weights: one CTA per tile; MOE_B200_PAIR_FP4=1 picks CTA pairs with
  *     256 decoded weight rows (slower on the shapes measured);
  *   - MOE_B200_INTERLEAVE=1: the bf16 GEMMs visit the experts largest first,

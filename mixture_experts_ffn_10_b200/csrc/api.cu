@@ -319,7 +319,18 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
     ta.c = fp4 ? gu_routed : gu;
     if (p.fused_ffn) {
       // gate_up and down in one launch: stage event 4 goes with event 5, after it
-      if ((e = launch_tc_ffn(ta, dn, ready, st)) != cudaSuccess) return cuda_fail(e, "fused gate_up + down GEMMs");
+      e = launch_tc_ffn(ta, dn, ready, st);
+      if (e == cudaErrorCooperativeLaunchTooLarge) {
+        // not every CTA can be resident at once here (SMs held by other work or a
+        // partitioned device): the two GEMMs as separate launches instead
+        cudaGetLastError();
+        ta.c = gu;
+        if ((e = launch_tc_gate_up(ta, st)) != cudaSuccess) return cuda_fail(e, "tensor-core gate_up GEMM");
+        ta.c = dn;
+        if ((e = launch_tc_down(ta, st)) != cudaSuccess) return cuda_fail(e, "tensor-core down GEMM");
+      } else if (e != cudaSuccess) {
+        return cuda_fail(e, "fused gate_up + down GEMMs");
+      }
       if ((e = mark(4)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     } else {
       e = fp4 ? (p.pair_fp4 ? launch_fp4p_gate_up(ta, st) : launch_fp4_gate_up(ta, st))
