@@ -62,7 +62,8 @@ class L2Flush:
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a workload's
 # dominant GEMM, each from one ncu capture of that kernel, with the kernel's source file and
-# the hash of that file and the headers it includes (kernel_sources_hash) at capture time.
+# the hash of the code of that file and the headers it includes (kernel_sources_hash,
+# comments stripped) at capture time.
 # A figure whose hash is not the current sources' belongs to an older kernel: reported null.
 #   mixtral_bf16 gate_up: full-size capture (2.4584 GB read + 0.2333 GB written; other
 #     boxes read up to 2.84 GB: how many repeated weight-tile fetches hit L2 varies).
@@ -73,17 +74,26 @@ class L2Flush:
 #   decode_T1 / decode_T8: the one launch of both GEMMs, full size (the fourth launch of
 #     that kernel): 0.3041 GB + 1.4 MB and 0.9444 GB + 1.2 MB.
 NCU_TRAFFIC = {
-    ("mixtral_bf16", "gate_up"): (2458378496 + 233282048, "gemm_tcs.cu", "bccc21e5b5ea"),
-    ("deepseek_bf16", "gate_up"): (8 * (2146914048 + 35875072), "gemm_tcs.cu", "bccc21e5b5ea"),
-    ("gptoss_mxfp4", "gate_up"): (329699840 + 37458432, "gemm_fp4.cu", "5a9b55fdd5ed"),
-    ("decode_T1", "gate_up"): (304128768 + 1417728, "gemm_tc.cu", "25f399db458c"),
-    ("decode_T8", "gate_up"): (944408832 + 1224192, "gemm_tc.cu", "25f399db458c"),
+    ("mixtral_bf16", "gate_up"): (2458378496 + 233282048, "gemm_tcs.cu", "c30a86d32a81"),
+    ("deepseek_bf16", "gate_up"): (8 * (2146914048 + 35875072), "gemm_tcs.cu", "c30a86d32a81"),
+    ("gptoss_mxfp4", "gate_up"): (329699840 + 37458432, "gemm_fp4.cu", "af0ca3377e18"),
+    ("decode_T1", "gate_up"): (304128768 + 1417728, "gemm_tc.cu", "f397cb915a5e"),
+    ("decode_T8", "gate_up"): (944408832 + 1224192, "gemm_tc.cu", "f397cb915a5e"),
 }
 
 
+def _code_of(text: bytes) -> bytes:
+    """A source file's code without its comments and blank-line differences, so that
+    editing a comment leaves the hash of the code unchanged."""
+    t = re.sub(rb"/\*.*?\*/", b" ", text, flags=re.S)
+    t = re.sub(rb"//[^\n]*", b"", t)
+    return b"\n".join(line.rstrip() for line in t.splitlines() if line.strip())
+
+
 def kernel_sources_hash(kernel_file: str = None) -> str:
-    """Short hash of one kernel source file of the library and every local header it
-    includes (transitively, plus include/moe.h); without a file, of all of csrc/."""
+    """Short hash of the code (comments stripped) of one kernel source file of the
+    library and every local header it includes (transitively, plus include/moe.h);
+    without a file, of all of csrc/."""
     import hashlib
     csrc = os.path.join(ROOT, "mixture_experts_ffn_10_b200", "csrc")
     if kernel_file is None:
@@ -102,7 +112,7 @@ def kernel_sources_hash(kernel_file: str = None) -> str:
     for f in [os.path.join(csrc, f) for f in files] + [os.path.join(ROOT, "include", "moe.h")]:
         h.update(os.path.basename(f).encode())
         with open(f, "rb") as fh:
-            h.update(fh.read())
+            h.update(_code_of(fh.read()))
     return h.hexdigest()[:12]
 
 

@@ -67,6 +67,13 @@ def test_traffic_figures_follow_their_kernel_sources(monkeypatch):
     assert bench.ncu_traffic("mixtral_bf16", "combine") is None
 
 
+def test_comment_edits_leave_the_code_hash_alone():
+    a = b"int f(int x) {  // doubles\n  return 2 * x; /* the\n body */\n}\n"
+    b = b"int f(int x) {\n\n  return 2 * x;\n}  // changed\n"
+    assert bench._code_of(a) == bench._code_of(b)
+    assert bench._code_of(a) != bench._code_of(a.replace(b"2 * x", b"3 * x"))
+
+
 def test_kernel_hash_covers_included_headers_only():
     import hashlib
     csrc = os.path.join(ROOT, "mixture_experts_ffn_10_b200", "csrc")
@@ -74,5 +81,5 @@ def test_kernel_hash_covers_included_headers_only():
     h = hashlib.sha256()
     for f in [os.path.join(csrc, f) for f in files] + [os.path.join(ROOT, "include", "moe.h")]:
         h.update(os.path.basename(f).encode())
-        h.update(open(f, "rb").read())
+        h.update(bench._code_of(open(f, "rb").read()))
     assert bench.kernel_sources_hash("gemm_tcs.cu") == h.hexdigest()[:12]
