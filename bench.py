@@ -77,7 +77,6 @@ NCU_TRAFFIC = {
     ("mixtral_bf16", "gate_up"): (2458378496 + 233282048, "gemm_tcs.cu", "c30a86d32a81"),
     ("deepseek_bf16", "gate_up"): (8 * (2146914048 + 35875072), "gemm_tcs.cu", "c30a86d32a81"),
     ("gptoss_mxfp4", "gate_up"): (329699840 + 37458432, "gemm_fp4.cu", "af0ca3377e18"),
-    ("decode_T1", "gate_up"): (304128768 + 1417728, "gemm_tc.cu", "f397cb915a5e"),
     ("decode_T8", "gate_up"): (944408832 + 1224192, "gemm_tc.cu", "f397cb915a5e"),
 }
 
@@ -311,6 +310,9 @@ def fuse_stages(model):
 
 
 def stage_label(dom, fused):
+    """fused: moe_forward_fused_gemms (2: the few-token kernel, 1: both GEMMs in one launch)."""
+    if fused == 2:
+        return "whole forward, one launch (few-token CUDA-core kernel)"
     return "gate_up + down grouped GEMMs (one launch)" if fused else f"{dom} grouped GEMM"
 
 
@@ -389,7 +391,7 @@ def measure_workload(cfg, steps, warmup, flush, stream):
     rows = torch.bincount(idx.flatten().long(), minlength=cfg.E)
     pk, pk_src = peaks()
     model = stage_model(cfg, distinct)
-    fused = moe.moe_forward_fused_gemms(shape, opts) == 1
+    fused = moe.moe_forward_fused_gemms(shape, opts)
     if fused:
         model = fuse_stages(model)
     dom = max(stage_ms, key=stage_ms.get)
@@ -639,7 +641,7 @@ def run_own(args, cfg):
     rows_per_expert = torch.bincount(idx.flatten().long(), minlength=cfg.E)
     pk, pk_src = peaks()
     model = stage_model(cfg, distinct)
-    fused = moe.moe_forward_fused_gemms(shape, opts) == 1
+    fused = moe.moe_forward_fused_gemms(shape, opts)
     if fused:
         model = fuse_stages(model)
     t_dom = dom_ms / 1e3

@@ -207,7 +207,12 @@ MOE_API size_t moe_workspace_size(const moe_shape *shape, const moe_options *opt
  *   - MXFP4 weights: one CTA per tile; MOE_B200_PAIR_FP4=1 picks CTA pairs with
  *     256 decoded weight rows (slower on the shapes measured);
  *   - MOE_B200_INTERLEAVE=1: the bf16 GEMMs visit the experts largest first,
- *     alternating with the smallest (results unchanged).
+ *     alternating with the smallest (results unchanged);
+ *   - MOE_B200_GEMV=N (N <= 4): bf16 batches of at most N tokens with E <= 256 and d,
+ *     F, Fs multiples of 64 run the whole forward in one cooperative launch (routing
+ *     inside it unless router_weight is given, then after the router kernel): each
+ *     warp streams weight tiles with TMA and multiplies them by the token rows with
+ *     warp-level mma.sync; off by default (slower on the shapes measured).
  * Launches: every kernel after the first may be scheduled while its
  * predecessor in the stream still runs (programmatic dependent launch) and
  * waits on the device for the predecessor's results; MOE_B200_PDL=0, read
@@ -279,7 +284,8 @@ MOE_API int moe_noalloc_debug_status(void *stream);
 MOE_API size_t moe_noalloc_workspace_bytes(void);
 
 /* Number of CUDA kernels one moe_forward of this problem launches (-1 if the
- * arguments are invalid; 0 for T == 0).  For launch accounting. */
+ * arguments are invalid; 0 for T == 0).  For launch accounting; with router_logits
+ * (the few-token kernel adds the router kernel when router_weight is given). */
 MOE_API int moe_forward_kernel_count(const moe_shape *shape, const moe_options *opts);
 
 /* The split-K factors moe_forward uses for the gate_up and down GEMMs of this
@@ -291,8 +297,10 @@ MOE_API int moe_forward_split_k(const moe_shape *shape, const moe_options *opts,
 
 /* 1 if moe_forward of this problem runs gate_up and down as one kernel launch
  * (batches of at most 64 tokens with bf16 weights; MOE_B200_FUSED_FFN=0 turns it
- * off), 0 if not, -1 if the arguments are invalid.  Stage events 4 and 5 are then
- * both recorded after that launch. */
+ * off), 2 if it runs the whole forward as one launch of the few-token kernel
+ * (MOE_B200_GEMV), 0 if neither, -1 if the arguments are invalid.  Stage events 4
+ * and 5 are then both recorded after that launch (with 2, events 1-3 before it and
+ * 4-6 after it). */
 MOE_API int moe_forward_fused_gemms(const moe_shape *shape, const moe_options *opts);
 
 /* Message of the last failed call on this thread ("" if none). */

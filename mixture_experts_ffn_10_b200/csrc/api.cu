@@ -125,6 +125,20 @@ int check_tensors(const moe_shape* s, const moe_options* o, const moe_tensors* t
   return MOE_OK;
 }
 
+// Largest dynamic shared memory a block may opt into on the current device.
+int smem_optin_of_current_device() {
+  static std::atomic<int> cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 232448;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (n <= 0) n = 232448;
+    cache[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
 int num_sms_of_current_device() {
   static std::atomic<int> cache[64] = {};  // callers may race: each writes the same value
   int dev = 0;
@@ -172,7 +186,9 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
     return cudaSuccess;
   };
   int* status = at<int>(ws, p.o_status);
-  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  // the status word and the few-token kernel's counters (kGemvDoneOffset bytes further)
+  const size_t counters = p.gemv ? kGemvRbOffset + (p.d + kGemvRowBlock - 1) / kGemvRowBlock * 4 : sizeof(int32_t);
+  cudaError_t e = cudaMemsetAsync(status, 0, counters, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   if ((e = mark(0)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
 
@@ -200,6 +216,64 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
   ra.sgate = (full && o->shared_gate) ? at<float>(ws, p.o_sgate) : nullptr;
   ra.router_weight = t->router_weight;
   ra.logits_out = t->logits_out;
+
+  // A few tokens: the whole forward in one launch, after the router GEMM when the layer
+  // computes the logits.  Stage events 1-3 precede the launch and 4-6 follow it.
+  if (full && p.gemv) {
+    GemvArgs ga{};
+    ga.ra = ra;
+    if (t->router_weight) {
+      if ((e = launch_router(ra, st)) != cudaSuccess) return cuda_fail(e, "router kernel");
+      ga.pre_routed = 1;
+      ga.idx = ra.idx;
+      ga.w = ra.w;
+      ga.sgate = ra.sgate;
+    }
+    for (int i = 1; i <= 3; i++)
+      if ((e = mark(i)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    ga.has_sgate = o->shared_gate;
+    ga.x = static_cast<const uint16_t*>(t->x);
+    ga.gate_up = static_cast<const uint16_t*>(t->gate_up);
+    ga.gate_up_bias = static_cast<const uint16_t*>(t->gate_up_bias);
+    ga.gate = static_cast<const uint16_t*>(t->gate);
+    ga.gate_bias = static_cast<const uint16_t*>(t->gate_bias);
+    ga.down = static_cast<const uint16_t*>(t->down);
+    ga.down_bias = static_cast<const uint16_t*>(t->down_bias);
+    ga.sh_gate_up = static_cast<const uint16_t*>(t->shared_gate_up);
+    ga.sh_down = static_cast<const uint16_t*>(t->shared_down);
+    ga.shared_output = static_cast<const uint16_t*>(t->shared_output);
+    ga.h = at<uint16_t>(ws, p.o_h);
+    ga.y = static_cast<uint16_t*>(t->y);
+    ga.done = at<int32_t>(ws, p.o_status + kGemvDoneOffset);
+    ga.rb_done = at<int32_t>(ws, p.o_status + kGemvRbOffset);
+    ga.Y = at<uint16_t>(ws, p.o_y);
+    ga.T = (int)p.T;
+    ga.d = (int)p.d;
+    ga.F = (int)p.F;
+    ga.Fs = (int)p.Fs;
+    ga.E = (int)p.E;
+    ga.k = (int)p.k;
+    ga.R = (int)p.R;
+    ga.Fmax = (int)p.Fmax;
+    ga.gu_layout = o->gu_layout;
+    ga.ffn = o->ffn;
+    ga.weigh_inputs = o->weigh_inputs;
+    ga.act = ActParams{o->act, o->alpha, o->beta, o->limit};
+    ga.status = status;
+    ga.warps = p.gemv_warps;
+    ga.xh_bytes = p.gemv_xh;
+    ga.smem_bytes = p.gemv_smem;
+    e = launch_gemv_ffn(ga, num_sms_of_current_device(), st);
+    if (e == cudaSuccess) {
+      for (int i = 4; i <= 6; i++)
+        if ((e = mark(i)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+      return MOE_OK;
+    }
+    if (e != cudaErrorCooperativeLaunchTooLarge) return cuda_fail(e, "few-token forward kernel");
+    // not every CTA can be resident at once here: the multi-launch path instead
+    cudaGetLastError();
+  }
+
   if ((e = t->router_weight ? launch_router(ra, st) : launch_route(ra, st)) != cudaSuccess)
     return cuda_fail(e, "route kernel");
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
@@ -448,6 +522,34 @@ bool use_fused_ffn() {
   return !(env && env[0] == '0');
 }
 
+// Batches of at most this many tokens (bf16 weights, E <= 256) run the whole forward
+// in one launch of the few-token kernel (gemv.cu) when MOE_B200_GEMV=N (N <= kGemvMaxTokens)
+// asks for it: measured slower than the multi-launch path on the decode layer (T = 1:
+// 90 vs 86 us), so off by default.
+int gemv_max_tokens() {
+  const char* env = std::getenv("MOE_B200_GEMV");
+  if (env && env[0] >= '0' && env[0] <= '9') return std::min(atoi(env), kGemvMaxTokens);
+  return kGemvDefaultTokens;
+}
+
+// Geometry of the few-token kernel: as many warps as shared memory allows (at most
+// kGemvMaxWarps, at least 4) beside the staging area of x or h (bf16); its tiles need
+// d, F and Fs in whole 64-element blocks.  False where that does not hold (then the
+// multi-launch path runs).
+bool plan_gemv(const moe_shape* s, Plan* p) {
+  if (s->d % 64 || s->F % 64 || s->Fs % 64) return false;
+  int64_t xh = std::max<int64_t>(s->T * s->d * 2, (p->R * s->F + (s->Fs > 0 ? s->T * s->Fs : 0)) * 2);
+  xh = (xh + 127) / 128 * 128;
+  const int64_t budget = smem_optin_of_current_device() - (int64_t)sizeof(GemvMeta) - 1024;
+  int64_t warps = kGemvMaxWarps;
+  while (warps >= 4 && gemv_smem((int)warps, (int)std::min<int64_t>(xh, 1 << 24)) > budget) warps--;
+  if (warps < 4) return false;
+  p->gemv_warps = (int)warps;
+  p->gemv_xh = (int)xh;
+  p->gemv_smem = gemv_smem((int)warps, (int)xh);
+  return true;
+}
+
 bool use_pair_gemm(int64_t R, int64_t E) {
   const char* env = std::getenv("MOE_B200_PAIR_GEMM");
   if (env && env[0] == '0') return false;
@@ -526,6 +628,8 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   p->max_tiles_gu = mt_routed * p->nt_gu_routed + mt_shared * p->nt_gu_shared;
   p->max_tiles_dn = mt_routed * p->nt_dn_routed + mt_shared * p->nt_dn_shared;
   p->fused_ffn = p->direct_x && !p->interleave && use_fused_ffn();
+  p->gemv_warps = p->gemv_xh = p->gemv_smem = 0;
+  p->gemv = p->tc && s->w_dtype == MOE_BF16 && !p->pair && s->T <= gemv_max_tokens() && s->E <= 8 * 32 && plan_gemv(s, p);
   p->n_sync = (p->splits_gu > 1 ? p->max_tiles_gu * kFixRegions : 0) +
               (p->splits_dn > 1 ? p->max_tiles_dn * kFixRegions : 0) + (p->fused_ffn ? p->NS : 0);
   const size_t elt = p->tc ? 2 : 4;
@@ -535,7 +639,7 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
     off = align256(off + bytes);
     return r;
   };
-  p->o_status = take(256);
+  p->o_status = take(p->gemv ? kGemvRbOffset + (p->d + kGemvRowBlock - 1) / kGemvRowBlock * 4 : 256);
   p->o_idx = take(p->R * 4);
   p->o_w = take(p->R * 4);
   p->o_hist = take(p->nchunks * p->E * 4);
@@ -602,6 +706,7 @@ int moe_forward_kernel_count(const moe_shape* s, const moe_options* o) {
   moe::make_plan(s, o, &p);
   // route, histogram, scan, scatter, gather (not for direct_x), gate_up, down (one
   // launch with gate_up when fused), combine; a single 64-token chunk sorts in one kernel
+  if (p.gemv) return 1;  // (plus the router GEMM when the layer computes the logits)
   return (p.nchunks == 1 ? 4 : 6) + (p.direct_x ? 0 : 1) + 1 - (p.fused_ffn ? 1 : 0) +
          (s->w_dtype == MOE_MXFP4 && p.Fs > 0 ? 2 : 0);  // the shared expert beside MXFP4 experts
 }
@@ -622,7 +727,7 @@ int moe_forward_fused_gemms(const moe_shape* s, const moe_options* o) {
   if (s->T == 0) return 0;
   moe::Plan p;
   moe::make_plan(s, o, &p);
-  return p.fused_ffn ? 1 : 0;
+  return p.gemv ? 2 : p.fused_ffn ? 1 : 0;
 }
 
 const char* moe_last_error(void) { return moe::g_err.c_str(); }

@@ -198,13 +198,40 @@ def test_kernel_count_of_each_workload(moe, name, count):
     ("tiny_fp32", 0), ("decode_T1", 1), ("decode_T8", 1), ("decode_T64", 1), ("decode_T256", 0),
     ("mixtral_bf16", 0), ("gptoss_mxfp4", 0), ("deepseek_bf16", 0)])
 def test_fused_gemms_for_small_bf16_batches(moe, name, fused, monkeypatch):
+    """1: gate_up and down in one launch (T <= 64), 0: separate launches;
+    MOE_B200_FUSED_FFN=0 steps down (2, the few-token kernel, is opt-in)."""
     from workloads import CONFIGS
     cfg = CONFIGS[name]
     shape, opts = moe.shape_of(cfg), moe.options_of(cfg)
     assert moe.moe_forward_fused_gemms(shape, opts) == fused
+    monkeypatch.setenv("MOE_B200_GEMV", "0")
+    assert moe.moe_forward_fused_gemms(shape, opts) == min(fused, 1)
+    assert moe.moe_forward_kernel_count(shape, opts) == (4 if fused else moe.moe_forward_kernel_count(shape, opts))
     monkeypatch.setenv("MOE_B200_FUSED_FFN", "0")
     assert moe.moe_forward_fused_gemms(shape, opts) == 0
     assert moe.moe_forward_kernel_count(shape, opts) == (5 if fused else moe.moe_forward_kernel_count(shape, opts))
+
+
+@pytest.mark.parametrize("T,gemv", [(1, True), (4, True), (5, False)])
+def test_few_token_kernel_limits(moe, T, gemv, monkeypatch):
+    """The few-token kernel (opt-in: MOE_B200_GEMV=N, N <= 4 tokens) serves bf16
+    weights, E <= 256 and d, F, Fs in whole 64-element blocks; forced CTA-pair GEMMs
+    keep their kernels."""
+    o = moe.make_options()
+    sh = moe.make_shape(T=T, d=4096, F=1536, E=128, k=8)
+    assert moe.moe_forward_fused_gemms(sh, o) != 2  # off by default
+    monkeypatch.setenv("MOE_B200_GEMV", "4")
+    assert (moe.moe_forward_fused_gemms(sh, o) == 2) == gemv
+    assert (moe.moe_forward_kernel_count(sh, o) == 1) == gemv
+    assert moe.moe_forward_fused_gemms(moe.make_shape(T=T, d=4096, F=1536, E=300, k=8), o) != 2
+    assert moe.moe_forward_fused_gemms(moe.make_shape(T=T, d=512, F=256, E=32, k=4, w_dtype="mxfp4"), o) != 2
+    assert moe.moe_forward_fused_gemms(moe.make_shape(T=T, d=200, F=256, E=32, k=4), o) != 2  # 64-element blocks
+    assert moe.moe_forward_fused_gemms(moe.make_shape(T=T, d=512, F=256, E=32, k=4, Fs=96), o) != 2
+    monkeypatch.setenv("MOE_B200_GEMV", "2")
+    assert (moe.moe_forward_fused_gemms(sh, o) == 2) == (T <= 2)
+    monkeypatch.setenv("MOE_B200_GEMV", "4")
+    monkeypatch.setenv("MOE_B200_PAIR_GEMM", "1")
+    assert moe.moe_forward_fused_gemms(sh, o) != 2
 
 
 def test_split_k_choice_follows_the_cost_model(moe):

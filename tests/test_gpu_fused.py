@@ -14,6 +14,13 @@ from gpu_cases import parity, run_gpu
 
 pytestmark = pytest.mark.gpu
 
+
+@pytest.fixture(autouse=True)
+def _tensor_core_path(monkeypatch):
+    """These cases test the tensor-core GEMMs: batches of at most 4 tokens would
+    otherwise run the few-token kernel (tests/test_gpu_gemv.py)."""
+    monkeypatch.setenv("MOE_B200_GEMV", "0")
+
 DEC = small(CONFIGS["decode_T1"], name="f_decode", d=512, F=256, E=32)
 CASES = {
     "T1": DEC,

@@ -57,7 +57,9 @@ CASES = {
 
 
 @pytest.mark.parametrize("name", list(CASES))
-def test_variant_matches_oracle(name):
+def test_variant_matches_oracle(name, monkeypatch):
+    if "split_k" in name:  # the split-K tensor-core GEMMs, not the few-token kernel
+        monkeypatch.setenv("MOE_B200_GEMV", "0")
     parity(CASES[name])
 
 
