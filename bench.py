@@ -77,6 +77,7 @@ NCU_TRAFFIC = {
     ("mixtral_bf16", "gate_up"): (2458378496 + 233282048, "gemm_tcs.cu", "c30a86d32a81"),
     ("deepseek_bf16", "gate_up"): (8 * (2146914048 + 35875072), "gemm_tcs.cu", "c30a86d32a81"),
     ("gptoss_mxfp4", "gate_up"): (329699840 + 37458432, "gemm_fp4.cu", "af0ca3377e18"),
+    ("decode_T1", "gate_up"): (304128768 + 1417728, "gemm_tc.cu", "f397cb915a5e"),
     ("decode_T8", "gate_up"): (944408832 + 1224192, "gemm_tc.cu", "f397cb915a5e"),
 }
 

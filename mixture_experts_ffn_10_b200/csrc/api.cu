@@ -19,6 +19,7 @@
 #include <string>
 
 #include "common.cuh"
+#include "gemv.cuh"
 
 namespace moe {
 namespace {
@@ -187,7 +188,8 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
   };
   int* status = at<int>(ws, p.o_status);
   // the status word and the few-token kernel's counters (kGemvDoneOffset bytes further)
-  const size_t counters = p.gemv ? kGemvRbOffset + (p.d + kGemvRowBlock - 1) / kGemvRowBlock * 4 : sizeof(int32_t);
+  const GemvPlan gp = full ? gemv_plan(s, p) : GemvPlan{};
+  const size_t counters = gp.on ? gemv_status_bytes(p.d) : sizeof(int32_t);
   cudaError_t e = cudaMemsetAsync(status, 0, counters, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   if ((e = mark(0)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
@@ -219,7 +221,7 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
 
   // A few tokens: the whole forward in one launch, after the router GEMM when the layer
   // computes the logits.  Stage events 1-3 precede the launch and 4-6 follow it.
-  if (full && p.gemv) {
+  if (gp.on) {
     GemvArgs ga{};
     ga.ra = ra;
     if (t->router_weight) {
@@ -260,9 +262,9 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
     ga.weigh_inputs = o->weigh_inputs;
     ga.act = ActParams{o->act, o->alpha, o->beta, o->limit};
     ga.status = status;
-    ga.warps = p.gemv_warps;
-    ga.xh_bytes = p.gemv_xh;
-    ga.smem_bytes = p.gemv_smem;
+    ga.warps = gp.warps;
+    ga.xh_bytes = gp.xh;
+    ga.smem_bytes = gp.smem;
     e = launch_gemv_ffn(ga, num_sms_of_current_device(), st);
     if (e == cudaSuccess) {
       for (int i = 4; i <= 6; i++)
@@ -532,22 +534,26 @@ int gemv_max_tokens() {
   return kGemvDefaultTokens;
 }
 
-// Geometry of the few-token kernel: as many warps as shared memory allows (at most
-// kGemvMaxWarps, at least 4) beside the staging area of x or h (bf16); its tiles need
-// d, F and Fs in whole 64-element blocks.  False where that does not hold (then the
-// multi-launch path runs).
-bool plan_gemv(const moe_shape* s, Plan* p) {
-  if (s->d % 64 || s->F % 64 || s->Fs % 64) return false;
-  int64_t xh = std::max<int64_t>(s->T * s->d * 2, (p->R * s->F + (s->Fs > 0 ? s->T * s->Fs : 0)) * 2);
+// The few-token kernel's plan: bf16 weights, no forced CTA pairs, T <= the limit,
+// E <= 256 (one routing warp of 8 experts per lane), d, F, Fs in whole 64-element
+// blocks, and as many warps as shared memory allows (at most kGemvMaxWarps, at least 4)
+// beside the staging area of x or h (bf16); off otherwise (then the multi-launch path
+// runs).
+GemvPlan gemv_plan(const moe_shape* s, const Plan& p) {
+  GemvPlan g;
+  if (!p.tc || s->w_dtype != MOE_BF16 || p.pair || s->T > gemv_max_tokens() || s->E > 8 * 32) return g;
+  if (s->d % 64 || s->F % 64 || s->Fs % 64) return g;
+  int64_t xh = std::max<int64_t>(s->T * s->d * 2, (p.R * s->F + (s->Fs > 0 ? s->T * s->Fs : 0)) * 2);
   xh = (xh + 127) / 128 * 128;
   const int64_t budget = smem_optin_of_current_device() - (int64_t)sizeof(GemvMeta) - 1024;
   int64_t warps = kGemvMaxWarps;
   while (warps >= 4 && gemv_smem((int)warps, (int)std::min<int64_t>(xh, 1 << 24)) > budget) warps--;
-  if (warps < 4) return false;
-  p->gemv_warps = (int)warps;
-  p->gemv_xh = (int)xh;
-  p->gemv_smem = gemv_smem((int)warps, (int)xh);
-  return true;
+  if (warps < 4) return g;
+  g.on = true;
+  g.warps = (int)warps;
+  g.xh = (int)xh;
+  g.smem = gemv_smem((int)warps, (int)xh);
+  return g;
 }
 
 bool use_pair_gemm(int64_t R, int64_t E) {
@@ -628,8 +634,6 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
   p->max_tiles_gu = mt_routed * p->nt_gu_routed + mt_shared * p->nt_gu_shared;
   p->max_tiles_dn = mt_routed * p->nt_dn_routed + mt_shared * p->nt_dn_shared;
   p->fused_ffn = p->direct_x && !p->interleave && use_fused_ffn();
-  p->gemv_warps = p->gemv_xh = p->gemv_smem = 0;
-  p->gemv = p->tc && s->w_dtype == MOE_BF16 && !p->pair && s->T <= gemv_max_tokens() && s->E <= 8 * 32 && plan_gemv(s, p);
   p->n_sync = (p->splits_gu > 1 ? p->max_tiles_gu * kFixRegions : 0) +
               (p->splits_dn > 1 ? p->max_tiles_dn * kFixRegions : 0) + (p->fused_ffn ? p->NS : 0);
   const size_t elt = p->tc ? 2 : 4;
@@ -639,7 +643,7 @@ size_t make_plan(const moe_shape* s, const moe_options* o, Plan* p) {
     off = align256(off + bytes);
     return r;
   };
-  p->o_status = take(p->gemv ? kGemvRbOffset + (p->d + kGemvRowBlock - 1) / kGemvRowBlock * 4 : 256);
+  p->o_status = take(gemv_plan(s, *p).on ? std::max<size_t>(256, gemv_status_bytes(p->d)) : 256);
   p->o_idx = take(p->R * 4);
   p->o_w = take(p->R * 4);
   p->o_hist = take(p->nchunks * p->E * 4);
@@ -706,7 +710,7 @@ int moe_forward_kernel_count(const moe_shape* s, const moe_options* o) {
   moe::make_plan(s, o, &p);
   // route, histogram, scan, scatter, gather (not for direct_x), gate_up, down (one
   // launch with gate_up when fused), combine; a single 64-token chunk sorts in one kernel
-  if (p.gemv) return 1;  // (plus the router GEMM when the layer computes the logits)
+  if (moe::gemv_plan(s, p).on) return 1;  // (plus the router GEMM when the layer computes the logits)
   return (p.nchunks == 1 ? 4 : 6) + (p.direct_x ? 0 : 1) + 1 - (p.fused_ffn ? 1 : 0) +
          (s->w_dtype == MOE_MXFP4 && p.Fs > 0 ? 2 : 0);  // the shared expert beside MXFP4 experts
 }
@@ -727,7 +731,7 @@ int moe_forward_fused_gemms(const moe_shape* s, const moe_options* o) {
   if (s->T == 0) return 0;
   moe::Plan p;
   moe::make_plan(s, o, &p);
-  return p.gemv ? 2 : p.fused_ffn ? 1 : 0;
+  return moe::gemv_plan(s, p).on ? 2 : p.fused_ffn ? 1 : 0;
 }
 
 const char* moe_last_error(void) { return moe::g_err.c_str(); }

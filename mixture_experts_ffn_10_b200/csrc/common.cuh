@@ -47,8 +47,6 @@ struct Plan {
   bool swap;          // bf16 GEMMs on CTA pairs with the weights as M (256 weight rows x <= 256 tokens)
   bool interleave;    // bf16 GEMMs visit the experts in interleaved order (sort.cuh: segment_scan)
   bool fused_ffn;     // direct_x: gate_up and down in one launch (launch_tc_ffn)
-  bool gemv;          // the whole forward in one launch of the few-token kernel (gemv.cu)
-  int gemv_warps, gemv_xh, gemv_smem;
   int bm;             // GEMM tile rows
   int nt_gu_routed, nt_gu_shared, nt_dn_routed, nt_dn_shared;  // N tiles per segment
   int splits_gu, splits_dn;  // split-K factors of the two GEMMs (1 = none)
@@ -309,74 +307,6 @@ cudaError_t launch_tc2_down(const TcArgs& a, cudaStream_t st);
 // single-CTA kernel.  a.c is the gate_up GEMM, dn the down GEMM; ready [NS] counts the
 // finished h regions of each segment (zero before the launch).
 cudaError_t launch_tc_ffn(const TcArgs& a, const GemmCommon& dn, int32_t* ready, cudaStream_t st);
-// ---------------------------------------------------------------- few-token forward
-// Batches of at most kGemvMaxTokens tokens with bf16 weights: the whole forward in one
-// cooperative launch (gemv.cu).  Every CTA routes the tokens itself (or reads the
-// routing kernel's result); then each warp streams its share of the chosen experts'
-// weights, tiles of 16 rows x kGemvKS, through its own shared-memory slots (TMA loads
-// it issues itself) and multiplies them by the tokens' rows with warp-level
-// mma.sync (the tokens are the 8 columns): gate_up (activation fused) first, then,
-// once every CTA has published its h features, down with the combine.
-constexpr int kGemvMaxTokens = 4;
-constexpr int kGemvDefaultTokens = 0;  // off unless MOE_B200_GEMV=N asks (measured slower)
-constexpr int kGemvMaxWarps = 16;
-constexpr int kGemvSlotsPerWarp = 2;
-constexpr int kGemvKB = 4;             // 64-element k-blocks per stage
-constexpr int kGemvKS = 64 * kGemvKB;  // K per stage
-constexpr int kGemvSlotBytes = 16 * kGemvKS * 2;  // 16 weight rows of one stage: 8 KiB
-constexpr int kGemvRowBlock = 16;      // output features per down unit
-constexpr int kGemvMaxEnt = kGemvMaxTokens * kMaxK + 1;  // distinct experts + the shared one
-constexpr int kGemvDoneOffset = 64;   // its CTA counter: workspace bytes after the status word
-constexpr int kGemvRbOffset = 128;    // its per-row-block counters [ceil(d / 16)]
-struct GemvArgs {
-  RouteArgs ra;             // in-kernel routing (router_logits given): idx, w, sgate unused
-  int pre_routed;           // 1: read idx, w (and sgate) that the routing kernel wrote
-  const int32_t* idx;       // [T, k] (pre_routed)
-  const float* w;           // [T, k] (pre_routed)
-  const float* sgate;       // [T] or null (pre_routed with a shared gate)
-  int has_sgate;            // shared expert output times sigmoid(x . g)
-  const uint16_t* x;        // [T, d]
-  const uint16_t* gate_up;  // as TcArgs
-  const uint16_t* gate_up_bias;
-  const uint16_t* gate;
-  const uint16_t* gate_bias;
-  const uint16_t* down;
-  const uint16_t* down_bias;
-  const uint16_t* sh_gate_up;
-  const uint16_t* sh_down;
-  const uint16_t* shared_output;  // [T, d] or null
-  uint16_t* h;              // [rows, Fmax] workspace
-  uint16_t* Y;              // [rows, d] workspace: each routed slot's (and shared) expert output
-  uint16_t* y;              // [T, d]
-  int32_t* done;            // CTAs that have published their h features (zero before the launch)
-  int32_t* rb_done;         // [ceil(d / 16)] down units finished per row block (zero before)
-  int T, d, F, Fs, E, k, R, Fmax;
-  int gu_layout, ffn, weigh_inputs;
-  ActParams act;
-  int* status;
-  int warps, xh_bytes, smem_bytes;  // geometry (make_plan)
-};
-// The few-token kernel's routing result and its list of distinct experts (static
-// shared memory): entry u is expert e[u] (-1: the shared expert) with cnt[u] token
-// slots; slot c is token tok[u][c], row row[u][c] of h and Y (t k + j, or R + t for
-// the shared expert), routing weight wt[u][c] (1 for the shared expert).
-struct GemvMeta {
-  int32_t idx[kGemvMaxTokens * kMaxK];
-  float w[kGemvMaxTokens * kMaxK];
-  float sgate[kGemvMaxTokens];
-  int n_ent;
-  int abort;
-  int e[kGemvMaxEnt], cnt[kGemvMaxEnt];
-  int tok[kGemvMaxEnt][kGemvMaxTokens], row[kGemvMaxEnt][kGemvMaxTokens];
-  float wt[kGemvMaxEnt][kGemvMaxTokens];
-};
-// Dynamic shared-memory bytes of the few-token kernel: alignment slack, the warps'
-// slots and the x / h staging area of xh bytes.
-__host__ __device__ constexpr int gemv_smem(int warps, int xh) {
-  return 1024 + warps * kGemvSlotsPerWarp * kGemvSlotBytes + xh;
-}
-cudaError_t launch_gemv_ffn(const GemvArgs& a, int num_sms, cudaStream_t st);
-
 // Split count for a GEMM of at most `tiles` tiles of `nkb` k-blocks on `sms` SMs.
 int choose_splits(int64_t tiles, int nkb, int sms);
 // MXFP4 expert stacks (gate_up / down are e2m1 codes), routed segments only (a shared

@@ -27,6 +27,7 @@
 // hold the first down stages meanwhile.  A down unit writes its Y rows; the last of
 // the units of a 16-feature row block (a per-block counter) combines that block.
 #include "epilogue.cuh"
+#include "gemv.cuh"
 #include "route.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
