@@ -125,6 +125,15 @@ def ncu_traffic(workload: str, stage: str):
     return rec[0]
 
 
+KERNEL_CHOICE_VARS = ("MOE_B200_PAIR_GEMM", "MOE_B200_SWAP_GEMM", "MOE_B200_FUSED_FFN", "MOE_B200_PAIR_FP4",
+                      "MOE_B200_INTERLEAVE", "MOE_B200_GEMV")
+
+
+def default_kernels() -> bool:
+    """True when no environment variable overrides the library's choice of kernels."""
+    return not any(os.environ.get(v) for v in KERNEL_CHOICE_VARS)
+
+
 def traffic_kernel_sources(workload: str, stage: str):
     """(kernel file, current hash) of the kernel a traffic figure belongs to, or None."""
     rec = NCU_TRAFFIC.get((workload, stage))
@@ -313,7 +322,7 @@ def fuse_stages(model):
 def stage_label(dom, fused):
     """fused: moe_forward_fused_gemms (2: the few-token kernel, 1: both GEMMs in one launch)."""
     if fused == 2:
-        return "whole forward, one launch (few-token CUDA-core kernel)"
+        return "whole forward, one launch (few-token kernel)"
     return "gate_up + down grouped GEMMs (one launch)" if fused else f"{dom} grouped GEMM"
 
 
@@ -407,7 +416,7 @@ def measure_workload(cfg, steps, warmup, flush, stream):
             "roofline": {"kernel": stage_label(dom, fused), "bound": "tensor" if tensor else "hbm",
                          "achieved": achieved, "unit": "TFLOP/s" if tensor else "GB/s", "peak": peak,
                          "frac": achieved / peak, "peak_source": f"{pk_src} (burst)",
-                         "traffic": ncu_traffic(cfg.name, dom)},
+                         "traffic": ncu_traffic(cfg.name, dom) if default_kernels() else None},
             "layer": {"tensor_frac": lf / (ms / 1e3) / 1e12 / pk["bf16_tflops"],
                       "hbm_frac": lb / (ms / 1e3) / 1e9 / pk["hbm_gbs"], "distinct_experts": distinct,
                       "rows_per_expert_max": int(rows.max()), "empty_experts": int((rows == 0).sum())},
@@ -657,7 +666,7 @@ def run_own(args, cfg):
                 "unit": unit, "frac": achieved / peak, "peak_source": f"{pk_src} (burst)",
                 "frac_vs_sustained_peak": (achieved / sustained) if sustained else None,
                 # the figures belong to the kernels the library picks by itself
-                "traffic": None if os.environ.get("MOE_B200_PAIR_GEMM") else ncu_traffic(cfg.name, dom),
+                "traffic": ncu_traffic(cfg.name, dom) if default_kernels() else None,
                 "kernel_sources": traffic_kernel_sources(cfg.name, dom) or kernel_sources_hash(),
                 "algorithmic_per_launch": m["flops"] if bound == "tensor" else m["bytes"],
                 "kernel_ms": dom_ms,

@@ -83,3 +83,15 @@ def test_kernel_hash_covers_included_headers_only():
         h.update(os.path.basename(f).encode())
         h.update(bench._code_of(open(f, "rb").read()))
     assert bench.kernel_sources_hash("gemm_tcs.cu") == h.hexdigest()[:12]
+
+
+def test_traffic_only_for_the_default_kernels(monkeypatch):
+    """An environment variable that overrides the kernel choice detaches the stored ncu
+    traffic figures (they were captured with the library's own choice)."""
+    import bench
+    assert bench.default_kernels()
+    for v in bench.KERNEL_CHOICE_VARS:
+        monkeypatch.setenv(v, "1")
+        assert not bench.default_kernels()
+        monkeypatch.delenv(v)
+    assert bench.default_kernels()
