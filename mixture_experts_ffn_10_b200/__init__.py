@@ -84,6 +84,16 @@ def _bind(lib: C.CDLL) -> C.CDLL:
     lib.moe_noalloc_debug_status.restype = C.c_int
     lib.moe_noalloc_workspace_bytes.argtypes = []
     lib.moe_noalloc_workspace_bytes.restype = C.c_size_t
+    lib.moe_permute.argtypes = [_P(moe_shape), _P(moe_options), C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_size_t,
+                                C.c_void_p]
+    lib.moe_permute.restype = C.c_int
+    lib.moe_experts_forward.argtypes = [_P(moe_shape), _P(moe_options), _P(moe_tensors), C.c_void_p, C.c_void_p,
+                                        C.c_void_p, C.c_size_t, C.c_void_p]
+    lib.moe_experts_forward.restype = C.c_int
+    lib.moe_combine.argtypes = [_P(moe_shape), C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p,
+                                C.c_void_p]
+    lib.moe_combine.restype = C.c_int
     lib.moe_forward_kernel_count.argtypes = [_P(moe_shape), _P(moe_options)]
     lib.moe_forward_kernel_count.restype = C.c_int
     lib.moe_forward_split_k.argtypes = [_P(moe_shape), _P(moe_options), _P(C.c_int), _P(C.c_int)]
@@ -128,7 +138,8 @@ _lib = _UnbuiltLibrary()
 EXPORTED = ("moe_options_init", "moe_workspace_size", "moe_forward", "moe_route",
             "moe_forward_events", "moe_forward_noalloc", "moe_noalloc_debug_status",
             "moe_noalloc_workspace_bytes", "moe_forward_kernel_count", "moe_forward_split_k",
-            "moe_forward_fused_gemms", "moe_last_error", "moe_debug_status", "moe_version")
+            "moe_forward_fused_gemms", "moe_last_error", "moe_debug_status", "moe_version",
+            "moe_permute", "moe_experts_forward", "moe_combine")
 
 
 class MoeError(RuntimeError):
@@ -179,6 +190,23 @@ def moe_noalloc_debug_status(stream: int) -> int:
 def moe_noalloc_workspace_bytes() -> int:
     """Size of the library's static scratch array (read from the library)."""
     return _lib.moe_noalloc_workspace_bytes()
+
+
+def moe_permute(shape, opts, idx: int, w: int, x: int, x_perm: int, row_expert: int, row_w: int,
+                expert_counts: int, pos: int, experts_per_rank: int, workspace: int, workspace_bytes: int,
+                stream: int) -> int:
+    return _lib.moe_permute(C.byref(shape), C.byref(opts), idx, w, x, x_perm, row_expert, row_w, expert_counts,
+                            pos, experts_per_rank, workspace, workspace_bytes, stream)
+
+
+def moe_experts_forward(shape, opts, tensors, row_expert: int, row_w: int, workspace: int,
+                        workspace_bytes: int, stream: int) -> int:
+    return _lib.moe_experts_forward(C.byref(shape), C.byref(opts), C.byref(tensors), row_expert, row_w,
+                                    workspace, workspace_bytes, stream)
+
+
+def moe_combine(shape, pos: int, Y: int, rows: int, shared_output: int, y: int, stream: int) -> int:
+    return _lib.moe_combine(C.byref(shape), pos, Y, rows, shared_output, y, stream)
 
 
 def moe_forward_kernel_count(shape, opts) -> int:

@@ -22,7 +22,8 @@ def _sources():
 
 def _headers():
     inc = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
-    return inc + [os.path.join(HERE, "..", "include", "moe.h")]
+    pub = os.path.join(HERE, "..", "include")
+    return inc + [os.path.join(pub, f) for f in os.listdir(pub) if f.endswith(".h")]
 
 
 def _stale(target, deps):

@@ -19,6 +19,8 @@
 #include <string>
 
 #include "common.cuh"
+#include "ep.cuh"
+#include "moe_ep.h"
 #include "gemv.cuh"
 
 namespace moe {
@@ -92,10 +94,13 @@ int check_shape_opts(const moe_shape* s, const moe_options* o) {
   return MOE_OK;
 }
 
-int check_tensors(const moe_shape* s, const moe_options* o, const moe_tensors* t, bool full) {
+// routed: the rows come with their expert (moe_experts_forward), no router input.
+int check_tensors(const moe_shape* s, const moe_options* o, const moe_tensors* t, bool full, bool routed = false) {
   if (!t) return fail(MOE_ERR_NULL, "tensors must not be NULL");
   if (s->T == 0) return MOE_OK;  // nothing is read or written (empty tensors may have NULL data)
-  if (!t->router_logits && !t->router_weight)
+  if (routed && (t->router_logits || t->router_weight || t->topk_idx || t->topk_w || t->logits_out))
+    return fail(MOE_ERR_ARG, "rows with their experts take no router input and give no topk outputs");
+  if (!routed && !t->router_logits && !t->router_weight)
     return fail(MOE_ERR_NULL, "router_logits or router_weight is required");
   if (t->router_logits && t->router_weight)
     return fail(MOE_ERR_ARG, "give router_logits or router_weight, not both");
@@ -162,11 +167,14 @@ int cuda_fail(cudaError_t e, const char* what) {
   return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+// pre_idx / pre_w: each row's expert and weight given ([T] with k = 1: the rows an
+// expert-parallel exchange delivered); the routing kernel is then not launched.
 int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws, size_t ws_bytes,
-        void* stream, bool full, void* const* events = nullptr, int n_events = 0) {
+        void* stream, bool full, void* const* events = nullptr, int n_events = 0, const int32_t* pre_idx = nullptr,
+        const float* pre_w = nullptr) {
   int rc = check_shape_opts(s, o);
   if (rc) return rc;
-  rc = check_tensors(s, o, t, full);
+  rc = check_tensors(s, o, t, full, pre_idx != nullptr);
   if (rc) return rc;
   Plan p;
   const size_t need = make_plan(s, o, &p);
@@ -221,10 +229,20 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
 
   // A few tokens: the whole forward in one launch, after the router GEMM when the layer
   // computes the logits.  Stage events 1-3 precede the launch and 4-6 follow it.
+  if (pre_idx) {
+    ra.idx = const_cast<int32_t*>(pre_idx);  // read only: no routing kernel runs
+    ra.w = const_cast<float*>(pre_w);
+    ra.idx_user = nullptr;
+    ra.w_user = nullptr;
+  }
   if (gp.on) {
     GemvArgs ga{};
     ga.ra = ra;
-    if (t->router_weight) {
+    if (pre_idx) {
+      ga.pre_routed = 1;
+      ga.idx = pre_idx;
+      ga.w = pre_w;
+    } else if (t->router_weight) {
       if ((e = launch_router(ra, st)) != cudaSuccess) return cuda_fail(e, "router kernel");
       ga.pre_routed = 1;
       ga.idx = ra.idx;
@@ -276,7 +294,7 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
     cudaGetLastError();
   }
 
-  if ((e = t->router_weight ? launch_router(ra, st) : launch_route(ra, st)) != cudaSuccess)
+  if (!pre_idx && (e = t->router_weight ? launch_router(ra, st) : launch_route(ra, st)) != cudaSuccess)
     return cuda_fail(e, "route kernel");
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   if (!full) return MOE_OK;
@@ -461,6 +479,91 @@ int run(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws
   if ((e = launch_combine(ca, st)) != cudaSuccess) return cuda_fail(e, "combine kernel");
   if ((e = mark(6)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   return MOE_OK;
+}
+
+// moe_permute: the sort of the given routing, the gather of x into expert order (no
+// scaling), each row's expert (modulo experts_per_rank), and copies of the counts, the
+// slot positions and the row weights to the caller's buffers.
+int permute(const moe_shape* s, const moe_options* o, const int32_t* idx, const float* w, const void* x, void* x_perm,
+            int32_t* row_expert, float* row_w, int32_t* expert_counts, int32_t* pos, int experts_per_rank, void* ws,
+            size_t ws_bytes, void* stream) {
+  int rc = check_shape_opts(s, o);
+  if (rc) return rc;
+  if (experts_per_rank < 0 || (experts_per_rank > 0 && s->E % experts_per_rank))
+    return fail(MOE_ERR_ARG, "experts_per_rank must divide E (or be 0)");
+  if (s->T == 0) return MOE_OK;
+  if (!idx || !w || !x || !x_perm || !row_expert || !row_w || !expert_counts || !pos)
+    return fail(MOE_ERR_NULL, "idx, w, x, x_perm, row_expert, row_w, expert_counts and pos are required");
+  if (!aligned16(x) || !aligned16(x_perm)) return fail(MOE_ERR_ALIGN, "x and x_perm must be 16-byte aligned");
+  Plan p;
+  const size_t need = make_plan(s, o, &p);
+  if (!ws || ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = at<int>(ws, p.o_status);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  SortArgs sa{};
+  sa.idx = idx;
+  sa.w = w;
+  sa.T = (int)p.T;
+  sa.k = (int)p.k;
+  sa.E = (int)p.E;
+  sa.NS = (int)p.NS;
+  sa.nchunks = (int)p.nchunks;
+  sa.R = (int)p.R;
+  sa.shared_rows = p.Fs > 0 ? (int)p.T : 0;
+  sa.hist = at<int32_t>(ws, p.o_hist);
+  sa.cnt = at<int32_t>(ws, p.o_cnt);
+  sa.off = at<int32_t>(ws, p.o_off);
+  sa.tile_gu = at<int32_t>(ws, p.o_tgu);
+  sa.tile_dn = at<int32_t>(ws, p.o_tdn);
+  sa.order = nullptr;
+  sa.bm = p.bm;
+  sa.nt_gu_routed = p.nt_gu_routed;
+  sa.nt_gu_shared = p.nt_gu_shared;
+  sa.nt_dn_routed = p.nt_dn_routed;
+  sa.nt_dn_shared = p.nt_dn_shared;
+  sa.pos = at<int32_t>(ws, p.o_pos);
+  sa.perm = at<int32_t>(ws, p.o_perm);
+  sa.roww = at<float>(ws, p.o_roww);
+  sa.sync = at<int32_t>(ws, p.o_sync);
+  sa.n_sync = (int)p.n_sync;
+  sa.status = status;
+  if ((e = launch_sort(sa, st)) != cudaSuccess) return cuda_fail(e, "sort kernels");
+  GatherArgs ga{x, sa.pos, sa.roww, x_perm, (int)p.R, (int)p.d, (int)p.T, (int)p.k, s->act_dtype == MOE_BF16, 0,
+                status};
+  if ((e = launch_gather(ga, st)) != cudaSuccess) return cuda_fail(e, "gather kernel");
+  if ((e = launch_row_expert(sa.off, (int)p.E, (int)p.R, experts_per_rank, row_expert, st)) != cudaSuccess)
+    return cuda_fail(e, "row expert kernel");
+  const struct {
+    void* dst;
+    const void* src;
+    size_t bytes;
+  } copies[3] = {{expert_counts, sa.cnt, (size_t)p.E * 4}, {pos, sa.pos, (size_t)p.R * 4}, {row_w, sa.roww, (size_t)p.R * 4}};
+  for (const auto& c : copies)
+    if ((e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyDeviceToDevice, st)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemcpyAsync");
+  return MOE_OK;
+}
+
+// moe_combine: the combine kernel on caller buffers.
+int combine(const moe_shape* s, const int32_t* pos, const void* Y, int64_t rows, const void* shared_output, void* y,
+            void* stream) {
+  if (!s) return fail(MOE_ERR_NULL, "shape must not be NULL");
+  if (s->act_dtype != MOE_F32 && s->act_dtype != MOE_BF16) return fail(MOE_ERR_DTYPE, "act_dtype %d", s->act_dtype);
+  if (s->T < 0 || s->k < 1 || s->d < 8 || s->d % 8 || rows < 0 || rows >= (1ll << 31) || s->T * s->k >= (1ll << 31))
+    return fail(MOE_ERR_SHAPE, "need T >= 0, k >= 1, d >= 8 a multiple of 8, 0 <= rows < 2^31");
+  if (s->T == 0) return MOE_OK;
+  if (!pos || !Y || !y) return fail(MOE_ERR_NULL, "pos, Y and y are required");
+  if (!aligned16(Y) || !aligned16(y) || (shared_output && !aligned16(shared_output)))
+    return fail(MOE_ERR_ALIGN, "Y, y and shared_output must be 16-byte aligned");
+  if (y == Y || (shared_output && y == shared_output)) return fail(MOE_ERR_ARG, "y must not alias an input");
+  CombineArgs ca{Y, pos, nullptr, shared_output, y, (int)s->T, (int)s->d, (int)s->k, (int)rows, 0,
+                 s->act_dtype == MOE_BF16, nullptr};
+  const cudaError_t e = launch_combine(ca, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "combine kernel");
 }
 
 }  // namespace
@@ -701,6 +804,27 @@ int moe_route(const moe_shape* s, const moe_options* o, const moe_tensors* t, vo
 int moe_forward_events(const moe_shape* s, const moe_options* o, const moe_tensors* t, void* ws, size_t ws_bytes,
                        void* stream, void* const* events, int n_events) {
   return moe::run(s, o, t, ws, ws_bytes, stream, true, events, n_events);
+}
+
+int moe_permute(const moe_shape* s, const moe_options* o, const int32_t* idx, const float* w, const void* x,
+                void* x_perm, int32_t* row_expert, float* row_w, int32_t* expert_counts, int32_t* pos,
+                int experts_per_rank, void* ws, size_t ws_bytes, void* stream) {
+  return moe::permute(s, o, idx, w, x, x_perm, row_expert, row_w, expert_counts, pos, experts_per_rank, ws, ws_bytes,
+                      stream);
+}
+
+int moe_experts_forward(const moe_shape* s, const moe_options* o, const moe_tensors* t, const int32_t* row_expert,
+                        const float* row_w, void* ws, size_t ws_bytes, void* stream) {
+  if (!s || !o) return moe::fail(MOE_ERR_NULL, "shape and options must not be NULL");
+  if (s->k != 1) return moe::fail(MOE_ERR_SHAPE, "moe_experts_forward takes one expert per row (k = 1)");
+  if (s->Fs != 0 || o->shared_gate) return moe::fail(MOE_ERR_UNSUPPORTED, "moe_experts_forward runs routed experts only");
+  if (s->T > 0 && (!row_expert || !row_w)) return moe::fail(MOE_ERR_NULL, "row_expert and row_w are required");
+  return moe::run(s, o, t, ws, ws_bytes, stream, true, nullptr, 0, row_expert, row_w);
+}
+
+int moe_combine(const moe_shape* s, const int32_t* pos, const void* Y, int64_t rows, const void* shared_output,
+                void* y, void* stream) {
+  return moe::combine(s, pos, Y, rows, shared_output, y, stream);
 }
 
 int moe_forward_kernel_count(const moe_shape* s, const moe_options* o) {

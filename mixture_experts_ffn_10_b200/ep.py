@@ -1,0 +1,149 @@
+"""Expert parallelism over a torch.distributed process group.
+
+Each of the W ranks holds its own tokens and E / W of the experts: rank g holds
+experts [g E/W, (g+1) E/W) (graph-op page "MoE": experts partitioned over devices,
+each running the experts it holds on the rows routed to them).  One forward, on every
+rank:
+
+  1. route the rank's tokens (moe_route)                        -> idx, w [T, k]
+  2. moe_permute: the routed rows in expert order, each row's expert as an index on
+     the rank holding it, rows per expert, and the row of every slot (pos)
+  3. rows for rank g = the rows of its experts (contiguous in expert order); the
+     counts go to every rank (all-to-all of W integers)
+  4. all-to-all of the rows, their experts and their routing weights
+  5. moe_experts_forward on the rows received: this rank's experts
+  6. all-to-all of the outputs back, with the splits of step 4 reversed
+  7. moe_combine of the outputs in slot order (+ shared_output)        -> y
+
+Every step on the data runs in the library's kernels (``LibraryOps``); this module
+only sizes the exchange (one host copy of the E per-expert counts per forward) and
+calls the collectives.  With one rank the exchange is a copy and the result equals
+moe_forward up to the order of its fp32 sums.
+"""
+from __future__ import annotations
+
+import types
+
+
+def _with(cfg, **kw):
+    """A copy of a configuration object with some fields replaced."""
+    d = dict(vars(cfg))
+    d.update(kw)
+    return types.SimpleNamespace(**d)
+
+
+class LibraryOps:
+    """The device steps, through the library's C ABI (device tensors on the current stream)."""
+
+    def __init__(self):
+        from . import (Workspace, _check, moe_combine, moe_experts_forward, moe_permute,
+                       moe_workspace_size, options_of, route, shape_of, tensors_of)
+        self._m = types.SimpleNamespace(Workspace=Workspace, check=_check, combine=moe_combine,
+                                        experts_forward=moe_experts_forward, permute=moe_permute,
+                                        workspace_size=moe_workspace_size, options_of=options_of,
+                                        route=route, shape_of=shape_of, tensors_of=tensors_of)
+
+    def _stream(self, t):
+        import torch
+        return torch.cuda.current_stream(t.device).cuda_stream
+
+    def route(self, cfg, inputs):
+        return self._m.route(cfg, inputs)
+
+    def permute(self, cfg, idx, w, x, experts_per_rank):
+        import torch
+        m = self._m
+        R = cfg.T * cfg.k
+        shape, opts = m.shape_of(cfg), m.options_of(cfg)
+        ws = m.Workspace(m.workspace_size(shape, opts), x.device)
+        x_perm = torch.empty((R, cfg.d), dtype=x.dtype, device=x.device)
+        row_expert = torch.empty(R, dtype=torch.int32, device=x.device)
+        row_w = torch.empty(R, dtype=torch.float32, device=x.device)
+        counts = torch.empty(cfg.E, dtype=torch.int32, device=x.device)
+        pos = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=x.device)
+        m.check(m.permute(shape, opts, idx.data_ptr(), w.data_ptr(), x.data_ptr(), x_perm.data_ptr(),
+                          row_expert.data_ptr(), row_w.data_ptr(), counts.data_ptr(), pos.data_ptr(),
+                          experts_per_rank, ws.ptr, ws.nbytes, self._stream(x)))
+        return x_perm, row_expert, row_w, counts, pos
+
+    def experts_forward(self, cfg_local, rows, row_expert, row_w, weights):
+        import torch
+        m = self._m
+        y = torch.empty_like(rows)
+        if rows.shape[0] == 0:
+            return y
+        shape, opts = m.shape_of(cfg_local), m.options_of(cfg_local)
+        ws = m.Workspace(m.workspace_size(shape, opts), rows.device)
+        tens = m.tensors_of({**weights, "x": rows}, y)
+        m.check(m.experts_forward(shape, opts, tens, row_expert.data_ptr(), row_w.data_ptr(), ws.ptr, ws.nbytes,
+                                  self._stream(rows)))
+        return y
+
+    def combine(self, cfg, pos, Y, shared_output=None):
+        import torch
+        m = self._m
+        y = torch.empty((cfg.T, cfg.d), dtype=Y.dtype, device=Y.device)
+        so = 0 if shared_output is None else shared_output.data_ptr()
+        m.check(m.combine(m.shape_of(cfg), pos.data_ptr(), Y.data_ptr(), Y.shape[0], so, y.data_ptr(),
+                          self._stream(Y)))
+        return y
+
+
+class ExpertParallelMoE:
+    """The MoE layer with its routed experts split over the ranks of ``group``.
+
+    cfg: the layer's configuration (attributes as in moe_shape / moe_options; cfg.T is
+    this rank's token count, cfg.E the total number of experts, Fs must be 0: a shared
+    expert is computed by the caller and passed as shared_output).  local: this rank's
+    expert tensors, gate_up / down (and their biases, gate / gate_bias for an unfused
+    stack) of its E / W experts, plus router_bias / selection_bias for the routing.
+    """
+
+    def __init__(self, cfg, local: dict, group=None, ops=None):
+        import torch.distributed as dist
+        self.dist = dist
+        self.group = group
+        self.world = dist.get_world_size(group) if dist.is_initialized() else 1
+        self.rank = dist.get_rank(group) if dist.is_initialized() else 0
+        if cfg.E % self.world:
+            raise ValueError(f"E={cfg.E} experts do not split over {self.world} ranks")
+        if cfg.Fs:
+            raise ValueError("a shared expert is not split: compute it apart and pass shared_output")
+        self.cfg = cfg
+        self.local = local
+        self.ops = ops if ops is not None else LibraryOps()
+        self.per_rank = cfg.E // self.world
+
+    def _a2a(self, out, inp, out_splits, in_splits):
+        if self.world == 1:
+            out.copy_(inp)
+        else:
+            self.dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
+
+    def forward(self, x, logits, shared_output=None):
+        import torch
+        cfg, ops, W, El = self.cfg, self.ops, self.world, self.per_rank
+        T = x.shape[0]
+        cfg_t = _with(cfg, T=T)
+        inputs = {"x": x, "logits": logits, "router_bias": self.local.get("router_bias"),
+                  "selection_bias": self.local.get("selection_bias")}
+        idx, w = ops.route(cfg_t, inputs)
+        x_perm, row_expert, row_w, counts, pos = ops.permute(cfg_t, idx, w, x, El if W > 1 else 0)
+        per_expert = counts.to("cpu").tolist()
+        send = [sum(per_expert[g * El:(g + 1) * El]) for g in range(W)]
+        send_t = torch.tensor(send, dtype=torch.int64, device=x.device)
+        recv_t = torch.empty_like(send_t)
+        self._a2a(recv_t, send_t, [1] * W, [1] * W)
+        recv = recv_t.to("cpu").tolist()
+        rows = sum(recv)
+        x_recv = torch.empty((rows, cfg.d), dtype=x.dtype, device=x.device)
+        e_recv = torch.empty(rows, dtype=torch.int32, device=x.device)
+        w_recv = torch.empty(rows, dtype=torch.float32, device=x.device)
+        self._a2a(x_recv, x_perm, recv, send)
+        self._a2a(e_recv, row_expert, recv, send)
+        self._a2a(w_recv, row_w, recv, send)
+        cfg_local = _with(cfg, T=rows, E=El, k=1, Fs=0, shared_gate=False)
+        y_recv = ops.experts_forward(cfg_local, x_recv, e_recv, w_recv, self.local)
+        Y = torch.empty((x_perm.shape[0], cfg.d), dtype=y_recv.dtype, device=y_recv.device)
+        self._a2a(Y, y_recv, send, recv)
+        return ops.combine(cfg_t, pos, Y, shared_output)

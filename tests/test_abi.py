@@ -18,8 +18,10 @@ def moe():
 
 
 def _declared():
-    with open(os.path.join(ROOT, "include", "moe.h")) as f:
-        src = f.read()
+    src = ""
+    for h in ("moe.h", "moe_ep.h"):
+        with open(os.path.join(ROOT, "include", h)) as f:
+            src += f.read()
     return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(", src)))
 
 
@@ -29,7 +31,7 @@ def test_header_declares_the_entry_points():
                                   "moe_noalloc_debug_status", "moe_noalloc_workspace_bytes",
                                   "moe_forward_kernel_count", "moe_forward_split_k",
                                   "moe_forward_fused_gemms", "moe_last_error", "moe_debug_status",
-                                  "moe_version"])
+                                  "moe_version", "moe_permute", "moe_experts_forward", "moe_combine"])
 
 
 def test_static_scratch_size_matches_the_header(moe):
@@ -253,3 +255,43 @@ def test_split_k_choice_follows_the_cost_model(moe):
     assert moe.moe_forward_kernel_count(f32, o) == 6
     with pytest.raises(moe.MoeError):
         moe.moe_forward_split_k(moe.make_shape(T=1, d=4096, F=1024, E=8, k=0), o)
+
+
+def test_expert_parallel_entry_points_validate_before_launch(moe):
+    """moe_permute, moe_experts_forward and moe_combine reject bad arguments on the host
+    (no device work): experts_per_rank must divide E; rows arriving with their expert
+    take k = 1, no shared expert and no router inputs; moe_combine checks its shape."""
+    s, o = _valid(moe), moe.make_options()
+    need = moe.moe_workspace_size(s, o)
+    args = [FAKE] * 8
+    assert moe.moe_permute(s, o, *args, 3, FAKE, need, None) == moe.MOE_ERR_ARG  # E = 8
+    assert moe.moe_permute(s, o, *args, -1, FAKE, need, None) == moe.MOE_ERR_ARG
+    bad = list(args)
+    bad[2] = None  # x
+    assert moe.moe_permute(s, o, *bad, 4, FAKE, need, None) == moe.MOE_ERR_NULL
+    bad = list(args)
+    bad[3] = FAKE + 8  # x_perm misaligned
+    assert moe.moe_permute(s, o, *bad, 4, FAKE, need, None) == moe.MOE_ERR_ALIGN
+    assert moe.moe_permute(s, o, *args, 4, FAKE, need - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert moe.moe_permute(_valid(moe, T=0), o, *args, 4, FAKE, need, None) == moe.MOE_OK
+
+    t = _tensors(moe)
+    t.router_logits = None
+    t.y = 2 * FAKE
+    s1 = _valid(moe, k=1)
+    need1 = moe.moe_workspace_size(s1, o)
+    assert moe.moe_experts_forward(s, o, t, FAKE, FAKE, FAKE, need, None) == moe.MOE_ERR_SHAPE  # k = 2
+    assert moe.moe_experts_forward(_valid(moe, k=1, Fs=64), o, t, FAKE, FAKE, FAKE, need1, None) == \
+        moe.MOE_ERR_UNSUPPORTED
+    assert moe.moe_experts_forward(s1, o, t, None, FAKE, FAKE, need1, None) == moe.MOE_ERR_NULL
+    t.router_logits = FAKE
+    assert moe.moe_experts_forward(s1, o, t, FAKE, FAKE, FAKE, need1, None) == moe.MOE_ERR_ARG
+    t.router_logits = None
+    t.topk_idx = FAKE
+    assert moe.moe_experts_forward(s1, o, t, FAKE, FAKE, FAKE, need1, None) == moe.MOE_ERR_ARG
+
+    assert moe.moe_combine(s, FAKE, FAKE, -1, None, 2 * FAKE, None) == moe.MOE_ERR_SHAPE
+    assert moe.moe_combine(s, None, FAKE, 16, None, 2 * FAKE, None) == moe.MOE_ERR_NULL
+    assert moe.moe_combine(s, FAKE, FAKE, 16, None, FAKE, None) == moe.MOE_ERR_ARG  # y aliases Y
+    assert moe.moe_combine(s, FAKE, FAKE + 8, 16, None, 2 * FAKE, None) == moe.MOE_ERR_ALIGN
+    assert moe.moe_combine(_valid(moe, T=0), FAKE, FAKE, 16, None, 2 * FAKE, None) == moe.MOE_OK
