@@ -744,6 +744,90 @@ def run_own(args, cfg):
     return 0
 
 
+def run_ep(args, cfg):
+    """The expert-parallel layer (mixture_experts_ffn_10_b200.ep), timed eagerly: every rank
+    holds cfg.T tokens of its own and E / N experts; a step is one forward of the layer --
+    routing, permute, the all-to-all of the rows, the rank's experts, the all-to-all back,
+    the combine -- with its host copy of the split sizes and its collectives, between CUDA
+    events on the rank's stream, L2 flushed before it; max over ranks.  At N = 1 the
+    exchange is a copy and the line also times moe_forward on the same tokens."""
+    import torch
+
+    import mixture_experts_ffn_10_b200 as moe
+    from mixture_experts_ffn_10_b200.ep import ExpertParallelMoE
+    from workloads import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    if cfg.E % world or cfg.Fs:
+        raise SystemExit(f"--ep needs E divisible by {world} and no shared expert ({cfg.name})")
+    inputs = make_inputs(cfg, "cuda")
+    El = cfg.E // world
+    keep = ("gate_up", "gate_up_scales", "gate_up_bias", "down", "down_scales", "down_bias", "gate", "gate_scales",
+            "gate_bias")
+    mine = {k: (v[rank * El:(rank + 1) * El].clone() if v is not None else None) for k, v in inputs.items()
+            if k in keep}
+    mine["router_bias"], mine["selection_bias"] = inputs.get("router_bias"), inputs.get("selection_bias")
+    layer = ExpertParallelMoE(cfg, mine, group=None)
+    flush = L2Flush(torch)
+    torch.cuda.synchronize()
+
+    def timed(fn, steps):
+        ts = []
+        for _ in range(steps):
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return ts
+
+    def ep_step():
+        layer.forward(inputs["x"], inputs["logits"])
+
+    sampler = ClockSampler(physical_gpu_index(local))
+    timed(ep_step, args.warmup)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ts = timed(ep_step, args.steps)
+    clocks = sampler.stop()
+    total = max_over_ranks(sum(ts), dist, "cuda")
+    out = {"metric": METRIC, "value": whole_job_throughput(world, cfg.T, args.steps, total), "unit": "tokens/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": cfg.act_dtype if cfg.w_dtype != "mxfp4" else "bf16 (mxfp4 weights)",
+           "data": "synthetic (seeded; random-init weights)",
+           "config": config_dict(cfg, {"parallelism": f"expert-parallel x{world}", "experts_per_rank": El,
+                                       "launch": "eager layer forwards (host split sizes each step)"}),
+           "clocks": clocks}
+    if world == 1:
+        y = torch.empty_like(inputs["x"])
+
+        def fwd_step():
+            moe.forward(cfg, inputs, y=y)
+
+        timed(fwd_step, args.warmup)
+        out["moe_forward_ms_per_step"] = statistics.median(timed(fwd_step, args.steps))
+        out["ep_ms_per_step_median"] = statistics.median(ts)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -758,6 +842,8 @@ def main():
     ap.add_argument("--other-steps", type=int, default=10, help="timed steps per other workload")
     ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of a CUDA graph replay")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle wall time")
+    ap.add_argument("--ep", action="store_true",
+                    help="time the expert-parallel layer (experts split over the N ranks) instead")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a workload field (profiling / sweeps), e.g. --set T=1024")
     args = ap.parse_args()
@@ -775,6 +861,8 @@ def main():
         cfg = small(cfg, name=cfg.name + "[" + ",".join(args.set) + "]")
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if args.ep:
+        return run_ep(args, cfg)
     return run_own(args, cfg)
 
 

@@ -16,9 +16,10 @@ rank:
   7. moe_combine of the outputs in slot order (+ shared_output)        -> y
 
 Every step on the data runs in the library's kernels (``LibraryOps``); this module
-only sizes the exchange (one host copy of the E per-expert counts per forward) and
-calls the collectives.  With one rank the exchange is a copy and the result equals
-moe_forward up to the order of its fp32 sums.
+only sizes the exchange (one host copy of the E per-expert counts per forward, and one
+of the W counts received) and calls the collectives.  With one rank the exchange is a
+copy, nothing waits on the host, and the result equals moe_forward up to the order of
+its fp32 sums.
 """
 from __future__ import annotations
 
@@ -129,12 +130,15 @@ class ExpertParallelMoE:
                   "selection_bias": self.local.get("selection_bias")}
         idx, w = ops.route(cfg_t, inputs)
         x_perm, row_expert, row_w, counts, pos = ops.permute(cfg_t, idx, w, x, El if W > 1 else 0)
-        per_expert = counts.to("cpu").tolist()
-        send = [sum(per_expert[g * El:(g + 1) * El]) for g in range(W)]
-        send_t = torch.tensor(send, dtype=torch.int64, device=x.device)
-        recv_t = torch.empty_like(send_t)
-        self._a2a(recv_t, send_t, [1] * W, [1] * W)
-        recv = recv_t.to("cpu").tolist()
+        if W == 1:  # every row stays: no split sizes to learn (and no host synchronisation)
+            send = recv = [T * cfg.k]
+        else:
+            per_expert = counts.to("cpu").tolist()
+            send = [sum(per_expert[g * El:(g + 1) * El]) for g in range(W)]
+            send_t = torch.tensor(send, dtype=torch.int64, device=x.device)
+            recv_t = torch.empty_like(send_t)
+            self._a2a(recv_t, send_t, [1] * W, [1] * W)
+            recv = recv_t.to("cpu").tolist()
         rows = sum(recv)
         x_recv = torch.empty((rows, cfg.d), dtype=x.dtype, device=x.device)
         e_recv = torch.empty(rows, dtype=torch.int32, device=x.device)
