@@ -100,7 +100,10 @@ class ExpertParallelMoE:
     stack) of its E / W experts, plus router_bias / selection_bias for the routing.
     """
 
-    def __init__(self, cfg, local: dict, group=None, ops=None):
+    def __init__(self, cfg, local: dict, group=None, ops=None, host_exchange=None):
+        """host_exchange: stage the exchanged tensors through host memory (for a backend
+        without device collectives, such as gloo); default: when the group's backend is
+        gloo."""
         import torch.distributed as dist
         self.dist = dist
         self.group = group
@@ -114,10 +117,17 @@ class ExpertParallelMoE:
         self.local = local
         self.ops = ops if ops is not None else LibraryOps()
         self.per_rank = cfg.E // self.world
+        if host_exchange is None:
+            host_exchange = self.world > 1 and dist.get_backend(group) == "gloo"
+        self.host_exchange = host_exchange
 
     def _a2a(self, out, inp, out_splits, in_splits):
         if self.world == 1:
             out.copy_(inp)
+        elif self.host_exchange and out.device.type != "cpu":
+            o = out.new_empty(out.shape, device="cpu")
+            self.dist.all_to_all_single(o, inp.to("cpu"), out_splits, in_splits, group=self.group)
+            out.copy_(o)
         else:
             self.dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
 
