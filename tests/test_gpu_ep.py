@@ -24,6 +24,8 @@ CASES = {
     "plain_relu": small(DEC, name="ep_plain", ffn="plain", act="relu", expert_bias=True),
     "fp32": small(CONFIGS["tiny_fp32"], name="ep_fp32", Fs=0),
     "mxfp4": small(CONFIGS["gptoss_mxfp4"], name="ep_mxfp4", T=100, d=320, F=352, E=8, k=4),
+    # 64 routed rows: the expert forward reads its rows in place (one launch for both GEMMs)
+    "rows_in_place": small(DEC, name="ep_in_place", T=16),
 }
 
 
@@ -53,13 +55,13 @@ def test_permute_is_the_stable_expert_sort(per_rank):
     assert torch.equal(x_perm.cpu(), inputs["x"].cpu()[torch.from_numpy(order // cfg.k)])
 
 
+@pytest.mark.parametrize("rows", [50, 70])
 @pytest.mark.parametrize("name", ["decode_small", "unfused_bias_weigh_inputs", "plain_relu", "fp32", "mxfp4"])
-def test_experts_forward_matches_the_oracle_row_by_row(name):
+def test_experts_forward_matches_the_oracle_row_by_row(name, rows):
     m = _m()
     from mixture_experts_ffn_10_b200.ep import LibraryOps, _with
     cfg = CASES[name]
     inputs = make_inputs(cfg, "cuda")
-    rows = 70
     g = torch.Generator().manual_seed(7)
     row_expert = torch.randint(0, cfg.E, (rows,), generator=g, dtype=torch.int32)
     row_w = torch.rand(rows, generator=g, dtype=torch.float32) + 0.25
