@@ -98,13 +98,25 @@ def _rank_main(rank, world, port, cfg, counts, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,counts,layout", [(2, [7, 5], "concat"), (4, [3, 0, 6, 2], "interleaved")])
-def test_expert_parallel_exchange_matches_one_device(world, counts, layout):
+VARIANTS = {
+    "concat": dict(gu_layout="concat", expert_bias=True),
+    "interleaved": dict(gu_layout="interleaved", expert_bias=True),
+    "unfused_weigh_inputs": dict(gu_layout="unfused", expert_bias=True, weigh_inputs=True),
+    "plain_relu": dict(ffn="plain", act="relu"),
+    "sigmoid_groups_bias": dict(score="sigmoid", n_group=4, topk_group=2, renormalize=True, routed_scale=2.5,
+                                selection_bias_std=0.1, router_bias=True),
+}
+
+
+@pytest.mark.parametrize("world,counts,variant", [
+    (2, [7, 5], "concat"), (4, [3, 0, 6, 2], "interleaved"), (2, [4, 9], "unfused_weigh_inputs"),
+    (2, [6, 6], "plain_relu"), (4, [5, 2, 3, 4], "sigmoid_groups_bias")])
+def test_expert_parallel_exchange_matches_one_device(world, counts, variant):
     sys.path.insert(0, ROOT)
     import oracle
     from workloads import CONFIGS, make_inputs, small
-    cfg = small(CONFIGS["decode_T1"], name="ep_cpu", T=sum(counts), d=64, F=32, E=8, k=3, gu_layout=layout,
-                expert_bias=True, act_dtype="f32", w_dtype="f32", logit_dtype="f32")
+    cfg = small(CONFIGS["decode_T1"], name="ep_cpu", T=sum(counts), d=64, F=32, E=8, k=3,
+                act_dtype="f32", w_dtype="f32", logit_dtype="f32", **VARIANTS[variant])
     with mp.Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, _free_port(), cfg, counts, out), nprocs=world, join=True)
