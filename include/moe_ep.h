@@ -2,8 +2,9 @@
  * moe_ep.h -- expert-parallel building blocks of libmoe_b200 (C ABI).
  *
  * The pieces a layer whose experts are split over devices needs around its exchange
- * of rows (graph-op page "MoE": experts partitioned over devices): the routed rows of
- * a batch in expert order, the expert FFNs of rows that arrive with their expert, and
+ * of rows (the pages define a single-device layer; the split rests on its structure:
+ * given the routing, each expert's rows are independent): the routed rows of a batch
+ * in expert order, the expert FFNs of rows that arrive with their expert, and
  * the combine of expert outputs.  Types, status codes and conventions are those of
  * moe.h; the exchange itself is the caller's (the package's ep module uses NCCL
  * all-to-all through torch.distributed).
@@ -17,9 +18,9 @@
 extern "C" {
 #endif
 
-/* ---- Expert-parallel building blocks (graph-op page "MoE": experts partitioned over
- * devices, each device running the experts it holds on the rows routed to them; the
- * exchange of rows between devices is the caller's, e.g. NCCL all-to-all, as in the
+/* ---- Expert-parallel building blocks (experts split over devices, each device
+ * running the experts it holds on the rows routed to them; the exchange of rows
+ * between devices is the caller's, e.g. NCCL all-to-all, as in the
  * package's ep module).  moe_forward of a problem equals, up to the order of its fp32
  * sums, moe_permute of its routing, moe_experts_forward of the permuted rows (each
  * with its expert and weight) and moe_combine of their outputs.  Routed experts only:

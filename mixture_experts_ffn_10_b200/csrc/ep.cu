@@ -1,7 +1,7 @@
 // ep.cu -- the expert of each routed row, for the expert-parallel exchange: rows in
 // expert order travel to the rank that holds their expert together with its index
-// there ("MoE" graph-op page: experts partitioned over devices exchange the rows routed
-// to them).
+// there (experts split over devices; given the routing, each expert's rows are
+// independent of the others').
 #include "ep.cuh"
 
 namespace moe {

@@ -1,8 +1,9 @@
 """Expert parallelism over a torch.distributed process group.
 
 Each of the W ranks holds its own tokens and E / W of the experts: rank g holds
-experts [g E/W, (g+1) E/W) (graph-op page "MoE": experts partitioned over devices,
-each running the experts it holds on the rows routed to them).  One forward, on every
+experts [g E/W, (g+1) E/W) and runs them on the rows routed to them from every rank.
+The pages define a single-device layer; this split rests only on its structure: given
+the routing, every expert's rows are independent of the others'.  One forward, on every
 rank:
 
   1. route the rank's tokens (moe_route)                        -> idx, w [T, k]
