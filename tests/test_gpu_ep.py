@@ -58,7 +58,6 @@ def test_permute_is_the_stable_expert_sort(per_rank):
 @pytest.mark.parametrize("rows", [50, 70])
 @pytest.mark.parametrize("name", ["decode_small", "unfused_bias_weigh_inputs", "plain_relu", "fp32", "mxfp4"])
 def test_experts_forward_matches_the_oracle_row_by_row(name, rows):
-    m = _m()
     from mixture_experts_ffn_10_b200.ep import LibraryOps, _with
     cfg = CASES[name]
     inputs = make_inputs(cfg, "cuda")
@@ -79,7 +78,6 @@ def test_experts_forward_matches_the_oracle_row_by_row(name, rows):
 
 
 def test_combine_sums_in_slot_order():
-    m = _m()
     from mixture_experts_ffn_10_b200.ep import LibraryOps
     cfg = CASES["decode_small"]
     g = torch.Generator().manual_seed(3)
