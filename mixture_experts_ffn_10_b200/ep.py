@@ -98,7 +98,9 @@ class ExpertParallelMoE:
     this rank's token count, cfg.E the total number of experts, Fs must be 0: a shared
     expert is computed by the caller and passed as shared_output).  local: this rank's
     expert tensors, gate_up / down (and their biases, gate / gate_bias for an unfused
-    stack) of its E / W experts, plus router_bias / selection_bias for the routing.
+    stack) of its E / W experts, plus router_bias / selection_bias for the routing and,
+    to route on logits the layer computes (forward without logits), router_weight
+    [d, E].
     """
 
     def __init__(self, cfg, local: dict, group=None, ops=None, host_exchange=None):
@@ -132,13 +134,19 @@ class ExpertParallelMoE:
         else:
             self.dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
 
-    def forward(self, x, logits, shared_output=None):
+    def forward(self, x, logits=None, shared_output=None):
+        """y [T, d] for this rank's tokens x [T, d], routed on logits [T, E] or, when they
+        are not given, on x . router_weight."""
         import torch
         cfg, ops, W, El = self.cfg, self.ops, self.world, self.per_rank
         T = x.shape[0]
         cfg_t = _with(cfg, T=T)
         inputs = {"x": x, "logits": logits, "router_bias": self.local.get("router_bias"),
                   "selection_bias": self.local.get("selection_bias")}
+        if logits is None:
+            if self.local.get("router_weight") is None:
+                raise ValueError("forward needs logits, or router_weight in the rank's tensors")
+            inputs["router_weight"] = self.local["router_weight"]
         idx, w = ops.route(cfg_t, inputs)
         x_perm, row_expert, row_w, counts, pos = ops.permute(cfg_t, idx, w, x, El if W > 1 else 0)
         if W == 1:  # every row stays: no split sizes to learn (and no host synchronisation)

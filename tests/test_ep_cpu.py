@@ -90,9 +90,11 @@ def _rank_main(rank, world, port, cfg, counts, out):
                                                      "gate_bias")}
         local["router_bias"] = inputs.get("router_bias")
         local["selection_bias"] = inputs.get("selection_bias")
+        local["router_weight"] = inputs.get("router_weight")
         mine = small(cfg, T=T)
         layer = ExpertParallelMoE(mine, local, ops=OracleOps(mine, local))
-        y = layer.forward(inputs["x"][t0:t0 + T], inputs["logits"][t0:t0 + T])
+        logits = inputs["logits"][t0:t0 + T] if inputs.get("logits") is not None else None
+        y = layer.forward(inputs["x"][t0:t0 + T], logits)
         out[rank] = y.numpy()
     finally:
         dist.destroy_process_group()
@@ -105,12 +107,13 @@ VARIANTS = {
     "plain_relu": dict(ffn="plain", act="relu"),
     "sigmoid_groups_bias": dict(score="sigmoid", n_group=4, topk_group=2, renormalize=True, routed_scale=2.5,
                                 selection_bias_std=0.1, router_bias=True),
+    "router_weight": dict(router="weight", router_bias=True),
 }
 
 
 @pytest.mark.parametrize("world,counts,variant", [
     (2, [7, 5], "concat"), (4, [3, 0, 6, 2], "interleaved"), (2, [4, 9], "unfused_weigh_inputs"),
-    (2, [6, 6], "plain_relu"), (4, [5, 2, 3, 4], "sigmoid_groups_bias")])
+    (2, [6, 6], "plain_relu"), (4, [5, 2, 3, 4], "sigmoid_groups_bias"), (2, [5, 8], "router_weight")])
 def test_expert_parallel_exchange_matches_one_device(world, counts, variant):
     sys.path.insert(0, ROOT)
     import oracle
