@@ -27,6 +27,10 @@ from __future__ import annotations
 import types
 
 
+# Tensors of the routing step, which the expert forward of routed rows does not take.
+_ROUTER_INPUTS = ("router_weight", "router_logits", "logits", "router_bias", "selection_bias")
+
+
 def _with(cfg, **kw):
     """A copy of a configuration object with some fields replaced."""
     d = dict(vars(cfg))
@@ -76,7 +80,8 @@ class LibraryOps:
             return y
         shape, opts = m.shape_of(cfg_local), m.options_of(cfg_local)
         ws = m.Workspace(m.workspace_size(shape, opts), rows.device)
-        tens = m.tensors_of({**weights, "x": rows}, y)
+        experts = {k: v for k, v in weights.items() if k not in _ROUTER_INPUTS}  # rows come routed
+        tens = m.tensors_of({**experts, "x": rows}, y)
         m.check(m.experts_forward(shape, opts, tens, row_expert.data_ptr(), row_w.data_ptr(), ws.ptr, ws.nbytes,
                                   self._stream(rows)))
         return y

@@ -26,6 +26,8 @@ CASES = {
     "mxfp4": small(CONFIGS["gptoss_mxfp4"], name="ep_mxfp4", T=100, d=320, F=352, E=8, k=4),
     # 64 routed rows: the expert forward reads its rows in place (one launch for both GEMMs)
     "rows_in_place": small(DEC, name="ep_in_place", T=16),
+    # routed on x . router_weight (no logits given)
+    "router_weight": small(DEC, name="ep_router", router="weight", router_bias=True),
 }
 
 
@@ -100,8 +102,8 @@ def test_layer_on_one_rank_matches_oracle_and_forward(name):
     from mixture_experts_ffn_10_b200.ep import ExpertParallelMoE
     cfg = CASES[name]
     inputs = make_inputs(cfg, "cuda")
-    local = {k: v for k, v in inputs.items() if k not in ("x", "logits", "router_weight")}
-    y = ExpertParallelMoE(cfg, local).forward(inputs["x"], inputs["logits"])
+    local = {k: v for k, v in inputs.items() if k not in ("x", "logits")}
+    y = ExpertParallelMoE(cfg, local).forward(inputs["x"], inputs.get("logits"))
     y_ref = m.forward(cfg, inputs)
     torch.cuda.synchronize()
     p = oracle.Problem(cfg, host(inputs))
