@@ -111,6 +111,29 @@ MUTATIONS = [
      ";",
      [("test_single_expert_equals_textbook_ffn",
        dict(act="silu", alpha=1.702, beta=0.0, limit=0.5))]),
+    ("kept weights renormalized with renormalize off (a softmax over the kept experts)",
+     "if (p->renormalize) {",
+     "if (1) {",
+     [("test_softmax_without_renormalize_keeps_at_least_k_over_E", {}), ("test_routing_worked_example", {})]),
+    ("e8m0 exponent bias 126",
+     "return ldexp(1.0, s - 127);",
+     "return ldexp(1.0, s - 126);",
+     [("test_e8m0_table", {})]),
+    ("e2m1 exponent bias 0",
+     "ldexp(1.0 + 0.5 * m, ex - 1)",
+     "ldexp(1.0 + 0.5 * m, ex)",
+     [("test_e2m1_table", {})]),
+    ("groups taken worst first",
+     "outranks(gscore[g], g, gscore[best], best)",
+     "outranks(gscore[best], best, gscore[g], g)",
+     [("test_group_limited_selection_matches_exhaustive_search", dict(sel_std=0.0)),
+      ("test_biased_group_selection_matches_exhaustive_search_on_independent_keys",
+       dict(score="sigmoid"))]),
+    ("sigmoid with the sign of its argument flipped",
+     "static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }",
+     "static double sigmoid(double v) { return 1.0 / (1.0 + exp(v)); }",
+     [("test_softmax_and_sigmoid_scores_match_scipy", {}),
+      ("test_single_expert_equals_textbook_ffn", dict(act="silu", alpha=1.0, beta=0.0, limit=0.0))]),
 ]
 
 
