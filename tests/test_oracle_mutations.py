@@ -134,6 +134,22 @@ MUTATIONS = [
      "static double sigmoid(double v) { return 1.0 / (1.0 + exp(v)); }",
      [("test_softmax_and_sigmoid_scores_match_scipy", {}),
       ("test_single_expert_equals_textbook_ffn", dict(act="silu", alpha=1.0, beta=0.0, limit=0.0))]),
+    ("GELU tanh form with a wrong cubic coefficient",
+     "(g + 0.044715 * g * g * g)));\n    break;",
+     "(g + 0.0447 * g * g * g)));\n    break;",
+     [("test_single_expert_equals_textbook_ffn", dict(act="gelu_tanh", alpha=1.0, beta=0.0, limit=0.0))]),
+    ("GELU erf form with its argument scaled by sqrt(2) instead of 1/sqrt(2)",
+     "a = 0.5 * g * (1.0 + erf(g / sqrt(2.0))); break;",
+     "a = 0.5 * g * (1.0 + erf(g * sqrt(2.0))); break;",
+     [("test_single_expert_equals_textbook_ffn", dict(act="gelu_erf", alpha=1.0, beta=0.5, limit=0.0))]),
+    ("shared expert weighed by the first routed weight",
+     "for (int64_t i = 0; i < d; i++) y[i] += gate * o[i];",
+     "for (int64_t i = 0; i < d; i++) y[i] += gate * w[0] * o[i];",
+     [("test_shared_expert_with_sigmoid_gate", {})]),
+    ("down stack read transposed ([F, d] per expert)",
+     "acc += weight(dn, dns, wdt, ee, d, F, o, f) * h[f];",
+     "acc += weight(dn, dns, wdt, ee, F, d, f, o) * h[f];",
+     [("test_single_expert_equals_textbook_ffn", dict(act="relu", alpha=1.0, beta=0.0, limit=0.0))]),
 ]
 
 
